@@ -1,0 +1,229 @@
+"""ctypes binding of libcf (the C ABI in include/cf.h): argument marshalling only.
+
+Every step of the codec runs in the CUDA kernels behind libcf.  This module
+only converts torch tensors / Python values to the C structs and pointers the
+ABI takes, and raises on a non-OK status.  If libcf.so is missing, loading
+fails loudly; there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcf.so")
+
+CF_OK, CF_E_ARG, CF_E_SHAPE, CF_E_ALIGN, CF_E_STATE, CF_E_NOMEM, CF_E_CUDA, CF_E_NONFINITE, CF_E_TIMEOUT = range(9)
+STATUS_NAMES = {0: "CF_OK", 1: "CF_E_ARG", 2: "CF_E_SHAPE", 3: "CF_E_ALIGN", 4: "CF_E_STATE", 5: "CF_E_NOMEM",
+                6: "CF_E_CUDA", 7: "CF_E_NONFINITE", 8: "CF_E_TIMEOUT"}
+CF_MODE_QUANT, CF_MODE_LOWRANK = 0, 1
+
+EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
+            "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
+            "cf_destroy"]
+
+
+class cf_config(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("bits", ctypes.c_int), ("group", ctypes.c_int),
+                ("sign_scale", ctypes.c_int), ("rank", ctypes.c_int), ("iters", ctypes.c_int)]
+
+
+class cf_shape(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+class cf_slot(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("base", ctypes.c_void_p), ("err", ctypes.c_void_p),
+                ("cache", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("q0", ctypes.c_void_p), ("U", ctypes.c_void_p), ("R", ctypes.c_void_p), ("V", ctypes.c_void_p)]
+
+
+class CfError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcf.so (built by ``python -m activation_residual_compression_02_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libcf.so not built ({_LIB_PATH}); run python -m "
+                              "activation_residual_compression_02_b200.build")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.cf_create.argtypes = [ctypes.POINTER(cf_config), I, ctypes.POINTER(cf_shape), ctypes.POINTER(P)]
+        L.cf_create.restype = I
+        L.cf_workspace_bytes.argtypes = [P]
+        L.cf_workspace_bytes.restype = SZ
+        L.cf_set_workspace.argtypes = [P, P, SZ]
+        L.cf_set_workspace.restype = I
+        L.cf_compress.argtypes = [P, ctypes.POINTER(cf_slot), I, P]
+        L.cf_compress.restype = I
+        L.cf_decompress.argtypes = [P, ctypes.POINTER(cf_slot), I, P]
+        L.cf_decompress.restype = I
+        L.cf_lowrank_workspace_bytes.argtypes = [P, I, I64, I64]
+        L.cf_lowrank_workspace_bytes.restype = SZ
+        PP = ctypes.POINTER(P)
+        L.cf_lowrank.argtypes = [P, I, I64, I64, PP, PP, PP, PP, PP, PP, PP, P]
+        L.cf_lowrank.restype = I
+        L.cf_check.argtypes = [P, P]
+        L.cf_check.restype = I
+        L.cf_payload_bytes.argtypes = [P, I]
+        L.cf_payload_bytes.restype = SZ
+        L.cf_last_error.argtypes = [P]
+        L.cf_last_error.restype = ctypes.c_char_p
+        L.cf_destroy.argtypes = [P]
+        L.cf_destroy.restype = I
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libcf takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libcf takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _parr(ts: Optional[Sequence[Optional[torch.Tensor]]]):
+    if ts is None:
+        return None
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t)
+    return arr
+
+
+class Slot:
+    """Per-slot tensors for one call (any may be None when a call does not use it)."""
+
+    __slots__ = ("x", "base", "err", "cache", "codes", "scales", "q0", "U", "R", "V")
+
+    def __init__(self, x=None, base=None, err=None, cache=None, codes=None, scales=None, q0=None, U=None, R=None,
+                 V=None):
+        self.x, self.base, self.err, self.cache = x, base, err, cache
+        self.codes, self.scales, self.q0, self.U, self.R, self.V = codes, scales, q0, U, R, V
+
+    def to_c(self) -> cf_slot:
+        return cf_slot(*[_ptr(getattr(self, f)) for f in Slot.__slots__])
+
+
+class Context:
+    """A libcf context (``cf_create`` ... ``cf_destroy``)."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], mode: int = CF_MODE_QUANT, bits: int = 2, group: int = 128,
+                 sign_scale: int = 0, rank: int = 16, iters: int = 2):
+        L = lib()
+        self.cfg = cf_config(mode, bits, group, sign_scale, rank, iters)
+        self.shapes = [tuple(int(v) for v in s) for s in shapes]
+        arr = (cf_shape * max(1, len(self.shapes)))(*[cf_shape(r, c) for r, c in self.shapes])
+        h = ctypes.c_void_p()
+        st = L.cf_create(ctypes.byref(self.cfg), len(self.shapes), arr, ctypes.byref(h))
+        if st != CF_OK:
+            raise CfError(st, "cf_create failed")
+        self._h = h
+        self._ws = None
+
+    # -- plumbing -----------------------------------------------------------
+    def _raise(self, st: int, what: str):
+        if st != CF_OK:
+            raise CfError(st, f"{what}: {lib().cf_last_error(self._h).decode()}")
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().cf_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self) -> int:
+        return int(lib().cf_workspace_bytes(self._h))
+
+    def lowrank_workspace_bytes(self, nmat: int, m: int, n: int) -> int:
+        return int(lib().cf_lowrank_workspace_bytes(self._h, nmat, m, n))
+
+    def set_workspace(self, ws: Optional[torch.Tensor]):
+        self._ws = ws
+        st = lib().cf_set_workspace(self._h, _ptr(ws) if ws is not None else None,
+                                    ws.numel() * ws.element_size() if ws is not None else 0)
+        self._raise(st, "cf_set_workspace")
+
+    def payload_bytes(self, slot: int) -> int:
+        return int(lib().cf_payload_bytes(self._h, slot))
+
+    # -- codec calls --------------------------------------------------------
+    def _slots(self, slots: Sequence[Slot]):
+        arr = (cf_slot * max(1, len(slots)))()
+        for i, s in enumerate(slots):
+            arr[i] = s.to_c()
+        return arr
+
+    def compress(self, slots: Sequence[Slot], step: int, stream: Optional[torch.cuda.Stream] = None):
+        self._raise(lib().cf_compress(self._h, self._slots(slots), step, _stream_handle(stream)), "cf_compress")
+
+    def decompress(self, slots: Sequence[Slot], step: int, stream: Optional[torch.cuda.Stream] = None):
+        self._raise(lib().cf_decompress(self._h, self._slots(slots), step, _stream_handle(stream)), "cf_decompress")
+
+    def lowrank(self, A: List[torch.Tensor], Q0: List[torch.Tensor], U: List[torch.Tensor], R: List[torch.Tensor],
+                V: List[torch.Tensor], E: Optional[List[torch.Tensor]] = None, C: Optional[List[torch.Tensor]] = None,
+                stream: Optional[torch.cuda.Stream] = None):
+        nmat = len(A)
+        m, n = (A[0].shape[0], A[0].shape[1]) if nmat else (0, 0)
+        st = lib().cf_lowrank(self._h, nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R), _parr(V), _parr(E),
+                              _parr(C), _stream_handle(stream))
+        self._raise(st, "cf_lowrank")
+
+    def check(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        """Synchronise and return the device status (CF_OK, CF_E_NONFINITE, ...)."""
+        return int(lib().cf_check(self._h, _stream_handle(stream)))
+
+
+def cf_create(shapes, **kw) -> Context:
+    return Context(shapes, **kw)
+
+
+def cf_compress(ctx: Context, slots, step, stream=None):
+    ctx.compress(slots, step, stream)
+
+
+def cf_decompress(ctx: Context, slots, step, stream=None):
+    ctx.decompress(slots, step, stream)
+
+
+def cf_lowrank(ctx: Context, A, Q0, U, R, V, E=None, C=None, stream=None):
+    ctx.lowrank(A, Q0, U, R, V, E, C, stream)
+
+
+def cf_check(ctx: Context, stream=None) -> int:
+    return ctx.check(stream)
+
+
+def cf_payload_bytes(ctx: Context, slot: int) -> int:
+    return ctx.payload_bytes(slot)
+
+
+def cf_destroy(ctx: Context):
+    ctx.close()

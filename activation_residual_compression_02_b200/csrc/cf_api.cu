@@ -1,0 +1,439 @@
+// cf_api.cu -- the libcf C ABI: validation, context, grouped launches.
+//
+// Semantics follow "Accelerating Parallel Diffusion Model Serving with
+// Residual Compression" (arXiv 2507.17511): abstract (send the compressed
+// step-wise residual, keep an error-feedback buffer), reproducibility table
+// "Dataset Splits" row (an uncompressed warmup step initialises the base
+// tensor) and "Pseudocode" row, Algorithm 3 (rank-r subspace iteration).
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+#include <string>
+#include <vector>
+
+#include "cf_internal.h"
+
+struct cf_ctx {
+    cf_config cfg{};
+    std::vector<cf_shape> shapes;
+    uint32_t *d_status = nullptr;
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    bool warm_sender = false;
+    bool warm_receiver = false;
+    int device = 0;
+    std::string err;
+};
+
+namespace {
+
+cf_status fail(cf_ctx *ctx, cf_status st, const char *fmt, ...)
+{
+    if (ctx) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof buf, fmt, ap);
+        va_end(ap);
+        ctx->err = buf;
+    }
+    return st;
+}
+
+cf_status cuda_fail(cf_ctx *ctx, cudaError_t e, const char *what)
+{
+    return fail(ctx, CF_E_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+cf_status validate_config(const cf_config *c, std::string &why)
+{
+    if (c->mode == CF_MODE_QUANT) {
+        if (c->bits != 1 && c->bits != 2 && c->bits != 4) { why = "bits must be 1, 2 or 4"; return CF_E_ARG; }
+        if (!pow2(c->group) || c->group < 8 || c->group > 256) { why = "group must be a power of two in [8, 256]"; return CF_E_ARG; }
+        if (c->sign_scale != 0 && c->sign_scale != 1) { why = "sign_scale must be 0 or 1"; return CF_E_ARG; }
+        return CF_OK;
+    }
+    if (c->mode == CF_MODE_LOWRANK) {
+        if (c->rank < 1 || c->rank > 32) { why = "rank must be in [1, 32]"; return CF_E_ARG; }
+        if (c->iters < 0 || c->iters > 1000) { why = "iters must be in [0, 1000]"; return CF_E_ARG; }
+        return CF_OK;
+    }
+    why = "mode must be CF_MODE_QUANT or CF_MODE_LOWRANK";
+    return CF_E_ARG;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Low-rank mode workspace: the fp32 residual of every slot (256-byte
+// aligned), then the Algorithm 3 buffers for the largest run of equal shapes.
+size_t lowrank_residual_bytes(const cf_ctx *ctx)
+{
+    size_t b = 0;
+    for (const cf_shape &s : ctx->shapes) b += round_up((size_t)(s.rows * s.cols) * 4, 256);
+    return b;
+}
+
+template <class F>
+void for_each_run(const std::vector<cf_shape> &shapes, F f)
+{
+    size_t i = 0;
+    while (i < shapes.size()) {
+        size_t j = i + 1;
+        while (j < shapes.size() && shapes[j].rows == shapes[i].rows && shapes[j].cols == shapes[i].cols) ++j;
+        f(i, j);
+        i = j;
+    }
+}
+
+size_t lowrank_mode_bytes(const cf_ctx *ctx)
+{
+    size_t algo = 0;
+    for_each_run(ctx->shapes, [&](size_t i, size_t j) {
+        const size_t b = cf::lowrank_workspace_bytes((int)(j - i), ctx->shapes[i].rows, ctx->shapes[i].cols,
+                                                     ctx->cfg.rank);
+        if (b > algo) algo = b;
+    });
+    return lowrank_residual_bytes(ctx) + algo;
+}
+
+cf_status check_quant_slot(cf_ctx *ctx, const cf_slot &s, int i, bool sender, int step)
+{
+    if (step == 0) {
+        if (!s.x) return fail(ctx, CF_E_ARG, "slot %d: x is NULL", i);
+        if (!aligned16(s.x)) return fail(ctx, CF_E_ALIGN, "slot %d: x not 16-byte aligned", i);
+        if (sender) {
+            if (!s.base || !s.err) return fail(ctx, CF_E_ARG, "slot %d: base/err is NULL", i);
+            if (!aligned16(s.base) || !aligned16(s.err)) return fail(ctx, CF_E_ALIGN, "slot %d: base/err not 16-byte aligned", i);
+        } else {
+            if (!s.cache) return fail(ctx, CF_E_ARG, "slot %d: cache is NULL", i);
+            if (!aligned16(s.cache)) return fail(ctx, CF_E_ALIGN, "slot %d: cache not 16-byte aligned", i);
+        }
+        return CF_OK;
+    }
+    if (sender) {
+        if (!s.x || !s.base || !s.err || !s.codes || !s.scales)
+            return fail(ctx, CF_E_ARG, "slot %d: x/base/err/codes/scales must be non-NULL", i);
+        if (!aligned16(s.x) || !aligned16(s.base) || !aligned16(s.err) || !aligned16(s.codes) || !aligned16(s.scales))
+            return fail(ctx, CF_E_ALIGN, "slot %d: pointers must be 16-byte aligned", i);
+    } else {
+        if (!s.codes || !s.scales || !s.cache) return fail(ctx, CF_E_ARG, "slot %d: codes/scales/cache must be non-NULL", i);
+        if (!aligned16(s.codes) || !aligned16(s.scales) || !aligned16(s.cache))
+            return fail(ctx, CF_E_ALIGN, "slot %d: pointers must be 16-byte aligned", i);
+    }
+    return CF_OK;
+}
+
+cf_status run_quant(cf_ctx *ctx, const cf_slot *slots, cf::QuantOp op, cudaStream_t stream)
+{
+    const int n = (int)ctx->shapes.size();
+    const int64_t tile = cf::quant_tile_elems();
+    cf::QuantLaunch *lp = new (std::nothrow) cf::QuantLaunch;
+    if (!lp) return fail(ctx, CF_E_NOMEM, "host allocation failed");
+    for (int first = 0; first < n; first += cf::kMaxSlotsPerLaunch) {
+        const int cnt = (n - first < cf::kMaxSlotsPerLaunch) ? n - first : cf::kMaxSlotsPerLaunch;
+        memset(lp, 0, sizeof *lp);
+        lp->nslots = cnt;
+        lp->status = ctx->d_status;
+        int64_t tiles = 0;
+        for (int k = 0; k < cnt; ++k) {
+            const cf_slot &s = slots[first + k];
+            const cf_shape &sh = ctx->shapes[first + k];
+            const int64_t elems = sh.rows * sh.cols;
+            cf::QuantSlotDesc &d = lp->slot[k];
+            d.x = s.x;
+            d.base = s.base;
+            d.err = s.err;
+            d.cache = s.cache;
+            d.codes = s.codes;
+            d.scales = s.scales;
+            d.nvec = elems / 8;
+            d.tile0 = tiles;
+            tiles += (elems + tile - 1) / tile;
+        }
+        lp->ntiles = tiles;
+        cudaError_t e = cf::launch_quant(op, ctx->cfg.bits, ctx->cfg.group, ctx->cfg.sign_scale, *lp, stream);
+        if (e != cudaSuccess) {
+            delete lp;
+            return cuda_fail(ctx, e, "quantised codec launch");
+        }
+    }
+    delete lp;
+    return CF_OK;
+}
+
+cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaStream_t stream)
+{
+    const size_t need = sender ? lowrank_mode_bytes(ctx) : 0;
+    if (sender && (!ctx->ws || ctx->ws_bytes < need))
+        return fail(ctx, CF_E_NOMEM, "low-rank mode needs %zu bytes of workspace (cf_set_workspace)", need);
+    const int n = (int)ctx->shapes.size();
+    const int r = ctx->cfg.rank;
+    for (int i = 0; i < n; ++i) {
+        const cf_slot &s = slots[i];
+        if (ctx->shapes[i].rows == 0) continue;  // an empty slot is never touched
+        if (!s.U || !s.R || !s.V) return fail(ctx, CF_E_ARG, "slot %d: U/R/V must be non-NULL", i);
+        if (!aligned16(s.U) || !aligned16(s.R) || !aligned16(s.V))
+            return fail(ctx, CF_E_ALIGN, "slot %d: U/R/V must be 16-byte aligned", i);
+        if (sender) {
+            if (!s.x || !s.base || !s.err || !s.q0) return fail(ctx, CF_E_ARG, "slot %d: x/base/err/q0 must be non-NULL", i);
+            if (!aligned16(s.x) || !aligned16(s.base) || !aligned16(s.err) || !aligned16(s.q0))
+                return fail(ctx, CF_E_ALIGN, "slot %d: x/base/err/q0 must be 16-byte aligned", i);
+            if (ctx->shapes[i].rows > 0 && (ctx->shapes[i].rows < r || ctx->shapes[i].cols < r))
+                return fail(ctx, CF_E_SHAPE, "slot %d: rows and cols must be >= rank", i);
+        } else {
+            if (!s.cache) return fail(ctx, CF_E_ARG, "slot %d: cache must be non-NULL", i);
+            if (!aligned16(s.cache)) return fail(ctx, CF_E_ALIGN, "slot %d: cache must be 16-byte aligned", i);
+        }
+    }
+    // fp32 residual of every slot, base <- x
+    std::vector<float *> a_ptr(n);
+    {
+        char *p = (char *)ctx->ws;
+        for (int i = 0; i < n; ++i) {
+            a_ptr[i] = (float *)p;
+            if (sender) p += round_up((size_t)(ctx->shapes[i].rows * ctx->shapes[i].cols) * 4, 256);
+        }
+    }
+    if (sender) {
+        std::vector<const void *> xs(n);
+        std::vector<void *> bs(n);
+        std::vector<const float *> es(n);
+        std::vector<int64_t> ns(n);
+        for (int i = 0; i < n; ++i) {
+            xs[i] = slots[i].x;
+            bs[i] = slots[i].base;
+            es[i] = slots[i].err;
+            ns[i] = ctx->shapes[i].rows * ctx->shapes[i].cols;
+        }
+        cudaError_t e = cf::launch_residual_f32(xs.data(), bs.data(), es.data(), a_ptr.data(), ns.data(), n, stream);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "residual launch");
+    }
+    char *algo_ws = (char *)ctx->ws + (sender ? lowrank_residual_bytes(ctx) : 0);
+    cf_status st = CF_OK;
+    for_each_run(ctx->shapes, [&](size_t i, size_t j) {
+        if (st != CF_OK) return;
+        const cf_shape sh = ctx->shapes[i];
+        if (sh.rows == 0) return;
+        std::vector<cf::LowrankMat> mats(j - i);
+        for (size_t k = i; k < j; ++k) {
+            cf::LowrankMat &m = mats[k - i];
+            m.A = a_ptr[k];
+            m.Q0 = slots[k].q0;
+            m.U = slots[k].U;
+            m.R = slots[k].R;
+            m.V = slots[k].V;
+            m.E = sender ? slots[k].err : nullptr;
+            m.C = sender ? nullptr : slots[k].cache;
+        }
+        cf::LowrankPlan plan{};
+        plan.nmat = (int)(j - i);
+        plan.m = sh.rows;
+        plan.n = sh.cols;
+        plan.r = ctx->cfg.rank;
+        plan.T = ctx->cfg.iters;
+        plan.ws = algo_ws;
+        plan.ws_bytes = ctx->ws_bytes - (size_t)(algo_ws - (char *)ctx->ws);
+        plan.status = ctx->d_status;
+        cudaError_t e = sender ? cf::run_lowrank(plan, mats.data(), stream)
+                               : cf::run_lowrank_decompress(plan, mats.data(), stream);
+        if (e != cudaSuccess) st = cuda_fail(ctx, e, sender ? "low-rank compress" : "low-rank decompress");
+    });
+    return st;
+}
+
+cf_status codec_call(cf_ctx *ctx, const cf_slot *slots, int step, void *stream_, bool sender)
+{
+    if (!ctx) return CF_E_ARG;
+    if (step < 0) return fail(ctx, CF_E_ARG, "step must be >= 0");
+    const int n = (int)ctx->shapes.size();
+    if (n > 0 && !slots) return fail(ctx, CF_E_ARG, "slots is NULL");
+    cudaStream_t stream = (cudaStream_t)stream_;
+    if (step > 0 && !(sender ? ctx->warm_sender : ctx->warm_receiver))
+        return fail(ctx, CF_E_STATE, "step %d before the warmup step (step 0) on this context", step);
+
+    if (step == 0 || ctx->cfg.mode == CF_MODE_QUANT) {
+        for (int i = 0; i < n; ++i) {
+            if (ctx->shapes[i].rows == 0) continue;  // an empty slot is never touched
+            cf_status st = check_quant_slot(ctx, slots[i], i, sender, step);
+            if (st != CF_OK) return st;
+        }
+        cf::QuantOp op = step == 0 ? (sender ? cf::QuantOp::WarmupSender : cf::QuantOp::WarmupReceiver)
+                                   : (sender ? cf::QuantOp::Compress : cf::QuantOp::Decompress);
+        cf_status st = run_quant(ctx, slots, op, stream);
+        if (st != CF_OK) return st;
+    } else {
+        cf_status st = run_lowrank_mode(ctx, slots, sender, stream);
+        if (st != CF_OK) return st;
+    }
+    if (step == 0) (sender ? ctx->warm_sender : ctx->warm_receiver) = true;
+    ctx->err.clear();
+    return CF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes, cf_ctx **out)
+{
+    if (!out) return CF_E_ARG;
+    *out = nullptr;
+    if (!config || nslots < 0 || (nslots > 0 && !shapes)) return CF_E_ARG;
+    std::string why;
+    cf_status st = validate_config(config, why);
+    if (st != CF_OK) return st;
+    for (int i = 0; i < nslots; ++i) {
+        const cf_shape &s = shapes[i];
+        if (s.rows < 0 || s.cols <= 0 || s.cols % 8 != 0) return CF_E_SHAPE;
+        if (s.rows > ((int64_t)1 << 40) / s.cols) return CF_E_SHAPE;
+        if (config->mode == CF_MODE_QUANT && s.cols % config->group != 0) return CF_E_SHAPE;
+        if (config->mode == CF_MODE_LOWRANK && s.rows > 0 && (s.rows < config->rank || s.cols < config->rank))
+            return CF_E_SHAPE;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CF_E_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return CF_E_CUDA;
+    if (prop.major != 10) return CF_E_CUDA;  // the kernels are built for sm_100a only
+
+    cf_ctx *ctx = new (std::nothrow) cf_ctx;
+    if (!ctx) return CF_E_NOMEM;
+    ctx->cfg = *config;
+    ctx->device = dev;
+    ctx->shapes.assign(shapes, shapes + nslots);
+    if (cudaMalloc(&ctx->d_status, 256) != cudaSuccess) {
+        delete ctx;
+        return CF_E_NOMEM;
+    }
+    if (cudaMemset(ctx->d_status, 0, 256) != cudaSuccess) {
+        cudaFree(ctx->d_status);
+        delete ctx;
+        return CF_E_CUDA;
+    }
+    *out = ctx;
+    return CF_OK;
+}
+
+size_t cf_workspace_bytes(const cf_ctx *ctx)
+{
+    if (!ctx || ctx->cfg.mode != CF_MODE_LOWRANK) return 0;
+    return lowrank_mode_bytes(ctx);
+}
+
+cf_status cf_set_workspace(cf_ctx *ctx, void *dev_ptr, size_t bytes)
+{
+    if (!ctx) return CF_E_ARG;
+    if (bytes > 0 && !dev_ptr) return fail(ctx, CF_E_ARG, "workspace pointer is NULL");
+    if (!aligned16(dev_ptr)) return fail(ctx, CF_E_ALIGN, "workspace must be 16-byte aligned");
+    ctx->ws = dev_ptr;
+    ctx->ws_bytes = bytes;
+    return CF_OK;
+}
+
+cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream)
+{
+    return codec_call(ctx, slots, step, cuda_stream, true);
+}
+
+cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream)
+{
+    return codec_call(ctx, slots, step, cuda_stream, false);
+}
+
+size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_t n)
+{
+    if (!ctx || ctx->cfg.mode != CF_MODE_LOWRANK || nmat < 0 || m < ctx->cfg.rank || n < ctx->cfg.rank) return 0;
+    return cf::lowrank_workspace_bytes(nmat, m, n, ctx->cfg.rank);
+}
+
+cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *const *A, const float *const *Q0,
+                     float *const *U, float *const *R, float *const *V, float *const *E_opt, float *const *C_opt,
+                     void *cuda_stream)
+{
+    if (!ctx) return CF_E_ARG;
+    if (ctx->cfg.mode != CF_MODE_LOWRANK) return fail(ctx, CF_E_ARG, "context is not in low-rank mode");
+    if (nmat < 0) return fail(ctx, CF_E_ARG, "nmat must be >= 0");
+    if (nmat == 0) return CF_OK;
+    if (!A || !Q0 || !U || !R || !V) return fail(ctx, CF_E_ARG, "A/Q0/U/R/V arrays must be non-NULL");
+    const int r = ctx->cfg.rank;
+    if (m < r || n < r) return fail(ctx, CF_E_SHAPE, "m and n must be >= rank");
+    if (n % 4 != 0) return fail(ctx, CF_E_SHAPE, "n must be a multiple of 4 (16-byte rows)");
+    if (m > ((int64_t)1 << 40) / n) return fail(ctx, CF_E_SHAPE, "matrix too large");
+    const size_t need = cf::lowrank_workspace_bytes(nmat, m, n, r);
+    if (!ctx->ws || ctx->ws_bytes < need)
+        return fail(ctx, CF_E_NOMEM, "cf_lowrank needs %zu bytes of workspace (cf_set_workspace)", need);
+    std::vector<cf::LowrankMat> mats(nmat);
+    for (int i = 0; i < nmat; ++i) {
+        if (!A[i] || !Q0[i] || !U[i] || !R[i] || !V[i]) return fail(ctx, CF_E_ARG, "matrix %d: NULL pointer", i);
+        if (!aligned16(A[i]) || !aligned16(Q0[i]) || !aligned16(U[i]) || !aligned16(R[i]) || !aligned16(V[i]))
+            return fail(ctx, CF_E_ALIGN, "matrix %d: pointers must be 16-byte aligned", i);
+        float *E = E_opt ? E_opt[i] : nullptr;
+        float *C = C_opt ? C_opt[i] : nullptr;
+        if (!aligned16(E) || !aligned16(C)) return fail(ctx, CF_E_ALIGN, "matrix %d: E/C must be 16-byte aligned", i);
+        mats[i] = cf::LowrankMat{A[i], Q0[i], U[i], R[i], V[i], E, C};
+    }
+    cf::LowrankPlan plan{};
+    plan.nmat = nmat;
+    plan.m = m;
+    plan.n = n;
+    plan.r = r;
+    plan.T = ctx->cfg.iters;
+    plan.ws = ctx->ws;
+    plan.ws_bytes = ctx->ws_bytes;
+    plan.status = ctx->d_status;
+    cudaError_t e = cf::run_lowrank(plan, mats.data(), (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "cf_lowrank");
+    ctx->err.clear();
+    return CF_OK;
+}
+
+cf_status cf_check(cf_ctx *ctx, void *cuda_stream)
+{
+    if (!ctx) return CF_E_ARG;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "stream synchronize");
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, ctx->d_status, sizeof word, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
+    if (word != 0) {
+        e = cudaMemset(ctx->d_status, 0, sizeof word);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "status clear");
+    }
+    if (word & cf::kStatusTimeout) return fail(ctx, CF_E_TIMEOUT, "a bounded device-side wait gave up");
+    if (word & cf::kStatusNonfinite) return fail(ctx, CF_E_NONFINITE, "a group scale was not finite");
+    if (word & cf::kStatusNotSpd) return fail(ctx, CF_E_NONFINITE, "a Gram matrix was not positive definite");
+    return CF_OK;
+}
+
+size_t cf_payload_bytes(const cf_ctx *ctx, int slot)
+{
+    if (!ctx || slot < 0 || slot >= (int)ctx->shapes.size()) return 0;
+    const cf_shape &s = ctx->shapes[slot];
+    const size_t n = (size_t)(s.rows * s.cols);
+    if (ctx->cfg.mode == CF_MODE_QUANT) return n * ctx->cfg.bits / 8 + 4 * (n / ctx->cfg.group);
+    const size_t r = (size_t)ctx->cfg.rank;
+    return 4 * r * ((size_t)s.rows + r + (size_t)s.cols);
+}
+
+const char *cf_last_error(const cf_ctx *ctx)
+{
+    if (!ctx) return "null context";
+    return ctx->err.c_str();
+}
+
+cf_status cf_destroy(cf_ctx *ctx)
+{
+    if (!ctx) return CF_E_ARG;
+    if (ctx->d_status) cudaFree(ctx->d_status);
+    delete ctx;
+    return CF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// cf_internal.h -- declarations shared by the libcf translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "cf.h"
+
+namespace cf {
+
+// Device status word bits (read and cleared by cf_check).
+constexpr uint32_t kStatusNonfinite = 0x1u;
+constexpr uint32_t kStatusTimeout = 0x2u;
+constexpr uint32_t kStatusNotSpd = 0x4u;
+
+// Slots per grouped launch of the quantised kernels; the descriptor table
+// travels as a __grid_constant__ kernel parameter (CUDA 12.1+ allows up to
+// 32 KB of parameters), so no per-call device allocation or copy is needed.
+constexpr int kMaxSlotsPerLaunch = 128;
+
+struct QuantSlotDesc {
+    const void *x;     // bf16
+    void *base;        // bf16
+    float *err;        // fp32
+    float *cache;      // fp32
+    uint8_t *codes;    // packed codes
+    float *scales;     // fp32 group scales
+    int64_t nvec;      // elements / 8
+    int64_t tile0;     // first tile index of this slot in the launch
+};
+
+struct QuantLaunch {
+    int nslots;
+    int pad_;
+    int64_t ntiles;
+    uint32_t *status;
+    QuantSlotDesc slot[kMaxSlotsPerLaunch];
+};
+
+enum class QuantOp { WarmupSender, WarmupReceiver, Compress, Decompress };
+
+// Elements per tile of the quantised kernels (one tile = one CTA iteration).
+int64_t quant_tile_elems();
+
+// Launch one grouped quantised kernel over `lp` (host-built).  bits/group/
+// sign_scale select the template instance.  Returns cudaSuccess or the launch
+// error.
+cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, const QuantLaunch &lp,
+                         cudaStream_t stream);
+
+// ---------------------------------------------------------------- low rank
+
+struct LowrankMat {
+    const float *A;    // [m x n] row-major
+    const float *Q0;   // [n x r]
+    float *U;          // [m x r]
+    float *R;          // [r x r]
+    float *V;          // [n x r]
+    float *E;          // [m x n] or null
+    float *C;          // [m x n] or null
+};
+
+struct LowrankPlan {
+    int nmat;
+    int64_t m, n;
+    int r, T;
+    void *ws;          // device workspace
+    size_t ws_bytes;
+    uint32_t *status;
+};
+
+size_t lowrank_workspace_bytes(int nmat, int64_t m, int64_t n, int r);
+
+// Runs Algorithm 3 (and the apply step) for plan.nmat matrices.  `mats` is a
+// host array.  Returns a cudaError_t from the launches.
+cudaError_t run_lowrank(const LowrankPlan &plan, const LowrankMat *mats, cudaStream_t stream);
+
+// Low-rank decompress: C += U R V^T for each matrix (E, A unused).
+cudaError_t run_lowrank_decompress(const LowrankPlan &plan, const LowrankMat *mats, cudaStream_t stream);
+
+// Residual materialisation for low-rank mode: A = (x - base) + err (fp32) into
+// `a_out`, base <- x.  One launch per slot list.
+cudaError_t launch_residual_f32(const void *const *x, void *const *base, const float *const *err,
+                                float *const *a_out, const int64_t *n, int nslots, cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace cf

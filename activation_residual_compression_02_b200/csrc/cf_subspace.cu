@@ -1,0 +1,860 @@
+// cf_subspace.cu -- Algorithm 3 (rank-r subspace iteration) for sm_100a.
+//
+// "Accelerating Parallel Diffusion Model Serving with Residual Compression"
+// (arXiv 2507.17511), reproducibility table, "Pseudocode" row, Algorithm 3:
+//   Q = orth(random Q0); repeat T: Z = A^T (A Q), Q = orth(Z);
+//   U = orth(A Q); V = Q.
+// orth() is CholeskyQR (G = Y^T Y, R = chol(G), Y R^{-1}); keeping the R of
+// the last step gives the payload (U, R, V) whose reconstruction is U R V^T.
+//
+// Kernels (one grouped launch each, over every matrix of the call):
+//  * k_gemm_tf32: the two products with A.  P = A Q (A K-major) and
+//    Z = A^T P (A read as an MN-major operand straight from its row-major
+//    storage).  A warp-specialised persistent tcgen05 kernel: one TMA warp
+//    streams 128x32 fp32 tiles of A (128-byte swizzle) plus the matching
+//    r-column slice of Q^T / P^T; four warps round each A tile to TF32 in
+//    shared memory (round to nearest: the tensor core would otherwise drop the
+//    low mantissa bits, a bias of about 2^-11 that alone costs ~7e-4 of the
+//    reconstruction); one thread issues tcgen05.mma (M=128, N=16/32, K=8)
+//    into a double-buffered TMEM accumulator; four warps drain TMEM with
+//    tcgen05.ld and write the r-column result.  The work is HBM-bound (8 flop
+//    per byte of A), so the tensor cores only have to keep up with the stream.
+//  * k_gram / k_chol_solve: CholeskyQR in fp64 -- Gram partials with fp64
+//    atomics, then every CTA recomputes the r x r Cholesky factor and solves
+//    its rows (Y R^{-1}).
+//  * k_apply: D = U (R V^T) on CUDA cores (K = r is far too thin for the
+//    tensor cores; the step is an HBM stream), fused with E = A - D and
+//    C += D.
+// Every mbarrier wait is bounded (about 2 s of %globaltimer); on expiry the
+// CTA raises an abort flag and a status bit, drains its own TMA loads and
+// MMAs, frees TMEM and returns.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "cf_internal.h"
+
+namespace cf {
+namespace {
+
+// ------------------------------------------------------------ constants --
+constexpr int kBM = 128;            // MMA M: rows of an output tile
+constexpr int kBK = 32;             // K per pipeline stage (fp32: 128 bytes)
+constexpr int kStages = 8;
+constexpr int kGemmThreads = 320;   // 10 warps: TMA, MMA, 4 convert, 4 epilogue
+constexpr int kATileBytes = kBM * kBK * 4;   // 16 KB
+constexpr int kBTileBytes = 32 * kBK * 4;    // room for N = 32
+constexpr int kMaxGemmMats = 40;
+constexpr int kTmemCols = 64;       // two accumulators of up to 32 columns
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+struct __align__(64) GemmMat {
+    CUtensorMap ta;    // A (fp32, row-major m x n)
+    CUtensorMap tb;    // B^T slice source: Q^T [RP x n] or P^T [RP x m] (K-major)
+    float *out;        // output
+    int64_t pad_[7];
+};
+
+struct GemmParams {
+    GemmMat mat[kMaxGemmMats];
+    int nmat;
+    int tiles_per_mat;
+    int ktiles;
+    int out_rows;      // valid output rows (m for A Q, n for A^T P)
+    int rp;            // N of the MMA (16 or 32)
+    int mn_major;      // 0: out = A Q (A K-major); 1: out = A^T P (A MN-major)
+    int out_mode;      // 0: transposed + TF32-rounded [rp][out_ld]; 1: exact row-major [rows][rp]
+    int out_ld;        // leading dimension of the transposed output
+    uint32_t *status;
+    unsigned long long wait_ns;
+};
+
+// ------------------------------------------------------- PTX wrappers ----
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *b)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: true when the phase of `parity` completed; false on abort or
+// timeout (the first thread to time out raises the abort flag and the status).
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *status,
+                                          unsigned long long limit_ns)
+{
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((i & 31) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_tf32(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float round_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version
+// 1 in bits 46-47, layout type 2 in bits 61-63).  Offsets are in bytes.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::tf32: D fp32, A/B tf32, M = 128, N = rp.
+__device__ __forceinline__ uint32_t instr_desc_tf32(int rp, int a_mn_major)
+{
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)(rp >> 3) << 17) |
+           ((uint32_t)(kBM >> 4) << 24);
+}
+
+struct GemmSmem {
+    uint64_t full[kStages];
+    uint64_t conv[kStages];
+    uint64_t empty[kStages];
+    uint64_t accf[2];
+    uint64_t acce[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// ------------------------------------------------------------ the GEMM ----
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_constant__ GemmParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = base;                                   // kStages x 16 KB
+    uint8_t *sB = base + kStages * kATileBytes;           // kStages x 4 KB
+    GemmSmem *S = (GemmSmem *)(sB + kStages * kBTileBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int total_tiles = p.nmat * p.tiles_per_mat;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&S->full[s], 1);
+            mbar_init(&S->conv[s], 128);
+            mbar_init(&S->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&S->accf[b], 1);
+            mbar_init(&S->acce[b], 128);
+        }
+        mbar_init(&S->drain, 1);
+        S->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S->tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S->tmem_base;
+    volatile int *abort_flag = &S->abort_flag;
+    const unsigned long long wait_ns = p.wait_ns;
+    const int rp = p.rp;
+    const uint32_t stage_bytes = (uint32_t)kATileBytes + (uint32_t)rp * kBK * 4;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+                const int mi = tile / p.tiles_per_mat;
+                const int mt = tile - mi * p.tiles_per_mat;
+                const GemmMat &M = p.mat[mi];
+                for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait_bounded(&S->empty[s], ph ^ 1u, abort_flag, p.status, wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(&S->full[s], stage_bytes);
+                    uint8_t *a = sA + s * kATileBytes;
+                    if (!p.mn_major) {
+                        tma_load_2d(a, &M.ta, kt * kBK, mt * kBM, &S->full[s]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tma_load_2d(a + j * 4096, &M.ta, mt * kBM + 32 * j, kt * kBK, &S->full[s]);
+                    }
+                    tma_load_2d(sB + s * kBTileBytes, &M.tb, kt * kBK, 0, &S->full[s]);
+                }
+            }
+            // Drain: every load this thread issued has landed before exit.
+            const uint32_t outstanding = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+            for (uint32_t j = it - outstanding; j < it; ++j) {
+                volatile int no_abort = 0;
+                wait_bounded(&S->full[j % kStages], (j / kStages) & 1u, &no_abort, p.status, kWaitNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ---
+        const uint32_t idesc = instr_desc_tf32(rp, p.mn_major);
+        uint32_t it = 0, lt = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            const uint32_t aph = (lt >> 1) & 1u;
+            if (!wait_bounded(&S->acce[b], aph ^ 1u, abort_flag, p.status, wait_ns)) break;
+            tc_fence_after();
+            const uint32_t dtm = tmem + (uint32_t)(b * 32);
+            for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                if (!wait_bounded(&S->conv[s], ph, abort_flag, p.status, wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_u32(sA + s * kATileBytes);
+                    const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / 8; ++k) {
+                        const uint64_t ad = p.mn_major ? smem_desc(a0 + k * 1024, 4096, 1024)
+                                                       : smem_desc(a0 + k * 32, 16, 1024);
+                        const uint64_t bd = smem_desc(b0 + k * 32, 16, 1024);
+                        tc_mma_tf32(dtm, ad, bd, idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&S->empty[s]);
+                }
+                __syncwarp();
+            }
+            if (ok && lane == 0) tc_commit(&S->accf[b]);
+            __syncwarp();
+        }
+        // Drain: all MMAs this thread issued have completed before TMEM is freed.
+        if (lane == 0) {
+            tc_commit(&S->drain);
+            volatile int no_abort = 0;
+            wait_bounded(&S->drain, 0, &no_abort, p.status, kWaitNs);
+        }
+        __syncwarp();
+    } else if (warp < 6) {
+        // ------------------------------------ TF32 rounding of A tiles --
+        const int ct = threadIdx.x - 64;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1u;
+                if (!wait_bounded(&S->full[s], ph, abort_flag, p.status, wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                float4 *a = (float4 *)(sA + s * kATileBytes);
+#pragma unroll
+                for (int i = 0; i < kATileBytes / 16 / 128; ++i) {
+                    float4 v = a[ct + 128 * i];
+                    v.x = round_tf32(v.x);
+                    v.y = round_tf32(v.y);
+                    v.z = round_tf32(v.z);
+                    v.w = round_tf32(v.w);
+                    a[ct + 128 * i] = v;
+                }
+                fence_proxy_async();
+                mbar_arrive(&S->conv[s]);
+            }
+        }
+    } else {
+        // ----------------------------------------------------- epilogue --
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        uint32_t lt = 0;
+        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            const uint32_t aph = (lt >> 1) & 1u;
+            if (!wait_bounded(&S->accf[b], aph, abort_flag, p.status, wait_ns)) break;
+            tc_fence_after();
+            uint32_t v[32];
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * 32);
+            {
+                uint32_t lo[16];
+                tc_ld16(taddr, lo);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) v[c] = lo[c];
+            }
+            if (rp > 16) {
+                uint32_t hi[16];
+                tc_ld16(taddr + 16, hi);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) v[16 + c] = hi[c];
+            }
+            tc_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&S->acce[b]);
+
+            const int mi = tile / p.tiles_per_mat;
+            const int mt = tile - mi * p.tiles_per_mat;
+            const int row = mt * kBM + 32 * q + lane;
+            float *out = p.mat[mi].out;
+            if (row < p.out_rows) {
+                if (p.out_mode == 0) {
+                    for (int c = 0; c < rp; ++c)
+                        out[(int64_t)c * p.out_ld + row] = round_tf32(__uint_as_float(v[c]));
+                } else {
+                    float4 *o = (float4 *)(out + (int64_t)row * rp);
+                    for (int c = 0; c < rp; c += 4)
+                        o[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                               __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+constexpr size_t kGemmSmemBytes = 1024 + kStages * (kATileBytes + kBTileBytes) + sizeof(GemmSmem);
+
+// ------------------------------------------------------ CholeskyQR -------
+constexpr int kGramThreads = 256;
+constexpr int kGramRows = 256;   // rows per Gram CTA
+
+struct CholMat {
+    const float *Y;     // input block [rows x ld]
+    double *G;          // Gram matrix [rp x rp] (fp64, zeroed before k_gram)
+    float *Qt;          // mode Q: rounded transposed output [rp x qt_ld] (rows >= r zero)
+    float *Qexact;      // mode Q: optional exact output [rows x r] (V)
+    float *U;           // mode U: [rows x r]
+    float *R;           // mode U: [r x r]
+};
+
+constexpr int kMaxCholMats = 64;
+
+struct CholParams {
+    CholMat mat[kMaxCholMats];
+    int nmat;
+    int rows;
+    int ld;             // row stride of Y (r or rp)
+    int r;
+    int qt_ld;
+    uint32_t *status;
+};
+
+// Gram partials: CTA (chunk, mat) adds Y[chunk]^T Y[chunk] (upper triangle)
+// into G in fp64.
+__global__ void __launch_bounds__(kGramThreads) k_gram(const __grid_constant__ CholParams p)
+{
+    const CholMat &M = p.mat[blockIdx.y];
+    const int r = p.r;
+    const int row0 = blockIdx.x * kGramRows;
+    const int nrows = min(kGramRows, p.rows - row0);
+    __shared__ float ys[kGramRows * 33];
+    for (int i = threadIdx.x; i < nrows * r; i += kGramThreads) {
+        const int rr = i / r, c = i - rr * r;
+        ys[rr * 33 + c] = M.Y[(int64_t)(row0 + rr) * p.ld + c];
+    }
+    __syncthreads();
+    const int npairs = r * (r + 1) / 2;
+    for (int pidx = threadIdx.x; pidx < npairs; pidx += kGramThreads) {
+        // pair index -> (i, j), i <= j
+        int i = 0, rem = pidx;
+        while (rem >= r - i) {
+            rem -= r - i;
+            ++i;
+        }
+        const int j = i + rem;
+        double acc = 0.0;
+        for (int k = 0; k < nrows; ++k) acc += (double)ys[k * 33 + i] * (double)ys[k * 33 + j];
+        atomicAdd(&M.G[i * 32 + j], acc);
+    }
+}
+
+// Cholesky of G (upper R, G = R^T R) by one thread into shared memory.
+__device__ void cholesky_upper(const double *G, double *R, int r, uint32_t *status, bool report)
+{
+    for (int i = 0; i < r * 32; ++i) R[i] = 0.0;
+    for (int pp = 0; pp < r; ++pp) {
+        double diag = G[pp * 32 + pp];
+        for (int k = 0; k < pp; ++k) diag -= R[k * 32 + pp] * R[k * 32 + pp];
+        if (!(diag > 0.0) || !isfinite(diag)) {
+            if (report) atomicOr(status, kStatusNotSpd);
+            diag = 1.0;  // keeps the solve finite; the status reports the failure
+        }
+        const double d = sqrt(diag);
+        R[pp * 32 + pp] = d;
+        for (int qq = pp + 1; qq < r; ++qq) {
+            double v = G[pp * 32 + qq];
+            for (int k = 0; k < pp; ++k) v -= R[k * 32 + pp] * R[k * 32 + qq];
+            R[pp * 32 + qq] = v / d;
+        }
+    }
+}
+
+constexpr int kSolveThreads = 256;
+
+// Y R^{-1} row by row (forward substitution over the columns), fp64.
+// mode 0: Qt (rounded, transposed) [+ Qexact];  mode 1: U (+ R by CTA 0).
+template <int MODE>
+__global__ void __launch_bounds__(kSolveThreads) k_chol_solve(const __grid_constant__ CholParams p)
+{
+    const CholMat &M = p.mat[blockIdx.y];
+    const int r = p.r;
+    __shared__ double Gs[32 * 32];
+    __shared__ double Rs[32 * 32];
+    for (int i = threadIdx.x; i < 32 * 32; i += kSolveThreads) Gs[i] = M.G[i];
+    __syncthreads();
+    if (threadIdx.x == 0) cholesky_upper(Gs, Rs, r, p.status, blockIdx.x == 0);
+    __syncthreads();
+    if (MODE == 1 && blockIdx.x == 0) {
+        for (int i = threadIdx.x; i < r * r; i += kSolveThreads) {
+            const int a = i / r, b = i - a * r;
+            M.R[i] = (float)Rs[a * 32 + b];
+        }
+    }
+    for (int row = blockIdx.x * kSolveThreads + threadIdx.x; row < p.rows; row += gridDim.x * kSolveThreads) {
+        double q[32];
+        const float *y = M.Y + (int64_t)row * p.ld;
+        for (int c = 0; c < r; ++c) {
+            double v = (double)y[c];
+            for (int k = 0; k < c; ++k) v -= q[k] * Rs[k * 32 + c];
+            q[c] = v / Rs[c * 32 + c];
+        }
+        if (MODE == 0) {
+            for (int c = 0; c < r; ++c) M.Qt[(int64_t)c * p.qt_ld + row] = round_tf32((float)q[c]);
+            if (M.Qexact)
+                for (int c = 0; c < r; ++c) M.Qexact[(int64_t)row * r + c] = (float)q[c];
+        } else {
+            for (int c = 0; c < r; ++c) M.U[(int64_t)row * r + c] = (float)q[c];
+        }
+    }
+}
+
+// -------------------------------------------------------------- apply ----
+constexpr int kApplyThreads = 256;
+constexpr int kApplyRows = 64;     // rows per CTA tile
+constexpr int kApplyCols = 128;    // columns per CTA tile (32 threads x float4)
+
+struct ApplyMat {
+    const float *A;   // [m x n] or null
+    const float *U;   // [m x r]
+    const float *R;   // [r x r]
+    const float *V;   // [n x r]
+    float *E;         // [m x n] or null: E = A - D
+    float *C;         // [m x n] or null: C += D
+};
+
+constexpr int kMaxApplyMats = 128;
+
+struct ApplyParams {
+    ApplyMat mat[kMaxApplyMats];
+    int nmat;
+    int m, n, r;
+    int row_tiles, col_tiles;
+};
+
+// D = U (R V^T) for a 64 x 128 tile: W = R V^T (r x 128) and the U rows are
+// staged in shared memory; each thread owns a float4 column strip of 8 rows.
+__global__ void __launch_bounds__(kApplyThreads) k_apply(const __grid_constant__ ApplyParams p)
+{
+    const int per_mat = p.row_tiles * p.col_tiles;
+    const int mi = blockIdx.x / per_mat;
+    const int t = blockIdx.x - mi * per_mat;
+    const int rt = t / p.col_tiles, ctile = t - rt * p.col_tiles;
+    const ApplyMat &M = p.mat[mi];
+    const int r = p.r, n = p.n;
+    const int row0 = rt * kApplyRows, col0 = ctile * kApplyCols;
+    __shared__ float Rs[32 * 32];
+    __shared__ float Vs[kApplyCols * 33];
+    __shared__ float Ws[32 * kApplyCols];
+    __shared__ float Us[kApplyRows * 33];
+    for (int i = threadIdx.x; i < r * r; i += kApplyThreads) Rs[(i / r) * 32 + (i % r)] = M.R[i];
+    for (int i = threadIdx.x; i < kApplyCols * r; i += kApplyThreads) {
+        const int j = i / r, c = i - j * r;
+        Vs[j * 33 + c] = (col0 + j < n) ? M.V[(int64_t)(col0 + j) * r + c] : 0.0f;
+    }
+    for (int i = threadIdx.x; i < kApplyRows * r; i += kApplyThreads) {
+        const int a = i / r, c = i - a * r;
+        Us[a * 33 + c] = (row0 + a < p.m) ? M.U[(int64_t)(row0 + a) * r + c] : 0.0f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < r * kApplyCols; i += kApplyThreads) {
+        const int k = i / kApplyCols, j = i - k * kApplyCols;
+        float w = 0.0f;
+        for (int q = k; q < r; ++q) w = fmaf(Rs[k * 32 + q], Vs[j * 33 + q], w);  // R is upper triangular
+        Ws[k * kApplyCols + j] = w;
+    }
+    __syncthreads();
+    const int cx = (threadIdx.x & 31) * 4;        // column offset in the tile
+    const int ry = threadIdx.x >> 5;              // 8 row groups of 4 rows
+    const int col = col0 + cx;
+    if (col >= n) return;                          // n % 8 == 0: a float4 is all in or all out
+    for (int rr = 0; rr < kApplyRows / 8; ++rr) {
+        const int a = ry + 8 * rr;
+        const int row = row0 + a;
+        if (row >= p.m) break;
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+        for (int k = 0; k < r; ++k) {
+            const float u = Us[a * 33 + k];
+            const float4 w = *(const float4 *)&Ws[k * kApplyCols + cx];
+            d0 = fmaf(u, w.x, d0);
+            d1 = fmaf(u, w.y, d1);
+            d2 = fmaf(u, w.z, d2);
+            d3 = fmaf(u, w.w, d3);
+        }
+        const int64_t off = (int64_t)row * n + col;
+        if (M.E) {
+            const float4 av = __ldcs((const float4 *)(M.A + off));
+            __stcs((float4 *)(M.E + off), make_float4(av.x - d0, av.y - d1, av.z - d2, av.w - d3));
+        }
+        if (M.C) {
+            const float4 cv = __ldcs((const float4 *)(M.C + off));
+            __stcs((float4 *)(M.C + off), make_float4(cv.x + d0, cv.y + d1, cv.z + d2, cv.w + d3));
+        }
+    }
+}
+
+// ----------------------------------------------------------- host side ---
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                              const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn()
+{
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeFn)p;
+    });
+    return fn;
+}
+
+// 2-D fp32 tensor map: dims {inner, outer}, row pitch in elements, box {bx, by}.
+bool make_map(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t pitch_elems, uint32_t bx,
+              uint32_t by)
+{
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch_elems * 4};
+    cuuint32_t box[2] = {bx, by};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int64_t rup(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+    int rp;
+    int64_t mp, np;                       // padded leading dims (multiples of 32)
+    size_t qt, pt, pe, z, g, total;       // per-matrix byte offsets inside the workspace
+};
+
+WsLayout layout(int nmat, int64_t m, int64_t n, int r)
+{
+    WsLayout L{};
+    L.rp = r <= 16 ? 16 : 32;
+    L.mp = rup(m, 32);
+    L.np = rup(n, 32);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (size_t)rup((int64_t)bytes, 256);
+        return o;
+    };
+    L.qt = take((size_t)nmat * L.rp * L.np * 4);
+    L.pt = take((size_t)nmat * L.rp * L.mp * 4);
+    L.pe = take((size_t)nmat * m * L.rp * 4);
+    L.z = take((size_t)nmat * n * L.rp * 4);
+    L.g = take((size_t)nmat * 32 * 32 * 8);
+    L.total = off;
+    return L;
+}
+
+cudaError_t gemm_launch(GemmParams &gp, int total_tiles, cudaStream_t stream)
+{
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(k_gemm_tf32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const int grid = total_tiles < num_sms() ? total_tiles : num_sms();
+    if (grid <= 0) return cudaSuccess;
+    k_gemm_tf32<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(gp);
+    return cudaGetLastError();
+}
+
+// out_i = A_i Q_i (mn_major = 0) or A_i^T P_i (mn_major = 1) for a chunk of matrices.
+cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLayout &L, int mn_major, int out_mode,
+                      cudaStream_t stream)
+{
+    char *ws = (char *)pl.ws;
+    const int64_t m = pl.m, n = pl.n;
+    GemmParams *gp = new GemmParams;
+    cudaError_t err = cudaSuccess;
+    for (int first = 0; first < pl.nmat && err == cudaSuccess; first += kMaxGemmMats) {
+        const int cnt = pl.nmat - first < kMaxGemmMats ? pl.nmat - first : kMaxGemmMats;
+        memset(gp, 0, sizeof *gp);
+        gp->nmat = cnt;
+        gp->rp = L.rp;
+        gp->mn_major = mn_major;
+        gp->out_mode = out_mode;
+        gp->status = pl.status;
+        gp->wait_ns = kWaitNs;
+        if (!mn_major) {
+            gp->tiles_per_mat = (int)((m + kBM - 1) / kBM);
+            gp->ktiles = (int)((n + kBK - 1) / kBK);
+            gp->out_rows = (int)m;
+            gp->out_ld = (int)L.mp;
+        } else {
+            gp->tiles_per_mat = (int)((n + kBM - 1) / kBM);
+            gp->ktiles = (int)((m + kBK - 1) / kBK);
+            gp->out_rows = (int)n;
+            gp->out_ld = 0;
+        }
+        for (int k = 0; k < cnt; ++k) {
+            const int i = first + k;
+            GemmMat &g = gp->mat[k];
+            bool ok;
+            if (!mn_major) {
+                ok = make_map(&g.ta, mats[i].A, n, m, n, kBK, kBM) &&
+                     make_map(&g.tb, ws + L.qt + (size_t)i * L.rp * L.np * 4, n, L.rp, L.np, kBK, L.rp);
+                g.out = out_mode == 0 ? (float *)(ws + L.pt + (size_t)i * L.rp * L.mp * 4)
+                                      : (float *)(ws + L.pe + (size_t)i * m * L.rp * 4);
+            } else {
+                ok = make_map(&g.ta, mats[i].A, n, m, n, 32, kBK) &&
+                     make_map(&g.tb, ws + L.pt + (size_t)i * L.rp * L.mp * 4, m, L.rp, L.mp, kBK, L.rp);
+                g.out = (float *)(ws + L.z + (size_t)i * n * L.rp * 4);
+            }
+            if (!ok) {
+                err = cudaErrorInvalidValue;
+                break;
+            }
+        }
+        if (err == cudaSuccess) err = gemm_launch(*gp, cnt * gp->tiles_per_mat, stream);
+    }
+    delete gp;
+    return err;
+}
+
+// CholeskyQR of a tall block for every matrix: mode 0 writes Qt (+ V when
+// `final_v`), mode 1 writes U and R.
+cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLayout &L, int src, int mode,
+                        bool final_v, cudaStream_t stream)
+{
+    char *ws = (char *)pl.ws;
+    const int64_t m = pl.m, n = pl.n;
+    const int r = pl.r;
+    // src: 0 = Q0 (n x r), 1 = Z (n x rp), 2 = P exact (m x rp)
+    const int rows = (int)(src == 2 ? m : n);
+    const int ld = src == 0 ? r : L.rp;
+    cudaError_t err = cudaMemsetAsync(ws + L.g, 0, (size_t)pl.nmat * 32 * 32 * 8, stream);
+    if (err != cudaSuccess) return err;
+    CholParams *cp = new CholParams;
+    for (int first = 0; first < pl.nmat && err == cudaSuccess; first += kMaxCholMats) {
+        const int cnt = pl.nmat - first < kMaxCholMats ? pl.nmat - first : kMaxCholMats;
+        memset(cp, 0, sizeof *cp);
+        cp->nmat = cnt;
+        cp->rows = rows;
+        cp->ld = ld;
+        cp->r = r;
+        cp->qt_ld = (int)L.np;
+        cp->status = pl.status;
+        for (int k = 0; k < cnt; ++k) {
+            const int i = first + k;
+            CholMat &c = cp->mat[k];
+            c.Y = src == 0 ? mats[i].Q0
+                           : (src == 1 ? (const float *)(ws + L.z + (size_t)i * n * L.rp * 4)
+                                       : (const float *)(ws + L.pe + (size_t)i * m * L.rp * 4));
+            c.G = (double *)(ws + L.g + (size_t)i * 32 * 32 * 8);
+            c.Qt = (float *)(ws + L.qt + (size_t)i * L.rp * L.np * 4);
+            c.Qexact = final_v ? mats[i].V : nullptr;
+            c.U = mats[i].U;
+            c.R = mats[i].R;
+        }
+        dim3 ggrid((unsigned)((rows + kGramRows - 1) / kGramRows), (unsigned)cnt);
+        k_gram<<<ggrid, kGramThreads, 0, stream>>>(*cp);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) break;
+        const int per = (int)((rows + kSolveThreads - 1) / kSolveThreads);
+        dim3 sgrid((unsigned)(per < 8 ? per : 8), (unsigned)cnt);
+        if (mode == 0)
+            k_chol_solve<0><<<sgrid, kSolveThreads, 0, stream>>>(*cp);
+        else
+            k_chol_solve<1><<<sgrid, kSolveThreads, 0, stream>>>(*cp);
+        err = cudaGetLastError();
+    }
+    delete cp;
+    return err;
+}
+
+cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sender, cudaStream_t stream)
+{
+    ApplyParams *ap = new ApplyParams;
+    cudaError_t err = cudaSuccess;
+    for (int first = 0; first < pl.nmat && err == cudaSuccess; first += kMaxApplyMats) {
+        const int cnt = pl.nmat - first < kMaxApplyMats ? pl.nmat - first : kMaxApplyMats;
+        memset(ap, 0, sizeof *ap);
+        ap->nmat = cnt;
+        ap->m = (int)pl.m;
+        ap->n = (int)pl.n;
+        ap->r = pl.r;
+        ap->row_tiles = (int)((pl.m + kApplyRows - 1) / kApplyRows);
+        ap->col_tiles = (int)((pl.n + kApplyCols - 1) / kApplyCols);
+        bool any = false;
+        for (int k = 0; k < cnt; ++k) {
+            const LowrankMat &s = mats[first + k];
+            ApplyMat &a = ap->mat[k];
+            a.A = s.A;
+            a.U = s.U;
+            a.R = s.R;
+            a.V = s.V;
+            a.E = sender ? s.E : nullptr;
+            a.C = s.C;
+            any = any || a.E || a.C;
+        }
+        if (!any) continue;
+        const int64_t blocks = (int64_t)cnt * ap->row_tiles * ap->col_tiles;
+        k_apply<<<(unsigned)blocks, kApplyThreads, 0, stream>>>(*ap);
+        err = cudaGetLastError();
+    }
+    delete ap;
+    return err;
+}
+
+}  // namespace
+
+size_t lowrank_workspace_bytes(int nmat, int64_t m, int64_t n, int r) { return layout(nmat, m, n, r).total; }
+
+cudaError_t run_lowrank(const LowrankPlan &pl, const LowrankMat *mats, cudaStream_t stream)
+{
+    if (pl.nmat <= 0) return cudaSuccess;
+    if (pl.m > INT32_MAX || pl.n > INT32_MAX) return cudaErrorInvalidValue;
+    const WsLayout L = layout(pl.nmat, pl.m, pl.n, pl.r);
+    if (pl.ws_bytes < L.total) return cudaErrorInvalidValue;
+    char *ws = (char *)pl.ws;
+    // Padded rows of Q^T (rows r..rp-1) must be zero: they feed zero columns.
+    cudaError_t err = cudaMemsetAsync(ws + L.qt, 0, (size_t)pl.nmat * L.rp * L.np * 4, stream);
+    if (err == cudaSuccess) err = cudaMemsetAsync(ws + L.pt, 0, (size_t)pl.nmat * L.rp * L.mp * 4, stream);
+    // Line 1: Q = orth(Q0).
+    if (err == cudaSuccess) err = cholqr_pass(pl, mats, L, 0, 0, pl.T == 0, stream);
+    // Lines 2-5: T times Z = A^T (A Q), Q = orth(Z).
+    for (int t = 0; t < pl.T && err == cudaSuccess; ++t) {
+        err = gemm_pass(pl, mats, L, 0, 0, stream);                      // P^T = (A Q)^T, TF32-rounded
+        if (err == cudaSuccess) err = gemm_pass(pl, mats, L, 1, 1, stream);   // Z = A^T P
+        if (err == cudaSuccess) err = cholqr_pass(pl, mats, L, 1, 0, t == pl.T - 1, stream);
+    }
+    // Lines 6-8: P = A Q; (U, R) = orth(P); V = Q.
+    if (err == cudaSuccess) err = gemm_pass(pl, mats, L, 0, 1, stream);
+    if (err == cudaSuccess) err = cholqr_pass(pl, mats, L, 2, 1, false, stream);
+    // Apply: E = A - U R V^T and/or C += U R V^T.
+    if (err == cudaSuccess) err = apply_pass(pl, mats, true, stream);
+    return err;
+}
+
+cudaError_t run_lowrank_decompress(const LowrankPlan &pl, const LowrankMat *mats, cudaStream_t stream)
+{
+    if (pl.m > INT32_MAX || pl.n > INT32_MAX) return cudaErrorInvalidValue;
+    return apply_pass(pl, mats, false, stream);
+}
+
+}  // namespace cf

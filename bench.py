@@ -1,0 +1,504 @@
+#!/usr/bin/env python
+"""Benchmark of the residual-compression codec on B200 (one JSON line).
+
+A step is one denoising step of the codec over every slot of the workload:
+cf_compress (residual + error feedback + k-bit group quantisation + packing,
+one grouped launch) followed by cf_decompress (unpack + dequantise +
+accumulate, one grouped launch), on synthetic activations shaped like the
+FLUX.1-dev patch-parallel shard (57 blocks x 1152 tokens x 3072 channels,
+bf16, 2-bit codes, groups of 128).  The warmup step 0 runs before timing.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cf|reference]
+
+Under torchrun (N > 1) every rank runs the whole workload on its own GPU
+(the codec has no cross-slot exchange: weak scaling, no data-path
+collective); rank 0 prints the line with the max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "codec GB/s of activation input and % of B200 HBM roofline (1 GPU)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def alg_bytes_per_elem(bits, group):
+    """Algorithmic HBM bytes per activation element (compress, decompress).
+
+    compress  : read X (2), base (2), E (4); write base (2), E (4), codes k/8,
+                scales 4/G
+    decompress: read codes k/8, scales 4/G, C (4); write C (4)
+    """
+    payload = bits / 8 + 4 / group
+    return 2 + 2 + 4 + 2 + 4 + payload, payload + 4 + 4
+
+
+def source_hash():
+    p = os.path.join(ROOT, "activation_residual_compression_02_b200", "csrc", "cf_quant.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu summary of the same source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if e and e.get("source_sha") == source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, dev_index):
+        self.samples = []
+        self.ok = False
+        self.reasons = set()
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_run(w, xs_host, threads):
+    """Time the oracle (compress + decompress) over host inputs
+    ``xs_host[slot] = [X_0, X_1, ...]`` (raw bf16 bits); step 0 (the warmup)
+    is untimed.  Returns (seconds, elements of the timed steps)."""
+    import concurrent.futures
+
+    import oracle
+
+    oracle.build()
+    slots = sorted(xs_host)
+    states = {s: oracle.QuantSlot(w.bits, w.group) for s in slots}
+    for s in slots:
+        states[s].step(0, xs_host[s][0])
+
+    def work(s):
+        for t in range(1, len(xs_host[s])):
+            states[s].step(t, xs_host[s][t])
+
+    t0 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(work, slots))
+    dt = time.perf_counter() - t0
+    elems = sum(x.size for s in slots for x in xs_host[s][1:])
+    return dt, elems
+
+
+def host_inputs(w, rows, steps, seed=0):
+    """Inputs of `steps` steps (warmup included) for `rows` token rows of every slot, generated on the host."""
+    import numpy as np
+
+    sub = w.scaled(rows=rows)
+    return {s: [synth.bf16_bits(x).numpy().view(np.uint16).ravel().copy()
+                for x in synth.activations(sub, s, steps, seed=seed)] for s in range(w.slots)}
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- main
+
+def run_reference(args, w):
+    # the oracle runs on rank 0's host cores only; other ranks exit without work
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    cores = cpu_cores()
+    steps = args.steps + args.warmup
+    budget = args.budget
+    # about 15 ns of oracle work per element per step on one core; size the
+    # per-step row sample so that the whole run stays within the budget
+    per_step_elems = budget / steps * cores / 15e-9
+    rows = int(max(1, min(w.rows, per_step_elems // (w.slots * w.cols))))
+    xs = host_inputs(w, rows, 1 + args.warmup + args.steps, seed=1)
+    warm = {s: v[:1 + args.warmup] for s, v in xs.items()}
+    oracle_run(w, warm, cores)
+    timed = {s: [v[0]] + v[1 + args.warmup:] for s, v in xs.items()}
+    dt, elems = oracle_run(w, timed, cores)
+    gbs = elems * 2 / dt / 1e9
+    sample = f"{rows} token rows of each of the {w.slots} slots, {args.steps} compressed steps"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {
+        "workload": f"{w.name}: {w.slots} slots x {w.rows} tokens x {w.cols} channels bf16, k={w.bits}, "
+                    f"G={w.group}, error feedback, {w.steps} denoising steps",
+        "slots": w.slots, "rows": w.rows, "cols": w.cols, "bits": w.bits, "group": w.group,
+        "l2": "inputs larger than L2 (every step streams the whole state)",
+    }
+
+
+def run_cf(args, w):
+    world, rank, local = dist_init()
+    import activation_residual_compression_02_b200 as cf
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shapes = [(w.rows, w.cols)] * w.slots
+    ctx = cf.Context(shapes, bits=w.bits, group=w.group)
+    st = cf.QuantState(shapes, w.bits, w.group, device=dev)
+    n_elem = w.elems
+    x_bytes = n_elem * 2
+
+    # all inputs of the run resident in HBM before timing
+    nsteps = min(w.steps, 1 + args.warmup + args.steps)
+    streams = [synth.SlotStream(w, s, seed=rank, device=dev) for s in range(w.slots)]
+    X = [[None] * w.slots for _ in range(nsteps)]
+    for s in range(w.slots):
+        for t in range(nsteps):
+            X[t][s] = streams[s].next().reshape(-1)
+        streams[s].state = None
+    del streams
+    torch.cuda.synchronize()
+
+    def x_at(i):  # step index i >= 1 cycles through the compressed steps
+        return X[1 + (i - 1) % (nsteps - 1)] if nsteps > 1 else X[0]
+
+    stream = torch.cuda.current_stream()
+    slots0 = st.slots(X[0])
+    ctx.compress(slots0, 0)
+    ctx.decompress(slots0, 0)
+    slot_lists = [st.slots(x_at(i)) for i in range(1, min(nsteps, 1 + args.warmup + args.steps))]
+    c_slots = [ctx._slots(sl) for sl in slot_lists]  # C slot arrays built once, outside the timing
+    L = cf.lib()
+    h = ctx.handle
+    sh = stream.cuda_stream
+
+    def step(i):
+        arr = c_slots[(i - 1) % len(c_slots)]
+        if L.cf_compress(h, arr, i, sh) != 0 or L.cf_decompress(h, arr, i, sh) != 0:
+            raise RuntimeError(L.cf_last_error(h).decode())
+
+    for i in range(1, args.warmup + 1):
+        step(i)
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            i = args.warmup + 1 + k
+            arr = c_slots[(i - 1) % len(c_slots)]
+            ev[k][0].record(stream)
+            if L.cf_compress(h, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+            ev[k][1].record(stream)
+            if L.cf_decompress(h, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+            ev[k][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    status = ctx.check()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world)
+    comp_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    deco_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    ms_per_step = ms / args.steps
+    value = world * x_bytes / (ms_per_step * 1e-3) / 1e9
+
+    bc, bd = alg_bytes_per_elem(w.bits, w.group)
+    peak, peak_kind = hbm_peak()
+    ach_c = bc * n_elem / (comp_ms * 1e-3) / 1e9
+    ach_d = bd * n_elem / (deco_ms * 1e-3) / 1e9
+    ach_pair = (bc + bd) * n_elem / (ms_per_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API, host buffers -----------------
+    e2e = None
+    if not args.no_e2e:
+        n_host = min(4, len(slot_lists))
+        host_x = [[X[1 + j][s].cpu().pin_memory() for s in range(w.slots)] for j in range(n_host)]
+        dev_x = [torch.empty_like(X[0][s]) for s in range(w.slots)]
+        host_codes = [torch.empty(st.codes[s].numel(), dtype=torch.uint8).pin_memory() for s in range(w.slots)]
+        host_scales = [torch.empty(st.scales[s].numel(), dtype=torch.float32).pin_memory() for s in range(w.slots)]
+        e2e_slots = st.slots(dev_x)
+        e2e_steps = max(3, min(args.steps, 20))
+        h2d = x_bytes
+        d2h = sum(c.numel() for c in host_codes) + 4 * sum(s_.numel() for s_ in host_scales)
+
+        def e2e_step(i):
+            hx = host_x[i % n_host]
+            for s in range(w.slots):
+                dev_x[s].copy_(hx[s], non_blocking=True)
+            ctx.compress(e2e_slots, i + 1, stream)
+            ctx.decompress(e2e_slots, i + 1, stream)
+            for s in range(w.slots):
+                host_codes[s].copy_(st.codes[s], non_blocking=True)
+                host_scales[s].copy_(st.scales[s], non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i + 1)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+        e2e = {"value": world * x_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "host_inputs": f"{n_host} pinned host copies of the step inputs, cycled"}
+    status = ctx.check()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+
+    # ---- CPU oracle on a bounded sample (rank 0, N = 1) -------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import numpy as np
+
+        cores = cpu_cores()
+        csteps = min(args.cpu_steps, nsteps - 1)
+        xs_host = {s: [X[t][s].view(torch.int16).cpu().numpy().view(np.uint16).copy() for t in range(1 + csteps)]
+                   for s in range(w.slots)}
+        dt, elems = oracle_run(w, xs_host, cores)
+        cpu = {"value": elems * 2 / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"the whole workload ({w.slots} slots x {w.rows} x {w.cols}) for {csteps} compressed "
+                         f"steps after the warmup (compress + decompress, {elems} elements), one slot per host "
+                         f"thread, {cores} threads, {dt:.1f} s wall"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(w),
+        "roofline": {"bound": "hbm", "kernel": "compress (residual+EF+quantise+pack, grouped)",
+                     "achieved": ach_c, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": ach_c / peak, "traffic": recorded_traffic("compress"),
+                     "alg_bytes_per_launch": bc * n_elem, "ms_per_launch": comp_ms},
+        "roofline_decompress": {"bound": "hbm", "achieved": ach_d, "peak": peak, "unit": "GB/s",
+                                "frac": ach_d / peak, "traffic": recorded_traffic("decompress"),
+                                "alg_bytes_per_launch": bd * n_elem, "ms_per_launch": deco_ms},
+        "roofline_step": {"achieved": ach_pair, "frac": ach_pair / peak, "frac_of_8tbs": ach_pair / 8000.0,
+                          "alg_bytes_per_step": (bc + bd) * n_elem},
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def run_lowrank_bench(args, w):
+    """Algorithm 3 on the low-rank workload (57 fp32 residual matrices of
+    4608 x 3072, r = 16, T = 2, Gaussian start blocks) through cf_lowrank,
+    with the error buffer E = A - U R V^T written (a step of the low-rank
+    codec's sender on given residuals)."""
+    world, rank, local = dist_init()
+    import activation_residual_compression_02_b200 as cf
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    m, n, r, T, k = w.rows, w.cols, w.rank, w.iters, w.slots
+    ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+    ws = torch.empty(ctx.lowrank_workspace_bytes(k, m, n), dtype=torch.uint8, device=dev)
+    ctx.set_workspace(ws)
+    A = [synth.lowrank_matrix(m, n, r, mat=i, seed=rank, device=dev) for i in range(k)]
+    Q0 = [synth.q0(n, r, seed=rank, mat=i, device=dev) for i in range(k)]
+    U = [torch.empty(m, r, device=dev) for _ in range(k)]
+    R = [torch.empty(r, r, device=dev) for _ in range(k)]
+    V = [torch.empty(n, r, device=dev) for _ in range(k)]
+    E = [torch.empty(m, n, device=dev) for _ in range(k)]
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        ctx.lowrank(A, Q0, U, R, V, E)
+    torch.cuda.synchronize()
+    assert ctx.check() == 0
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            ctx.lowrank(A, Q0, U, R, V, E)
+        end.record(stream)
+        torch.cuda.synchronize()
+    status = ctx.check()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    ms = max_over_ranks(start.elapsed_time(end), world) / args.steps
+    elems = k * m * n
+    peak, peak_kind = hbm_peak()
+    alg_bytes = elems * (4 + 4)          # A read once, E written once
+    flops = 2.0 * (2 * T + 1) * m * n * r * k + 2.0 * m * n * r * k
+    line = {
+        "metric": "low-rank codec GB/s of fp32 residual input (Algorithm 3 + apply)", "value":
+            world * elems * 4 / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "tf32/f64", "data": "synthetic",
+        "config": {"workload": f"lowrank: {k} matrices x {m} x {n} fp32, rank-{r} signal + 0.01 noise, r={r}, "
+                               f"T={T}, Gaussian Q0, E = A - U R V^T written",
+                   "l2": "inputs larger than L2 (3.2 GB of A per step)"},
+        "roofline": {"bound": "hbm", "kernel": "whole cf_lowrank call", "achieved": alg_bytes / (ms * 1e-3) / 1e9,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": alg_bytes / (ms * 1e-3) / 1e9 / peak, "traffic": None,
+                     "alg_bytes_per_step": alg_bytes, "tflops": flops / (ms * 1e-3) / 1e12},
+        "gpu_launches": None, "e2e": None, "cpu_baseline": None, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cf", "reference"], default="cf")
+    ap.add_argument("--workload", default="flux", choices=["flux", "cogvideox", "stress", "tiny", "lowrank"])
+    ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--slots", type=int, default=None, help="override the slot count (profiling a smaller case)")
+    ap.add_argument("--budget", type=float, default=120.0, help="seconds of oracle work for --impl reference")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = synth.WORKLOADS[args.workload]
+    if args.slots:
+        w = w.scaled(slots=args.slots)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    if w.mode == 1:
+        return run_lowrank_bench(args, w)
+    return run_cf(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

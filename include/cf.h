@@ -1,0 +1,206 @@
+/*
+ * cf.h -- C ABI of the B200 residual-compression activation codec (libcf).
+ *
+ * What the codec computes (page titles and sections):
+ *  - "Accelerating Parallel Diffusion Model Serving with Residual Compression"
+ *    (arXiv 2507.17511), abstract: between parallel devices, send only the
+ *    compressed step-wise residual of each activation, and carry the
+ *    compression error forward (error feedback) so that it does not
+ *    accumulate across denoising steps.
+ *  - Same paper, reproducibility table, "Dataset Splits" row (Appendix D,
+ *    Figure 8): at least one uncompressed warmup step initialises the base
+ *    tensor that later residuals are taken against.
+ *  - Same paper, reproducibility table, "Pseudocode" row, Algorithm 3
+ *    (Subspace Iteration, rank r): the low-rank compressor.
+ *  - xDiT issue 573 ("Proposal: Integrating a compression-based acceleration
+ *    method into xDiT"): residuals plus error feedback, 8-16x less traffic.
+ *
+ * Per communicated tensor ("slot": one layer's activation shard, or its K or
+ * its V) and per denoising step t:
+ *   sender    A   = (X_t - base) + E          residual plus carried error
+ *             payload = Q(A)                   k-bit group codes + fp32 scales,
+ *                                              or rank-r factors (U, R, V)
+ *             E   = A - deq(payload)           new carried error
+ *             base = X_t
+ *   receiver  C   = C + deq(payload)           reconstruction cache
+ * Step 0 is the uncompressed warmup: base = X_0, E = 0 and C = X_0.  Then
+ * C_t + E_t = X_t holds at every step, up to fp32 rounding.
+ *
+ * Quantiser (the pages give no formula; these are the readings this library
+ * takes): groups of G contiguous channels of one token row;
+ *   k = 2, 4: s = max|A| over the group, L = 2^(k-1)-1, inv = L/s,
+ *             code = clamp(rne(A*inv), -L, L) + L, deq = ((code-L)/L)*s;
+ *   k = 1   : code = (A >= 0), deq = code ? s : -s, with
+ *             s = (binary-tree sum of |A|)/G (sign_scale 0, the default) or
+ *             s = max|A| (sign_scale 1).
+ * A group whose scale is below 2^-120, or not finite, is sent as an all-zero
+ * group (scale 0, every code the zero level); a non-finite scale also raises
+ * CF_E_NONFINITE at the next cf_check.  Every floating-point step is one
+ * IEEE-754 binary32 operation with round-to-nearest-even and no fused
+ * multiply-add, so results are bit-reproducible.
+ *
+ * Layouts (all row-major, token rows of `cols` channels, flat index
+ * i = row*cols + col):
+ *   x, base  bf16 [rows*cols]          err, cache  fp32 [rows*cols]
+ *   codes    u8 [rows*cols*k/8]: one LSB-first bit stream; the code of
+ *            element i occupies bits [i*k, i*k+k).  Group g = i/G starts at
+ *            byte g*G*k/8.
+ *   scales   fp32 [rows*cols/G], scales[g] for group g.
+ *   low-rank payload: U fp32 [rows x r], R fp32 [r x r] (upper triangular),
+ *            V fp32 [cols x r]; the reconstruction is U R V^T.
+ *
+ * Ownership: the library owns only the context, its device status word and
+ * host-side bookkeeping.  Activations, state (base, err, cache), payloads and
+ * the workspace are caller memory (device pointers).  The library performs
+ * no transmission between devices.
+ *
+ * Concurrency and errors: every call except cf_create, cf_destroy and
+ * cf_check is stream-ordered and asynchronous.  Argument, shape, alignment
+ * and state errors return before anything is launched and leave all buffers
+ * untouched.  Device-side conditions (non-finite scale, a bounded wait that
+ * gave up) set bits in the context's status word and are reported by the
+ * next cf_check.  A context is not thread-safe; separate contexts are
+ * independent.  There is no CPU fallback: without a usable sm_100 device
+ * cf_create returns CF_E_CUDA.
+ */
+#ifndef CF_H
+#define CF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct cf_ctx cf_ctx;
+
+typedef enum cf_status {
+    CF_OK = 0,
+    CF_E_ARG = 1,        /* bad argument value (null pointer, unsupported k/G/r, ...) */
+    CF_E_SHAPE = 2,      /* shape not allowed (cols % G, cols % 8, rows < r, ...) */
+    CF_E_ALIGN = 3,      /* pointer not 16-byte aligned */
+    CF_E_STATE = 4,      /* step > 0 before the warmup step on this context */
+    CF_E_NOMEM = 5,      /* host or device allocation failed, or workspace too small */
+    CF_E_CUDA = 6,       /* CUDA runtime error (launch, no device, wrong arch) */
+    CF_E_NONFINITE = 7,  /* a group scale or a Gram matrix was not finite / not SPD */
+    CF_E_TIMEOUT = 8     /* a bounded device-side wait gave up */
+} cf_status;
+
+enum { CF_MODE_QUANT = 0, CF_MODE_LOWRANK = 1 };
+
+typedef struct cf_config {
+    int mode;        /* CF_MODE_QUANT or CF_MODE_LOWRANK */
+    int bits;        /* quant: k = 1, 2 or 4 */
+    int group;       /* quant: G = 8, 16, 32, 64, 128 or 256; must divide cols */
+    int sign_scale;  /* k = 1: 0 = mean |A| scale (default), 1 = absmax scale */
+    int rank;        /* low-rank: r, 1..32 */
+    int iters;       /* low-rank: T >= 0 subspace iterations */
+} cf_config;
+
+typedef struct cf_shape {
+    int64_t rows;    /* tokens of this slot's shard (>= 0) */
+    int64_t cols;    /* channels (> 0, multiple of 8) */
+} cf_shape;
+
+/* Per-slot device pointers for one call; all 16-byte aligned, all caller
+ * owned.  Fields a call does not use may be NULL (see each call), and so may
+ * every field of a slot with rows == 0. */
+typedef struct cf_slot {
+    const void *x;   /* bf16 [rows*cols]  activation X_t (read only) */
+    void *base;      /* bf16 [rows*cols]  sender's base tensor X_{t-1} */
+    float *err;      /* fp32 [rows*cols]  sender's error-feedback buffer E */
+    float *cache;    /* fp32 [rows*cols]  receiver's reconstruction C */
+    uint8_t *codes;  /* quant payload codes, rows*cols*k/8 bytes */
+    float *scales;   /* quant payload scales, rows*cols/G */
+    const float *q0; /* low-rank: Gaussian start block [cols x r] for this call */
+    float *U;        /* low-rank payload [rows x r] */
+    float *R;        /* low-rank payload [r x r] */
+    float *V;        /* low-rank payload [cols x r] */
+} cf_slot;
+
+/* Create a context for `nslots` slots of the given shapes (host array).
+ * Validates the configuration and the shapes, checks that device 0 of the
+ * current CUDA context is sm_100, and allocates the device status word.
+ * nslots may be 0 for a context used only with cf_lowrank.
+ * Errors: CF_E_ARG, CF_E_SHAPE, CF_E_NOMEM, CF_E_CUDA; *out is NULL then. */
+cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes, cf_ctx **out);
+
+/* Device workspace cf_compress needs for this context, in bytes (0 in
+ * quantised mode; in low-rank mode the fp32 residuals of every slot plus the
+ * small per-slot buffers of Algorithm 3). */
+size_t cf_workspace_bytes(const cf_ctx *ctx);
+
+/* Register caller-owned device workspace (16-byte aligned) used by
+ * cf_compress / cf_lowrank until replaced.  Errors: CF_E_ALIGN, CF_E_NOMEM
+ * (smaller than cf_workspace_bytes). */
+cf_status cf_set_workspace(cf_ctx *ctx, void *dev_ptr, size_t bytes);
+
+/* Sender side of step `step` for every slot, in one grouped launch.
+ *   step 0: warmup -- base = x, err = 0.  Uses x, base, err.
+ *   step >= 1, quantised: A = (x - base) + err; codes, scales = Q(A);
+ *           err = A - deq; base = x.  Uses x, base, err, codes, scales.
+ *   step >= 1, low-rank: A as above into the workspace; Algorithm 3 with
+ *           start block q0 gives U, R, V; err = A - U R V^T; base = x.
+ *           Uses x, base, err, q0, U, R, V.
+ * `slots` is a host array of nslots entries; `cuda_stream` a cudaStream_t
+ * (NULL = legacy default stream).  Errors before launch: CF_E_ARG,
+ * CF_E_ALIGN, CF_E_STATE (step >= 1 before a warmup), CF_E_NOMEM (workspace
+ * missing in low-rank mode); CF_E_CUDA if a launch fails. */
+cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
+
+/* Receiver side of step `step` for every slot, in one grouped launch.
+ *   step 0: warmup -- cache = float(x).  Uses x, cache.
+ *   step >= 1, quantised: cache += deq(codes, scales).  Uses codes, scales,
+ *           cache.
+ *   step >= 1, low-rank: cache += U R V^T.  Uses U, R, V, cache.
+ * Errors as cf_compress (CF_E_STATE: step >= 1 before a receiver warmup). */
+cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
+
+/* Workspace cf_lowrank needs for nmat matrices of m x n at this context's
+ * rank: the r-column blocks of Algorithm 3 (Q^T, P^T, P, Z, padded to 16 or
+ * 32 columns) and their fp64 Gram matrices, about 4*rp*(2m + 2n) + 8 KB
+ * bytes per matrix.  Returns 0 for a quantised-mode context or bad sizes. */
+size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_t n);
+
+/* Algorithm 3 (subspace iteration, rank r = config.rank, T = config.iters
+ * iterations, CholeskyQR orthogonalisation) on nmat given fp32 matrices.
+ * All pointer arguments are HOST arrays of nmat DEVICE pointers:
+ *   A[i]  fp32 [m x n] row-major (read only; n % 4 == 0)
+ *   Q0[i] fp32 [n x r] Gaussian start block (read only)
+ *   U[i]  fp32 [m x r]  R[i] fp32 [r x r]  V[i] fp32 [n x r]  (written)
+ *   E_opt NULL or E[i] fp32 [m x n]: E = A - U R V^T       (written)
+ *   C_opt NULL or C[i] fp32 [m x n]: C += U R V^T          (updated)
+ * Uses the registered workspace (>= cf_lowrank_workspace_bytes).  The two
+ * products with A (A Q and A^T P) run on the tensor cores in TF32 with
+ * operands rounded to nearest; Gram matrices and Cholesky run in fp64.
+ * Errors before launch: CF_E_ARG, CF_E_SHAPE (m < r, n < r, n % 4),
+ * CF_E_ALIGN, CF_E_NOMEM; device-side: CF_E_NONFINITE (Gram matrix not
+ * positive definite), CF_E_TIMEOUT, at the next cf_check. */
+cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *const *A,
+                     const float *const *Q0, float *const *U, float *const *R, float *const *V,
+                     float *const *E_opt, float *const *C_opt, void *cuda_stream);
+
+/* Synchronise `cuda_stream`, read and clear the device status word.
+ * Returns CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or CF_E_CUDA (an asynchronous
+ * CUDA error, e.g. from an earlier launch). */
+cf_status cf_check(cf_ctx *ctx, void *cuda_stream);
+
+/* Payload bytes of slot `slot` per compressed step: rows*cols*k/8 +
+ * 4*rows*cols/G (quantised) or 4*r*(rows + r + cols) (low-rank); 0 for a bad
+ * slot index. */
+size_t cf_payload_bytes(const cf_ctx *ctx, int slot);
+
+/* Human-readable message of the last error on this context ("" if none).
+ * The string is owned by the context. */
+const char *cf_last_error(const cf_ctx *ctx);
+
+/* Free the context (waits for nothing; the caller must not destroy a
+ * context while its launches are still running on a stream). */
+cf_status cf_destroy(cf_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CF_H */

@@ -1,0 +1,193 @@
+"""GPU parity of the low-rank path (Algorithm 3) against the fp64 CPU oracle.
+
+The factors (U, R, V) are unique only up to rotations within the subspace, so
+the comparison is on what is unique: the reconstruction D = U R V^T, the new
+error E = A - D and the updated cache C + D, each within 1e-3 relative
+Frobenius of the oracle's (the tolerance of the low-rank path; TF32 operands
+rounded to nearest give about 3e-5 on the low-rank workload).  U and V must
+also be orthonormal.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def cf():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import activation_residual_compression_02_b200 as m
+
+    m.lib()
+    return m
+
+
+def run_gpu(cf, As, Q0s, r, T, with_e=True, with_c=True):
+    m, n = As[0].shape
+    ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+    ws = torch.empty(ctx.lowrank_workspace_bytes(len(As), m, n), dtype=torch.uint8, device="cuda")
+    ctx.set_workspace(ws)
+    A = [a.cuda() for a in As]
+    Q0 = [q.cuda() for q in Q0s]
+    U = [torch.empty(m, r, device="cuda") for _ in As]
+    R = [torch.empty(r, r, device="cuda") for _ in As]
+    V = [torch.empty(n, r, device="cuda") for _ in As]
+    E = [torch.empty(m, n, device="cuda") for _ in As] if with_e else None
+    C0 = [torch.randn(m, n, generator=torch.Generator().manual_seed(i)) for i in range(len(As))] if with_c else None
+    C = [c.cuda() for c in C0] if with_c else None
+    ctx.lowrank(A, Q0, U, R, V, E, C)
+    st = ctx.check()
+    assert st == cf.CF_OK, st
+    out = dict(U=[u.cpu().double().numpy() for u in U], R=[x.cpu().double().numpy() for x in R],
+               V=[v.cpu().double().numpy() for v in V])
+    if with_e:
+        out["E"] = [e.cpu().double().numpy() for e in E]
+    if with_c:
+        out["C"] = [c.cpu().double().numpy() for c in C]
+        out["C0"] = [c.numpy() for c in C0]
+    ctx.close()
+    return out
+
+
+def rel(a, b, ref):
+    return np.linalg.norm(a - b) / np.linalg.norm(ref)
+
+
+def check(oracle, As, Q0s, out, T, idx=None):
+    idx = range(len(As)) if idx is None else idx
+    for i in idx:
+        A = As[i].numpy()
+        Uo, Ro, Vo = oracle.subspace_iteration(A, Q0s[i].numpy(), T)
+        C0 = out["C0"][i] if "C0" in out else None
+        Do, Eo, Co = oracle.lowrank_apply(A, Uo, Ro, Vo, C0)
+        U, R, V = out["U"][i], out["R"][i], out["V"][i]
+        r = U.shape[1]
+        Dg = U @ R @ V.T
+        assert rel(Dg, Do, Do) <= TOL, (i, rel(Dg, Do, Do))
+        assert np.abs(U.T @ U - np.eye(r)).max() < 1e-4
+        assert np.abs(V.T @ V - np.eye(r)).max() < 1e-4
+        assert np.allclose(R, np.triu(R))
+        if "E" in out:
+            assert rel(out["E"][i], Eo, Do) <= TOL, i
+        if "C" in out:
+            assert rel(out["C"][i], Co, Do) <= TOL, i
+
+
+@pytest.mark.parametrize("m,n,r,T", [(256, 256, 16, 2), (300, 200, 16, 2), (4444 // 4, 1920 // 4, 16, 2),
+                                     (200, 72, 8, 2), (160, 96, 24, 1), (192, 128, 32, 2), (130, 64, 16, 0),
+                                     (128, 128, 1, 3)])
+def test_lowrank_matches_oracle(cf, oracle, m, n, r, T):
+    k = 3
+    As = [synth.lowrank_matrix(m, n, r, mat=i, noise=0.01) for i in range(k)]
+    Q0s = [synth.q0(n, r, seed=0, mat=i) for i in range(k)]
+    out = run_gpu(cf, As, Q0s, r, T)
+    check(oracle, As, Q0s, out, T)
+
+
+def test_lowrank_many_matrices_chunked(cf, oracle):
+    """More matrices than one launch's descriptor table holds."""
+    m, n, r, T = 128, 96, 8, 2
+    k = 45
+    As = [synth.lowrank_matrix(m, n, r, mat=i, noise=0.01) for i in range(k)]
+    Q0s = [synth.q0(n, r, seed=0, mat=i) for i in range(k)]
+    out = run_gpu(cf, As, Q0s, r, T, with_c=False)
+    check(oracle, As, Q0s, out, T, idx=[0, 39, 40, 44])
+
+
+def test_lowrank_exact_rank_recovered(cf):
+    """An exactly rank-r matrix is reconstructed to TF32 accuracy."""
+    m, n, r = 512, 384, 16
+    As = [synth.lowrank_matrix(m, n, r, mat=7, noise=0.0)]
+    Q0s = [synth.q0(n, r, seed=0, mat=7)]
+    out = run_gpu(cf, As, Q0s, r, 2, with_c=False)
+    D = out["U"][0] @ out["R"][0] @ out["V"][0].T
+    A = As[0].double().numpy()
+    assert np.linalg.norm(D - A) / np.linalg.norm(A) < 1e-4
+
+
+def test_lowrank_full_size_sampled(cf, oracle):
+    """The low-rank workload at full size (57 x 4608 x 3072, r = 16, T = 2) in
+    one call; the oracle re-runs three of the matrices."""
+    w = synth.LOWRANK
+    m, n, r = w.rows, w.cols, w.rank
+    ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=w.iters)
+    ws = torch.empty(ctx.lowrank_workspace_bytes(w.slots, m, n), dtype=torch.uint8, device="cuda")
+    ctx.set_workspace(ws)
+    A = [synth.lowrank_matrix(m, n, r, mat=i, device="cuda") for i in range(w.slots)]
+    Q0 = [synth.q0(n, r, seed=0, mat=i, device="cuda") for i in range(w.slots)]
+    U = [torch.empty(m, r, device="cuda") for _ in A]
+    R = [torch.empty(r, r, device="cuda") for _ in A]
+    V = [torch.empty(n, r, device="cuda") for _ in A]
+    E = [torch.empty(m, n, device="cuda") for _ in A]
+    ctx.lowrank(A, Q0, U, R, V, E)
+    assert ctx.check() == cf.CF_OK
+    for i in (0, w.slots // 2, w.slots - 1):
+        Ah = A[i].cpu().numpy()
+        Uo, Ro, Vo = oracle.subspace_iteration(Ah, Q0[i].cpu().numpy(), w.iters)
+        Do, Eo, _ = oracle.lowrank_apply(Ah, Uo, Ro, Vo)
+        Dg = U[i].cpu().double().numpy() @ R[i].cpu().double().numpy() @ V[i].cpu().double().numpy().T
+        assert rel(Dg, Do, Do) <= TOL
+        assert rel(E[i].cpu().double().numpy(), Eo, Do) <= TOL
+    ctx.close()
+
+
+def test_lowrank_mode_through_slots(cf, oracle):
+    """cf_compress / cf_decompress in low-rank mode: residual + error feedback
+    into Algorithm 3, E and the receiver cache updated, base advanced."""
+    rows, cols, r, T = 192, 256, 16, 2
+    shapes = [(rows, cols), (rows, cols)]
+    ctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+    ws = torch.empty(max(ctx.workspace_bytes(), 16), dtype=torch.uint8, device="cuda")
+    ctx.set_workspace(ws)
+    # activations whose step-wise change is (nearly) rank r, so that the
+    # rank-r payload captures the residual and the comparison is well posed
+    xs = []
+    for i in range(2):
+        x = synth.gaussian((rows, cols), 0, i, 99)
+        seq = [x.to(torch.bfloat16)]
+        for t in range(1, 3):
+            L = synth.lowrank_matrix(rows, cols, r, mat=100 * i + t, noise=0.0)
+            x = seq[-1].float() + 0.5 * L / L.pow(2).mean().sqrt()
+            seq.append(x.to(torch.bfloat16))
+        xs.append(seq)
+    base = [torch.empty(rows * cols, dtype=torch.bfloat16, device="cuda") for _ in shapes]
+    err = [torch.empty(rows * cols, device="cuda") for _ in shapes]
+    cache = [torch.empty(rows * cols, device="cuda") for _ in shapes]
+    U = [torch.empty(rows, r, device="cuda") for _ in shapes]
+    R = [torch.empty(r, r, device="cuda") for _ in shapes]
+    V = [torch.empty(cols, r, device="cuda") for _ in shapes]
+    ob = [None, None]
+    oe = [None, None]
+    oc = [None, None]
+    for t in range(3):
+        q0 = [synth.q0(cols, r, seed=0, mat=i, call=t) for i in range(2)]
+        slots = [cf.Slot(x=xs[i][t].reshape(-1).cuda(), base=base[i], err=err[i], cache=cache[i], q0=q0[i].cuda(),
+                         U=U[i], R=R[i], V=V[i]) for i in range(2)]
+        ctx.compress(slots, t)
+        ctx.decompress(slots, t)
+        for i in range(2):
+            xb = xs[i][t].view(torch.int16).numpy().view(np.uint16).ravel().copy()
+            if t == 0:
+                ob[i], oe[i] = oracle.warmup_sender(xb)
+                oc[i] = oracle.warmup_receiver(xb).astype(np.float64)
+                continue
+            a = oracle.residual(xb, ob[i], oe[i]).reshape(rows, cols)
+            Uo, Ro, Vo = oracle.subspace_iteration(a, q0[i].numpy(), T)
+            Do, Eo, _ = oracle.lowrank_apply(a, Uo, Ro, Vo)
+            torch.cuda.synchronize()
+            eg = err[i].cpu().double().numpy().reshape(rows, cols)
+            assert rel(eg, Eo, Do) <= TOL, (t, i)
+            oc[i] = oc[i] + Do.ravel()
+            assert rel(cache[i].cpu().double().numpy(), oc[i], Do) <= TOL, (t, i)
+            assert np.array_equal(base[i].view(torch.int16).cpu().numpy().view(np.uint16), xb)
+            # continue the oracle from the GPU's error buffer (E is unique only to 1e-3)
+            oe[i] = err[i].cpu().numpy().copy()
+    assert ctx.check() == cf.CF_OK
+    for i in range(2):
+        x = xs[i][2].float().reshape(-1).cuda()
+        assert (torch.linalg.vector_norm(cache[i] + err[i] - x) / torch.linalg.vector_norm(x)).item() < 1e-5

@@ -1,0 +1,209 @@
+"""GPU parity of the quantised codec against the CPU oracle (through the C ABI).
+
+Codes and scales must be bit-exact; so must E, base and the receiver cache,
+because every floating-point step on both sides is a single IEEE binary32
+operation with round-to-nearest-even.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cf():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import activation_residual_compression_02_b200 as m
+
+    m.lib()
+    return m
+
+
+def u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+
+
+def run_case(cf, oracle, shapes, steps, bits, group, ss=0, seed=0, w=synth.TINY, check_every_step=True):
+    """Run the codec on the GPU and the oracle on the CPU for `steps` steps."""
+    ctx = cf.Context(shapes, bits=bits, group=group, sign_scale=ss)
+    st = cf.QuantState(shapes, bits, group)
+    streams = [synth.SlotStream(w.scaled(rows=r, cols=c), slot=i, seed=seed) for i, (r, c) in enumerate(shapes)]
+    ors = [oracle.QuantSlot(bits, group, ss) for _ in shapes]
+    for t in range(steps):
+        xs_cpu = [s.next() for s in streams]
+        xs = [x.cuda() for x in xs_cpu]
+        slots = st.slots(xs)
+        ctx.compress(slots, t)
+        ctx.decompress(slots, t)
+        for i, x in enumerate(xs_cpu):
+            ors[i].step(t, u16(x))
+        if check_every_step or t == steps - 1:
+            torch.cuda.synchronize()
+            for i in range(len(shapes)):
+                o = ors[i]
+                assert np.array_equal(u16(st.base[i]), o.base), (t, i, "base")
+                assert np.array_equal(st.err[i].cpu().numpy(), o.err), (t, i, "err")
+                assert np.array_equal(st.cache[i].cpu().numpy(), o.cache), (t, i, "cache")
+                if t > 0:
+                    assert np.array_equal(st.codes[i].cpu().numpy(), o.codes), (t, i, "codes")
+                    assert np.array_equal(st.scales[i].cpu().numpy(), o.scales), (t, i, "scales")
+    assert ctx.check() == cf.CF_OK
+    ctx.close()
+
+
+@pytest.mark.parametrize("bits,group,ss", [(2, 128, 0), (4, 64, 0), (1, 128, 0), (1, 128, 1), (2, 8, 0), (2, 16, 0),
+                                           (4, 32, 0), (4, 256, 0), (1, 8, 0), (1, 256, 1), (2, 256, 0), (4, 8, 0)])
+def test_tiny_workload_bit_exact(cf, oracle, bits, group, ss):
+    run_case(cf, oracle, [(256, 512)], 4, bits, group, ss)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 128), (4, 64), (1, 128)])
+def test_ragged_multi_slot_grouped_launch(cf, oracle, bits, group):
+    """Several slots of different sizes in one grouped launch: tails that end
+    inside a tile, inside a warp, single rows, and an empty slot."""
+    shapes = [(37, 512), (1, 256), (0, 256), (300, 768), (5, 1024), (129, 256)]
+    shapes = [(r, c) for r, c in shapes if c % group == 0]
+    run_case(cf, oracle, shapes, 4, bits, group, w=synth.COGVIDEOX)
+
+
+def test_grouped_equals_per_slot(cf):
+    """Launch-shape invariance: one grouped launch over all slots equals one
+    context (and launch) per slot, bit for bit."""
+    shapes = [(64, 512), (33, 1024), (128, 256)]
+    bits, group = 2, 128
+    xs_steps = [[x.cuda() for x in synth.activations(synth.FLUX.scaled(rows=r, cols=c), i, 3)] for i, (r, c) in
+                enumerate(shapes)]
+    ctx = cf.Context(shapes, bits=bits, group=group)
+    st = cf.QuantState(shapes, bits, group)
+    for t in range(3):
+        slots = st.slots([xs_steps[i][t] for i in range(len(shapes))])
+        ctx.compress(slots, t)
+        ctx.decompress(slots, t)
+    singles = []
+    for i, sh in enumerate(shapes):
+        c1 = cf.Context([sh], bits=bits, group=group)
+        s1 = cf.QuantState([sh], bits, group)
+        for t in range(3):
+            sl = s1.slots([xs_steps[i][t]])
+            c1.compress(sl, t)
+            c1.decompress(sl, t)
+        singles.append(s1)
+    torch.cuda.synchronize()
+    for i in range(len(shapes)):
+        for f in ("base", "err", "cache", "codes", "scales"):
+            assert torch.equal(getattr(st, f)[i], getattr(singles[i], f)[0]), (i, f)
+
+
+def test_constant_group_round_trip(cf):
+    """A constant residual reconstructs exactly: E = 0 and C = X."""
+    shapes = [(16, 256)]
+    for bits in (1, 2, 4):
+        ctx = cf.Context(shapes, bits=bits, group=64)
+        st = cf.QuantState(shapes, bits, 64)
+        x0 = torch.full((16 * 256,), 1.0, dtype=torch.bfloat16, device="cuda")
+        x1 = torch.full((16 * 256,), 1.75, dtype=torch.bfloat16, device="cuda")
+        for t, x in enumerate((x0, x1)):
+            sl = st.slots([x])
+            ctx.compress(sl, t)
+            ctx.decompress(sl, t)
+        torch.cuda.synchronize()
+        assert torch.all(st.err[0] == 0)
+        assert torch.equal(st.cache[0], x1.float())
+        assert torch.all(st.scales[0] == 0.75)
+
+
+def test_nonfinite_sets_status(cf):
+    shapes = [(4, 128)]
+    ctx = cf.Context(shapes, bits=2, group=64)
+    st = cf.QuantState(shapes, 2, 64)
+    x0 = torch.zeros(512, dtype=torch.bfloat16, device="cuda")
+    x1 = x0.clone()
+    x1[70] = float("inf")
+    for t, x in enumerate((x0, x1)):
+        sl = st.slots([x])
+        ctx.compress(sl, t)
+        ctx.decompress(sl, t)
+    assert ctx.check() == cf.CF_E_NONFINITE
+    # the flag was cleared by the read
+    assert ctx.check() == cf.CF_OK
+    torch.cuda.synchronize()
+    assert st.scales[0][1].item() == 0.0       # the group holding the inf is sent as zero
+
+
+def test_argument_errors_launch_nothing(cf):
+    shapes = [(8, 128)]
+    with pytest.raises(cf.CfError) as e:
+        cf.Context(shapes, bits=3, group=128)
+    assert e.value.status == cf.CF_E_ARG
+    with pytest.raises(cf.CfError) as e:
+        cf.Context([(8, 100)], bits=2, group=128)
+    assert e.value.status == cf.CF_E_SHAPE
+    ctx = cf.Context(shapes, bits=2, group=128)
+    st = cf.QuantState(shapes, 2, 128)
+    x = torch.zeros(1024, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cf.CfError) as e:          # compressed step before the warmup
+        ctx.compress(st.slots([x]), 1)
+    assert e.value.status == cf.CF_E_STATE
+    raw = torch.zeros(1024 + 8, dtype=torch.bfloat16, device="cuda")
+    bad = cf.Slot(x=raw[1:1025], base=st.base[0], err=st.err[0])  # 2-byte offset: misaligned
+    with pytest.raises(cf.CfError) as e:
+        ctx.compress([bad], 0)
+    assert e.value.status == cf.CF_E_ALIGN
+    with pytest.raises(cf.CfError) as e:
+        ctx.compress([cf.Slot(x=x, base=None, err=st.err[0])], 0)
+    assert e.value.status == cf.CF_E_ARG
+    assert ctx.check() == cf.CF_OK
+    assert ctx.payload_bytes(0) == 1024 * 2 // 8 + 4 * (1024 // 128)
+
+
+# ------------------------------------------------ full-size sampled parity
+
+FULL = [
+    ("flux", synth.FLUX, 3),
+    ("cogvideox", synth.COGVIDEOX, 3),
+]
+
+
+@pytest.mark.parametrize("name,w,steps", FULL)
+def test_full_size_sampled_rows_bit_exact(cf, oracle, name, w, steps):
+    """Full-size workload in the benchmark's launch configuration (one grouped
+    launch per step over every slot); the oracle recomputes sampled token rows
+    of sampled slots (rows are independent in the quantised path)."""
+    shapes = [(w.rows, w.cols)] * w.slots
+    ctx = cf.Context(shapes, bits=w.bits, group=w.group)
+    st = cf.QuantState(shapes, w.bits, w.group)
+    streams = [synth.SlotStream(w, i, seed=0, device="cuda") for i in range(w.slots)]
+    sample_slots = sorted({0, w.slots // 2, w.slots - 1})
+    sample_rows = sorted({0, 1, w.rows // 3, w.rows - 1})
+    ors = {(s, r): oracle.QuantSlot(w.bits, w.group) for s in sample_slots for r in sample_rows}
+    C = w.cols
+    for t in range(steps):
+        xs = [s.next() for s in streams]
+        slots = st.slots(xs)
+        ctx.compress(slots, t)
+        ctx.decompress(slots, t)
+        torch.cuda.synchronize()
+        for s in sample_slots:
+            xrow = xs[s].view(w.rows, C)
+            for r in sample_rows:
+                o = ors[(s, r)]
+                o.step(t, u16(xrow[r]))
+                sl = slice(r * C, (r + 1) * C)
+                assert np.array_equal(st.err[s][sl].cpu().numpy(), o.err), (t, s, r)
+                assert np.array_equal(st.cache[s][sl].cpu().numpy(), o.cache), (t, s, r)
+                assert np.array_equal(u16(st.base[s][sl]), o.base), (t, s, r)
+                if t > 0:
+                    cb = C * w.bits // 8
+                    assert np.array_equal(st.codes[s][r * cb:(r + 1) * cb].cpu().numpy(), o.codes), (t, s, r)
+                    gs = C // w.group
+                    assert np.array_equal(st.scales[s][r * gs:(r + 1) * gs].cpu().numpy(), o.scales), (t, s, r)
+    # property at every element: C + E = X (EF identity), relative L2 <= 1e-6
+    for s in sample_slots:
+        x = xs[s].float().reshape(-1)
+        rel = torch.linalg.vector_norm(st.cache[s] + st.err[s] - x) / torch.linalg.vector_norm(x)
+        assert rel.item() <= 1e-6
+    assert ctx.check() == cf.CF_OK
