@@ -132,7 +132,6 @@ cf_status check_quant_slot(cf_ctx *ctx, const cf_slot &s, int i, bool sender, in
 cf_status run_quant(cf_ctx *ctx, const cf_slot *slots, cf::QuantOp op, cudaStream_t stream)
 {
     const int n = (int)ctx->shapes.size();
-    const int64_t tile = cf::quant_tile_elems();
     cf::QuantLaunch *lp = new (std::nothrow) cf::QuantLaunch;
     if (!lp) return fail(ctx, CF_E_NOMEM, "host allocation failed");
     for (int first = 0; first < n; first += cf::kMaxSlotsPerLaunch) {
@@ -140,7 +139,6 @@ cf_status run_quant(cf_ctx *ctx, const cf_slot *slots, cf::QuantOp op, cudaStrea
         memset(lp, 0, sizeof *lp);
         lp->nslots = cnt;
         lp->status = ctx->d_status;
-        int64_t tiles = 0;
         for (int k = 0; k < cnt; ++k) {
             const cf_slot &s = slots[first + k];
             const cf_shape &sh = ctx->shapes[first + k];
@@ -153,10 +151,7 @@ cf_status run_quant(cf_ctx *ctx, const cf_slot *slots, cf::QuantOp op, cudaStrea
             d.codes = s.codes;
             d.scales = s.scales;
             d.nvec = elems / 8;
-            d.tile0 = tiles;
-            tiles += (elems + tile - 1) / tile;
         }
-        lp->ntiles = tiles;
         cudaError_t e = cf::launch_quant(op, ctx->cfg.bits, ctx->cfg.group, ctx->cfg.sign_scale, *lp, stream);
         if (e != cudaSuccess) {
             delete lp;

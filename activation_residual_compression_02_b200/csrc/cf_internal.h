@@ -29,7 +29,7 @@ struct QuantSlotDesc {
     uint8_t *codes;    // packed codes
     float *scales;     // fp32 group scales
     int64_t nvec;      // elements / 8
-    int64_t tile0;     // first tile index of this slot in the launch
+    int64_t tile0;     // first tile index of this slot in the launch (set by launch_quant)
 };
 
 struct QuantLaunch {
@@ -42,14 +42,11 @@ struct QuantLaunch {
 
 enum class QuantOp { WarmupSender, WarmupReceiver, Compress, Decompress };
 
-// Elements per tile of the quantised kernels (one tile = one CTA iteration).
-int64_t quant_tile_elems();
-
-// Launch one grouped quantised kernel over `lp` (host-built).  bits/group/
-// sign_scale select the template instance.  Returns cudaSuccess or the launch
-// error.
-cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, const QuantLaunch &lp,
-                         cudaStream_t stream);
+// Launch one grouped quantised kernel over `lp` (host-built slot table;
+// tile0/ntiles are filled in here for the chosen kernel's tile size).
+// bits/group/sign_scale select the template instance.  Returns cudaSuccess or
+// the launch error.
+cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, QuantLaunch &lp, cudaStream_t stream);
 
 // ---------------------------------------------------------------- low rank
 

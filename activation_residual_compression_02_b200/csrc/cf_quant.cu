@@ -23,10 +23,14 @@
 // magnitude bits (exact, and a NaN or infinity is seen as non-finite).
 #include <cuda_bf16.h>
 
+#include <stdlib.h>
+#include <string.h>
+
 #include <mutex>
 #include <unordered_map>
 
 #include "cf_internal.h"
+#include "cf_ptx.cuh"
 
 namespace cf {
 namespace {
@@ -270,52 +274,310 @@ __global__ void __launch_bounds__(kThreads) k_quant(const __grid_constant__ Quan
     }
 }
 
+// ------------------------------------------------ TMA-staged variant ----
+// The same arithmetic as k_quant, but the input streams are staged through
+// shared memory by one producer thread with bulk-async copies (TMA,
+// cp.async.bulk, no tensor map), so that a CTA always has kTmaStages - 1
+// tiles in flight without spending registers on them.  Compress stages x,
+// base and err (64 B per vector); decompress stages the cache (32 B per
+// vector) and loads the small codes/scales directly before it waits.
+constexpr int kTmaConsumers = 256;               // 8 consumer warps
+constexpr int kTmaThreads = kTmaConsumers + 32;  // + 1 producer warp
+constexpr int kTmaVec = 512;                     // vectors per tile (= one stage)
+constexpr int kTmaStages = 3;
+constexpr unsigned long long kQuantWaitNs = 2000000000ull;
+
+template <QuantOp OP>
+__host__ __device__ constexpr int tma_bytes_per_vec()
+{
+    return OP == QuantOp::Compress ? 64 : 32;
+}
+
+struct TmaBarriers {
+    uint64_t full[kTmaStages];
+    uint64_t empty[kTmaStages];
+    int abort_flag;
+};
+
+template <QuantOp OP>
+constexpr size_t tma_smem_bytes()
+{
+    return (size_t)kTmaStages * kTmaVec * tma_bytes_per_vec<OP>() + sizeof(TmaBarriers);
+}
+
+template <QuantOp OP, int K, int G, int SS>
+__global__ void __launch_bounds__(kTmaThreads) k_quant_tma(const __grid_constant__ QuantLaunch p)
+{
+    using namespace ptx;
+    constexpr int LPG = G / 8;
+    constexpr int L = (K >= 2) ? (1 << (K - 1)) - 1 : 1;
+    constexpr int BPV = tma_bytes_per_vec<OP>();
+    constexpr int kStageBytes = kTmaVec * BPV;
+    using Word = typename CodeWord<K>::T;
+
+    extern __shared__ __align__(128) uint8_t tma_smem[];
+    TmaBarriers *bar = reinterpret_cast<TmaBarriers *>(tma_smem + kTmaStages * kStageBytes);
+    __shared__ float lut[16];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid < 16) lut[tid] = (K >= 2) ? __fdiv_rn((float)(tid - L), (float)L) : 0.0f;
+    if (tid == 0) {
+        for (int s = 0; s < kTmaStages; ++s) {
+            mbar_init(&bar->full[s], 1);
+            mbar_init(&bar->empty[s], kTmaConsumers / 32);
+        }
+        bar->abort_flag = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+    volatile int *abort_flag = &bar->abort_flag;
+
+    if (warp == kTmaConsumers / 32) {
+        // ---------------------------------------------------- producer --
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            uint32_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
+                const int s = it % kTmaStages;
+                const uint32_t ph = (it / kTmaStages) & 1u;
+                if (!wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, p.status, kQuantWaitNs)) break;
+                const QuantSlotDesc &S = p.slot[find_slot(p, tile)];
+                const int64_t v0 = (tile - S.tile0) * kTmaVec;
+                const int64_t left = S.nvec - v0;
+                const uint32_t nv = (uint32_t)(left < kTmaVec ? left : kTmaVec);
+                uint8_t *st = tma_smem + s * kStageBytes;
+                mbar_expect_tx(&bar->full[s], nv * BPV);
+                if constexpr (OP == QuantOp::Compress) {
+                    bulk_g2s(st, static_cast<const uint4 *>(S.x) + v0, nv * 16, &bar->full[s], pol);
+                    bulk_g2s(st + kTmaVec * 16, static_cast<const uint4 *>(S.base) + v0, nv * 16, &bar->full[s], pol);
+                    bulk_g2s(st + kTmaVec * 32, S.err + v0 * 8, nv * 32, &bar->full[s], pol);
+                } else {
+                    bulk_g2s(st, S.cache + v0 * 8, nv * 32, &bar->full[s], pol);
+                }
+            }
+            // every copy this thread issued has landed before the CTA exits
+            const uint32_t out = it < (uint32_t)kTmaStages ? it : (uint32_t)kTmaStages;
+            for (uint32_t j = it - out; j < it; ++j) {
+                volatile int no_abort = 0;
+                wait_bounded(&bar->full[j % kTmaStages], (j / kTmaStages) & 1u, &no_abort, p.status, kQuantWaitNs);
+            }
+        }
+        return;
+    }
+
+    // ------------------------------------------------------- consumers --
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
+        const int s = it % kTmaStages;
+        const uint32_t ph = (it / kTmaStages) & 1u;
+        const QuantSlotDesc &S = p.slot[find_slot(p, tile)];
+        const int64_t v0 = (tile - S.tile0) * kTmaVec;
+        const int64_t left = S.nvec - v0;
+        const int nv = (int)(left < kTmaVec ? left : kTmaVec);
+        const uint8_t *st = tma_smem + s * kStageBytes;
+
+        if constexpr (OP == QuantOp::Compress) {
+            bool ok = wait_bounded(&bar->full[s], ph, abort_flag, p.status, kQuantWaitNs);
+            if (!__all_sync(kFull, ok)) break;
+            uint4 xv[2], bv[2];
+            float4 ea[2], eb[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int vl = tid + u * kTmaConsumers;
+                if (vl < nv) {
+                    xv[u] = reinterpret_cast<const uint4 *>(st)[vl];
+                    bv[u] = reinterpret_cast<const uint4 *>(st + kTmaVec * 16)[vl];
+                    const float4 *e = reinterpret_cast<const float4 *>(st + kTmaVec * 32);
+                    ea[u] = e[2 * vl];
+                    eb[u] = e[2 * vl + 1];
+                } else {
+                    xv[u] = bv[u] = make_uint4(0, 0, 0, 0);
+                    ea[u] = eb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->empty[s]);
+
+            uint4 *B = static_cast<uint4 *>(S.base);
+            float4 *E = reinterpret_cast<float4 *>(S.err);
+            Word *codes = reinterpret_cast<Word *>(S.codes);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int vl = tid + u * kTmaConsumers;
+                const bool valid = vl < nv;
+                const int64_t v = v0 + vl;
+                float xf[8], bf[8], a[8];
+                unpack8(xv[u], xf);
+                unpack8(bv[u], bf);
+                const float e[8] = {ea[u].x, ea[u].y, ea[u].z, ea[u].w, eb[u].x, eb[u].y, eb[u].z, eb[u].w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(__fsub_rn(xf[j], bf[j]), e[j]);
+                bool nonfinite;
+                float sc = group_scale<K, G, SS>(a, nonfinite);
+                const bool zero = nonfinite || !(sc >= kScaleMin);
+                if (zero) sc = 0.0f;
+                if (nonfinite && valid) atomicOr(p.status, kStatusNonfinite);
+                uint32_t word = 0;
+                if constexpr (K >= 2) {
+                    const float inv = __fdiv_rn((float)L, zero ? 1.0f : sc);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        int q = __float2int_rn(__fmul_rn(a[j], inv));
+                        q = min(max(q, -L), L);
+                        const int c = zero ? L : q + L;
+                        word |= (uint32_t)c << (K * j);
+                        a[j] = __fsub_rn(a[j], __fmul_rn(lut[c], sc));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const bool pos = zero || (a[j] >= 0.0f);
+                        word |= (uint32_t)pos << j;
+                        a[j] = __fsub_rn(a[j], pos ? sc : -sc);
+                    }
+                }
+                if (valid) {
+                    __stcs(B + v, xv[u]);
+                    __stcs(E + 2 * v, make_float4(a[0], a[1], a[2], a[3]));
+                    __stcs(E + 2 * v + 1, make_float4(a[4], a[5], a[6], a[7]));
+                    codes[v] = (Word)word;
+                    if ((lane & (LPG - 1)) == 0) S.scales[v / LPG] = sc;
+                }
+            }
+        } else {
+            // codes and scales do not go through the stage: load them first
+            const Word *codes = reinterpret_cast<const Word *>(S.codes);
+            Word cw[2];
+            float sv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int vl = tid + u * kTmaConsumers;
+                if (vl < nv) {
+                    cw[u] = __ldcs(codes + v0 + vl);
+                    sv[u] = __ldcs(S.scales + (v0 + vl) / LPG);
+                } else {
+                    cw[u] = 0;
+                    sv[u] = 0.0f;
+                }
+            }
+            bool ok = wait_bounded(&bar->full[s], ph, abort_flag, p.status, kQuantWaitNs);
+            if (!__all_sync(kFull, ok)) break;
+            float4 ca[2], cb[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int vl = tid + u * kTmaConsumers;
+                if (vl < nv) {
+                    const float4 *c = reinterpret_cast<const float4 *>(st);
+                    ca[u] = c[2 * vl];
+                    cb[u] = c[2 * vl + 1];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->empty[s]);
+            float4 *C = reinterpret_cast<float4 *>(S.cache);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int vl = tid + u * kTmaConsumers;
+                if (vl < nv) {
+                    const int64_t v = v0 + vl;
+                    const uint32_t w = cw[u];
+                    const float sc = sv[u];
+                    float d[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t c = (w >> (K * j)) & ((1u << K) - 1u);
+                        if constexpr (K >= 2)
+                            d[j] = __fmul_rn(lut[c], sc);
+                        else
+                            d[j] = c ? sc : -sc;
+                    }
+                    const float4 a = ca[u], b = cb[u];
+                    __stcs(C + 2 * v, make_float4(__fadd_rn(a.x, d[0]), __fadd_rn(a.y, d[1]), __fadd_rn(a.z, d[2]),
+                                                  __fadd_rn(a.w, d[3])));
+                    __stcs(C + 2 * v + 1, make_float4(__fadd_rn(b.x, d[4]), __fadd_rn(b.y, d[5]),
+                                                      __fadd_rn(b.z, d[6]), __fadd_rn(b.w, d[7])));
+                }
+            }
+        }
+    }
+}
+
 using KernelFn = void (*)(QuantLaunch);
 
-template <QuantOp OP, int K, int SS>
+template <QuantOp OP, int K, int SS, bool TMA>
 KernelFn pick_group(int group)
 {
     switch (group) {
-    case 8: return k_quant<OP, K, 8, SS>;
-    case 16: return k_quant<OP, K, 16, SS>;
-    case 32: return k_quant<OP, K, 32, SS>;
-    case 64: return k_quant<OP, K, 64, SS>;
-    case 128: return k_quant<OP, K, 128, SS>;
-    case 256: return k_quant<OP, K, 256, SS>;
+    case 8: return TMA ? k_quant_tma<OP, K, 8, SS> : k_quant<OP, K, 8, SS>;
+    case 16: return TMA ? k_quant_tma<OP, K, 16, SS> : k_quant<OP, K, 16, SS>;
+    case 32: return TMA ? k_quant_tma<OP, K, 32, SS> : k_quant<OP, K, 32, SS>;
+    case 64: return TMA ? k_quant_tma<OP, K, 64, SS> : k_quant<OP, K, 64, SS>;
+    case 128: return TMA ? k_quant_tma<OP, K, 128, SS> : k_quant<OP, K, 128, SS>;
+    case 256: return TMA ? k_quant_tma<OP, K, 256, SS> : k_quant<OP, K, 256, SS>;
     default: return nullptr;
     }
 }
 
+template <bool TMA>
 KernelFn pick(QuantOp op, int bits, int group, int ss)
 {
     switch (op) {
     case QuantOp::WarmupSender: return k_quant<QuantOp::WarmupSender, 2, 8, 0>;
     case QuantOp::WarmupReceiver: return k_quant<QuantOp::WarmupReceiver, 2, 8, 0>;
     case QuantOp::Compress:
-        if (bits == 1) return ss ? pick_group<QuantOp::Compress, 1, 1>(group) : pick_group<QuantOp::Compress, 1, 0>(group);
-        if (bits == 2) return pick_group<QuantOp::Compress, 2, 0>(group);
-        if (bits == 4) return pick_group<QuantOp::Compress, 4, 0>(group);
+        if (bits == 1)
+            return ss ? pick_group<QuantOp::Compress, 1, 1, TMA>(group) : pick_group<QuantOp::Compress, 1, 0, TMA>(group);
+        if (bits == 2) return pick_group<QuantOp::Compress, 2, 0, TMA>(group);
+        if (bits == 4) return pick_group<QuantOp::Compress, 4, 0, TMA>(group);
         return nullptr;
     case QuantOp::Decompress:
-        if (bits == 1) return pick_group<QuantOp::Decompress, 1, 0>(group);
-        if (bits == 2) return pick_group<QuantOp::Decompress, 2, 0>(group);
-        if (bits == 4) return pick_group<QuantOp::Decompress, 4, 0>(group);
+        if (bits == 1) return pick_group<QuantOp::Decompress, 1, 0, TMA>(group);
+        if (bits == 2) return pick_group<QuantOp::Decompress, 2, 0, TMA>(group);
+        if (bits == 4) return pick_group<QuantOp::Decompress, 4, 0, TMA>(group);
         return nullptr;
     }
     return nullptr;
 }
 
-int blocks_per_sm(KernelFn fn)
+// Launch shape of one kernel instance: threads, dynamic shared memory and
+// resident CTAs per SM (cached; the attribute call raises the dynamic shared
+// memory limit of the TMA-staged instances once).
+struct Shape {
+    int threads;
+    size_t smem;
+    int per_sm;
+};
+
+Shape launch_shape(KernelFn fn, bool tma, QuantOp op)
 {
     static std::mutex mu;
-    static std::unordered_map<const void *, int> cache;
+    static std::unordered_map<const void *, Shape> cache;
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find((const void *)fn);
     if (it != cache.end()) return it->second;
+    Shape sh{kThreads, 0, 1};
+    if (tma) {
+        sh.threads = kTmaThreads;
+        sh.smem = op == QuantOp::Compress ? tma_smem_bytes<QuantOp::Compress>() : tma_smem_bytes<QuantOp::Decompress>();
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh.smem);
+    }
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kThreads, 0) != cudaSuccess || nb < 1) nb = 1;
-    cache[(const void *)fn] = nb;
-    return nb;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, sh.threads, sh.smem) != cudaSuccess || nb < 1) nb = 1;
+    sh.per_sm = nb;
+    cache[(const void *)fn] = sh;
+    return sh;
+}
+
+// Staging of the compress / decompress streams: "tma" (bulk-async copies
+// through shared memory) or "reg" (vector loads straight into registers).
+bool use_tma_staging()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char *e = getenv("CF_QUANT_STAGING");
+        v = (e && strcmp(e, "tma") == 0) ? 1 : 0;
+    }
+    return v == 1;
 }
 
 }  // namespace
@@ -332,17 +594,24 @@ int num_sms()
     return sms;
 }
 
-int64_t quant_tile_elems() { return (int64_t)kTileVec * 8; }
-
-cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, const QuantLaunch &lp,
-                         cudaStream_t stream)
+cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, QuantLaunch &lp, cudaStream_t stream)
 {
-    if (lp.ntiles <= 0) return cudaSuccess;
-    KernelFn fn = pick(op, bits, group, sign_scale);
+    const bool tma = use_tma_staging() && (op == QuantOp::Compress || op == QuantOp::Decompress);
+    KernelFn fn = tma ? pick<true>(op, bits, group, sign_scale) : pick<false>(op, bits, group, sign_scale);
     if (!fn) return cudaErrorInvalidValue;
-    const int64_t cap = (int64_t)num_sms() * blocks_per_sm(fn);
-    const int grid = (int)(lp.ntiles < cap ? lp.ntiles : cap);
-    fn<<<grid, kThreads, 0, stream>>>(lp);
+    // tile prefix of every slot, in this kernel's tile size
+    const int64_t tile_vec = tma ? kTmaVec : kTileVec;
+    int64_t tiles = 0;
+    for (int k = 0; k < lp.nslots; ++k) {
+        lp.slot[k].tile0 = tiles;
+        tiles += (lp.slot[k].nvec + tile_vec - 1) / tile_vec;
+    }
+    lp.ntiles = tiles;
+    if (tiles <= 0) return cudaSuccess;
+    const Shape sh = launch_shape(fn, tma, op);
+    const int64_t cap = (int64_t)num_sms() * sh.per_sm;
+    const int grid = (int)(tiles < cap ? tiles : cap);
+    fn<<<grid, sh.threads, sh.smem, stream>>>(lp);
     return cudaGetLastError();
 }
 

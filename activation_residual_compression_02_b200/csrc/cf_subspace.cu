@@ -10,7 +10,8 @@
 // Kernels (one grouped launch each, over every matrix of the call):
 //  * k_gemm_tf32: the two products with A.  P = A Q (A K-major) and
 //    Z = A^T P (A read as an MN-major operand straight from its row-major
-//    storage).  A warp-specialised persistent tcgen05 kernel: one TMA warp
+//    storage, staged with the 128-byte/32-byte-atom swizzle that MN-major
+//    32-bit operands require).  A warp-specialised persistent tcgen05 kernel: one TMA warp
 //    streams 128x32 fp32 tiles of A (128-byte swizzle) plus the matching
 //    r-column slice of Q^T / P^T; four warps round each A tile to TF32 in
 //    shared memory (round to nearest: the tensor core would otherwise drop the
@@ -33,6 +34,7 @@
 #include <mutex>
 
 #include "cf_internal.h"
+#include "cf_ptx.cuh"
 
 namespace cf {
 namespace {
@@ -70,63 +72,7 @@ struct GemmParams {
 };
 
 // ------------------------------------------------------- PTX wrappers ----
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t globaltimer()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *b)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait: true when the phase of `parity` completed; false on abort or
-// timeout (the first thread to time out raises the abort flag and the status).
-__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *status,
-                                          unsigned long long limit_ns)
-{
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
-        if ((i & 31) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > limit_ns) {
-                *abort_flag = 1;
-                atomicOr(status, kStatusTimeout);
-                return false;
-            }
-        }
-    }
-}
+using namespace ptx;
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
 {
@@ -137,7 +83,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -175,16 +120,25 @@ __device__ __forceinline__ float round_tf32(float x)
     return __uint_as_float(r);
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version
-// 1 in bits 46-47, layout type 2 in bits 61-63).  Offsets are in bytes.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+// Shared-memory matrix descriptor (sm_100 format: version 1 in bits 46-47,
+// layout type in bits 61-63).  Offsets are in bytes.
+//   K-major operands : 128-byte swizzle (type 2), 8-row groups at SBO = 1024.
+//   MN-major TF32 A  : the only MN-major layout the tensor core takes for
+//                      32-bit elements is the 128-byte swizzle with 32-byte
+//                      atoms (type 1): 128-byte rows of 32 MN-consecutive
+//                      elements, 4-row K groups at SBO, 32-element MN blocks
+//                      at LBO.
+constexpr uint32_t kLayoutSw128 = 2;
+constexpr uint32_t kLayoutSw128Atom32 = 1;
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
 {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;
-    d |= (uint64_t)2 << 61;
+    d |= (uint64_t)layout << 61;
     return d;
 }
 
@@ -231,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
         }
         mbar_init(&S->drain, 1);
         S->abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S->tmem_base)),
@@ -307,9 +261,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
                     const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
 #pragma unroll
                     for (int k = 0; k < kBK / 8; ++k) {
-                        const uint64_t ad = p.mn_major ? smem_desc(a0 + k * 1024, 4096, 1024)
-                                                       : smem_desc(a0 + k * 32, 16, 1024);
-                        const uint64_t bd = smem_desc(b0 + k * 32, 16, 1024);
+                        const uint64_t ad = p.mn_major ? smem_desc(a0 + k * 1024, 4096, 512, kLayoutSw128Atom32)
+                                                       : smem_desc(a0 + k * 32, 16, 1024, kLayoutSw128);
+                        const uint64_t bd = smem_desc(b0 + k * 32, 16, 1024, kLayoutSw128);
                         tc_mma_tf32(dtm, ad, bd, idesc, (kt > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(&S->empty[s]);
@@ -627,7 +581,7 @@ EncodeFn encode_fn()
 
 // 2-D fp32 tensor map: dims {inner, outer}, row pitch in elements, box {bx, by}.
 bool make_map(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t pitch_elems, uint32_t bx,
-              uint32_t by)
+              uint32_t by, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     EncodeFn fn = encode_fn();
     if (!fn) return false;
@@ -636,7 +590,7 @@ bool make_map(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer,
     cuuint32_t box[2] = {bx, by};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -721,7 +675,7 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
                 g.out = out_mode == 0 ? (float *)(ws + L.pt + (size_t)i * L.rp * L.mp * 4)
                                       : (float *)(ws + L.pe + (size_t)i * m * L.rp * 4);
             } else {
-                ok = make_map(&g.ta, mats[i].A, n, m, n, 32, kBK) &&
+                ok = make_map(&g.ta, mats[i].A, n, m, n, 32, kBK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
                      make_map(&g.tb, ws + L.pt + (size_t)i * L.rp * L.mp * 4, m, L.rp, L.mp, kBK, L.rp);
                 g.out = (float *)(ws + L.z + (size_t)i * n * L.rp * 4);
             }
