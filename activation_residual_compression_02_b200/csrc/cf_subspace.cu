@@ -46,19 +46,19 @@ constexpr int kStages = 8;
 constexpr int kGemmThreads = 320;   // 10 warps: TMA, MMA, 4 convert, 4 epilogue
 constexpr int kATileBytes = kBM * kBK * 4;   // 16 KB
 constexpr int kBTileBytes = 32 * kBK * 4;    // room for N = 32
-constexpr int kMaxGemmMats = 40;
+constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parameters
 constexpr int kTmemCols = 64;       // two accumulators of up to 32 columns
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 struct __align__(64) GemmMat {
-    CUtensorMap ta;    // A (fp32, row-major m x n)
-    CUtensorMap tb;    // B^T slice source: Q^T [RP x n] or P^T [RP x m] (K-major)
-    float *out;        // output
-    int64_t pad_[7];
+    CUtensorMap ta;    // A (fp32, row-major m x n) of this matrix
 };
 
 struct GemmParams {
     GemmMat mat[kMaxGemmMats];
+    CUtensorMap tb;    // B^T blocks of every matrix, 3-D {K, rp, matrix}: Q^T or P^T (K-major)
+    float *out;        // output of matrix 0; matrix i at out + i * out_stride
+    int64_t out_stride;
     int nmat;
     int tiles_per_mat;
     int ktiles;
@@ -80,6 +80,15 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
             "r"(smem_u32(dst)),
         "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(smem_u32(dst)),
+        "l"((uint64_t)map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
                         for (int j = 0; j < 4; ++j)
                             tma_load_2d(a + j * 4096, &M.ta, mt * kBM + 32 * j, kt * kBK, &S->full[s]);
                     }
-                    tma_load_2d(sB + s * kBTileBytes, &M.tb, kt * kBK, 0, &S->full[s]);
+                    tma_load_3d(sB + s * kBTileBytes, &p.tb, kt * kBK, 0, mi, &S->full[s]);
                 }
             }
             // Drain: every load this thread issued has landed before exit.
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
             const int mi = tile / p.tiles_per_mat;
             const int mt = tile - mi * p.tiles_per_mat;
             const int row = mt * kBM + 32 * q + lane;
-            float *out = p.mat[mi].out;
+            float *out = p.out + (int64_t)mi * p.out_stride;
             if (row < p.out_rows) {
                 if (p.out_mode == 0) {
                     for (int c = 0; c < rp; ++c)
@@ -368,14 +377,14 @@ constexpr int kGramRows = 256;   // rows per Gram CTA
 
 struct CholMat {
     const float *Y;     // input block [rows x ld]
-    double *G;          // Gram matrix [rp x rp] (fp64, zeroed before k_gram)
-    float *Qt;          // mode Q: rounded transposed output [rp x qt_ld] (rows >= r zero)
+    double *G;          // Gram matrix [32 x 32] (fp64, zeroed before k_gram)
+    float *Qt;          // mode Q: rounded transposed output [rp x qt_ld] (rows >= r stay zero)
     float *Qexact;      // mode Q: optional exact output [rows x r] (V)
     float *U;           // mode U: [rows x r]
     float *R;           // mode U: [r x r]
 };
 
-constexpr int kMaxCholMats = 64;
+constexpr int kMaxCholMats = 192;
 
 struct CholParams {
     CholMat mat[kMaxCholMats];
@@ -416,24 +425,35 @@ __global__ void __launch_bounds__(kGramThreads) k_gram(const __grid_constant__ C
     }
 }
 
-// Cholesky of G (upper R, G = R^T R) by one thread into shared memory.
-__device__ void cholesky_upper(const double *G, double *R, int r, uint32_t *status, bool report)
+// Upper Cholesky factor of G (G = R^T R) by one warp: lane j owns column j.
+// Step p: lane p forms the diagonal, then every lane q > p forms R[p][q].
+// A pivot that is not positive (G not positive definite) is reported and
+// replaced by 1 so that the solve stays finite.
+__device__ void cholesky_upper_warp(const double *G, double *R, double *inv_diag, int r, uint32_t *status,
+                                    bool report)
 {
-    for (int i = 0; i < r * 32; ++i) R[i] = 0.0;
+    const int lane = threadIdx.x & 31;
+    for (int i = lane; i < 32 * 32; i += 32) R[i] = 0.0;
+    __syncwarp();
     for (int pp = 0; pp < r; ++pp) {
-        double diag = G[pp * 32 + pp];
-        for (int k = 0; k < pp; ++k) diag -= R[k * 32 + pp] * R[k * 32 + pp];
-        if (!(diag > 0.0) || !isfinite(diag)) {
-            if (report) atomicOr(status, kStatusNotSpd);
-            diag = 1.0;  // keeps the solve finite; the status reports the failure
+        if (lane == pp) {
+            double diag = G[pp * 32 + pp];
+            for (int k = 0; k < pp; ++k) diag -= R[k * 32 + pp] * R[k * 32 + pp];
+            if (!(diag > 0.0) || !isfinite(diag)) {
+                if (report) atomicOr(status, kStatusNotSpd);
+                diag = 1.0;
+            }
+            const double d = sqrt(diag);
+            R[pp * 32 + pp] = d;
+            inv_diag[pp] = 1.0 / d;
         }
-        const double d = sqrt(diag);
-        R[pp * 32 + pp] = d;
-        for (int qq = pp + 1; qq < r; ++qq) {
-            double v = G[pp * 32 + qq];
-            for (int k = 0; k < pp; ++k) v -= R[k * 32 + pp] * R[k * 32 + qq];
-            R[pp * 32 + qq] = v / d;
+        __syncwarp();
+        if (lane > pp && lane < r) {
+            double v = G[pp * 32 + lane];
+            for (int k = 0; k < pp; ++k) v -= R[k * 32 + pp] * R[k * 32 + lane];
+            R[pp * 32 + lane] = v * inv_diag[pp];
         }
+        __syncwarp();
     }
 }
 
@@ -448,9 +468,10 @@ __global__ void __launch_bounds__(kSolveThreads) k_chol_solve(const __grid_const
     const int r = p.r;
     __shared__ double Gs[32 * 32];
     __shared__ double Rs[32 * 32];
+    __shared__ double inv_diag[32];
     for (int i = threadIdx.x; i < 32 * 32; i += kSolveThreads) Gs[i] = M.G[i];
     __syncthreads();
-    if (threadIdx.x == 0) cholesky_upper(Gs, Rs, r, p.status, blockIdx.x == 0);
+    if (threadIdx.x < 32) cholesky_upper_warp(Gs, Rs, inv_diag, r, p.status, blockIdx.x == 0);
     __syncthreads();
     if (MODE == 1 && blockIdx.x == 0) {
         for (int i = threadIdx.x; i < r * r; i += kSolveThreads) {
@@ -458,28 +479,44 @@ __global__ void __launch_bounds__(kSolveThreads) k_chol_solve(const __grid_const
             M.R[i] = (float)Rs[a * 32 + b];
         }
     }
-    for (int row = blockIdx.x * kSolveThreads + threadIdx.x; row < p.rows; row += gridDim.x * kSolveThreads) {
-        double q[32];
-        const float *y = M.Y + (int64_t)row * p.ld;
-        for (int c = 0; c < r; ++c) {
+    const int row = blockIdx.x * kSolveThreads + threadIdx.x;
+    if (row >= p.rows) return;
+    double q[32];
+    const float *y = M.Y + (int64_t)row * p.ld;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        if (c < r) {
             double v = (double)y[c];
+#pragma unroll
             for (int k = 0; k < c; ++k) v -= q[k] * Rs[k * 32 + c];
-            q[c] = v / Rs[c * 32 + c];
+            q[c] = v * inv_diag[c];
         }
-        if (MODE == 0) {
-            for (int c = 0; c < r; ++c) M.Qt[(int64_t)c * p.qt_ld + row] = round_tf32((float)q[c]);
-            if (M.Qexact)
-                for (int c = 0; c < r; ++c) M.Qexact[(int64_t)row * r + c] = (float)q[c];
-        } else {
-            for (int c = 0; c < r; ++c) M.U[(int64_t)row * r + c] = (float)q[c];
+    }
+    if (MODE == 0) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+            if (c < r) M.Qt[(int64_t)c * p.qt_ld + row] = round_tf32((float)q[c]);
+        if (M.Qexact) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+                if (c < r) M.Qexact[(int64_t)row * r + c] = (float)q[c];
         }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+            if (c < r) M.U[(int64_t)row * r + c] = (float)q[c];
     }
 }
 
 // -------------------------------------------------------------- apply ----
+// D = U (R V^T) with E = A - D and/or C += D.  W = R V^T is held in
+// registers: a thread owns CPT adjacent columns (4 for r <= 16, 2 for
+// r <= 32) for all RMAX rows of W, and walks a long strip of rows; the U
+// rows of the CTA's strip are staged in shared memory (zero-padded to
+// RMAX) and read as broadcasts.  A and C are streamed with 4 rows in flight
+// per thread.
 constexpr int kApplyThreads = 256;
-constexpr int kApplyRows = 64;     // rows per CTA tile
-constexpr int kApplyCols = 128;    // columns per CTA tile (32 threads x float4)
+constexpr int kApplyRows = 256;     // rows per CTA strip (8 warps x 32 rows)
 
 struct ApplyMat {
     const float *A;   // [m x n] or null
@@ -490,7 +527,7 @@ struct ApplyMat {
     float *C;         // [m x n] or null: C += D
 };
 
-constexpr int kMaxApplyMats = 128;
+constexpr int kMaxApplyMats = 192;
 
 struct ApplyParams {
     ApplyMat mat[kMaxApplyMats];
@@ -499,63 +536,115 @@ struct ApplyParams {
     int row_tiles, col_tiles;
 };
 
-// D = U (R V^T) for a 64 x 128 tile: W = R V^T (r x 128) and the U rows are
-// staged in shared memory; each thread owns a float4 column strip of 8 rows.
-__global__ void __launch_bounds__(kApplyThreads) k_apply(const __grid_constant__ ApplyParams p)
+template <int RMAX, bool HAS_E, bool HAS_C>
+__global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constant__ ApplyParams p)
 {
+    constexpr int CPT = 64 / RMAX;           // columns per thread
+    constexpr int COLS = 32 * CPT;           // columns per CTA
+    constexpr int RPW = kApplyRows / 8;      // rows per warp
     const int per_mat = p.row_tiles * p.col_tiles;
     const int mi = blockIdx.x / per_mat;
     const int t = blockIdx.x - mi * per_mat;
-    const int rt = t / p.col_tiles, ctile = t - rt * p.col_tiles;
+    const int ct = t % p.col_tiles, rt = t / p.col_tiles;
     const ApplyMat &M = p.mat[mi];
-    const int r = p.r, n = p.n;
-    const int row0 = rt * kApplyRows, col0 = ctile * kApplyCols;
-    __shared__ float Rs[32 * 32];
-    __shared__ float Vs[kApplyCols * 33];
-    __shared__ float Ws[32 * kApplyCols];
-    __shared__ float Us[kApplyRows * 33];
-    for (int i = threadIdx.x; i < r * r; i += kApplyThreads) Rs[(i / r) * 32 + (i % r)] = M.R[i];
-    for (int i = threadIdx.x; i < kApplyCols * r; i += kApplyThreads) {
-        const int j = i / r, c = i - j * r;
-        Vs[j * 33 + c] = (col0 + j < n) ? M.V[(int64_t)(col0 + j) * r + c] : 0.0f;
+    const int r = p.r, n = p.n, m = p.m;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int row0 = rt * kApplyRows;
+    const int col = ct * COLS + lane * CPT;
+
+    __shared__ float Rs[32 * 33];
+    __shared__ float Vs[COLS * (RMAX + 1)];
+    __shared__ __align__(16) float Us[kApplyRows * RMAX];
+    for (int i = threadIdx.x; i < 32 * 33; i += kApplyThreads) {
+        const int a = i / 33, b = i - a * 33;
+        Rs[i] = (a < r && b < r) ? M.R[a * r + b] : 0.0f;
     }
-    for (int i = threadIdx.x; i < kApplyRows * r; i += kApplyThreads) {
-        const int a = i / r, c = i - a * r;
-        Us[a * 33 + c] = (row0 + a < p.m) ? M.U[(int64_t)(row0 + a) * r + c] : 0.0f;
+    for (int i = threadIdx.x; i < COLS * RMAX; i += kApplyThreads) {
+        const int j = i / RMAX, c = i - j * RMAX;
+        const int gc = ct * COLS + j;
+        Vs[j * (RMAX + 1) + c] = (gc < n && c < r) ? M.V[(int64_t)gc * r + c] : 0.0f;
+    }
+    for (int i = threadIdx.x; i < kApplyRows * RMAX; i += kApplyThreads) {
+        const int a = i / RMAX, c = i - a * RMAX;
+        Us[i] = (row0 + a < m && c < r) ? M.U[(int64_t)(row0 + a) * r + c] : 0.0f;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < r * kApplyCols; i += kApplyThreads) {
-        const int k = i / kApplyCols, j = i - k * kApplyCols;
-        float w = 0.0f;
-        for (int q = k; q < r; ++q) w = fmaf(Rs[k * 32 + q], Vs[j * 33 + q], w);  // R is upper triangular
-        Ws[k * kApplyCols + j] = w;
-    }
-    __syncthreads();
-    const int cx = (threadIdx.x & 31) * 4;        // column offset in the tile
-    const int ry = threadIdx.x >> 5;              // 8 row groups of 4 rows
-    const int col = col0 + cx;
-    if (col >= n) return;                          // n % 8 == 0: a float4 is all in or all out
-    for (int rr = 0; rr < kApplyRows / 8; ++rr) {
-        const int a = ry + 8 * rr;
-        const int row = row0 + a;
-        if (row >= p.m) break;
-        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-        for (int k = 0; k < r; ++k) {
-            const float u = Us[a * 33 + k];
-            const float4 w = *(const float4 *)&Ws[k * kApplyCols + cx];
-            d0 = fmaf(u, w.x, d0);
-            d1 = fmaf(u, w.y, d1);
-            d2 = fmaf(u, w.z, d2);
-            d3 = fmaf(u, w.w, d3);
+    // W[k][col + c] = sum_{q >= k} R[k][q] V[col + c][q], in registers
+    float w[RMAX][CPT];
+#pragma unroll
+    for (int k = 0; k < RMAX; ++k)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            float acc = 0.0f;
+            const int j = lane * CPT + c;
+#pragma unroll
+            for (int q = 0; q < RMAX; ++q) acc = fmaf(Rs[k * 33 + q], Vs[j * (RMAX + 1) + q], acc);
+            w[k][c] = acc;
         }
-        const int64_t off = (int64_t)row * n + col;
-        if (M.E) {
-            const float4 av = __ldcs((const float4 *)(M.A + off));
-            __stcs((float4 *)(M.E + off), make_float4(av.x - d0, av.y - d1, av.z - d2, av.w - d3));
+    if (col >= n) return;   // n % 4 == 0 and CPT divides 4: a thread's columns are all in or all out
+
+    const int rbeg = warp * RPW;
+    for (int a0 = rbeg; a0 < rbeg + RPW; a0 += 4) {
+        float av[4][CPT], cv[4][CPT];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int row = row0 + a0 + u;
+            const int64_t off = (int64_t)row * n + col;
+            if (row < m) {
+                if (HAS_E && M.E) {
+                    if constexpr (CPT == 4) {
+                        const float4 v = __ldcs((const float4 *)(M.A + off));
+                        av[u][0] = v.x; av[u][1] = v.y; av[u][2] = v.z; av[u][3] = v.w;
+                    } else {
+                        const float2 v = __ldcs((const float2 *)(M.A + off));
+                        av[u][0] = v.x; av[u][1] = v.y;
+                    }
+                }
+                if (HAS_C && M.C) {
+                    if constexpr (CPT == 4) {
+                        const float4 v = __ldcs((const float4 *)(M.C + off));
+                        cv[u][0] = v.x; cv[u][1] = v.y; cv[u][2] = v.z; cv[u][3] = v.w;
+                    } else {
+                        const float2 v = __ldcs((const float2 *)(M.C + off));
+                        cv[u][0] = v.x; cv[u][1] = v.y;
+                    }
+                }
+            }
         }
-        if (M.C) {
-            const float4 cv = __ldcs((const float4 *)(M.C + off));
-            __stcs((float4 *)(M.C + off), make_float4(cv.x + d0, cv.y + d1, cv.z + d2, cv.w + d3));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int row = row0 + a0 + u;
+            if (row >= m) break;
+            float d[CPT];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) d[c] = 0.0f;
+            const float *urow = Us + (a0 + u) * RMAX;
+#pragma unroll
+            for (int k = 0; k < RMAX; k += 4) {
+                const float4 uk = *(const float4 *)(urow + k);
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    d[c] = fmaf(uk.x, w[k][c], d[c]);
+                    d[c] = fmaf(uk.y, w[k + 1][c], d[c]);
+                    d[c] = fmaf(uk.z, w[k + 2][c], d[c]);
+                    d[c] = fmaf(uk.w, w[k + 3][c], d[c]);
+                }
+            }
+            const int64_t off = (int64_t)row * n + col;
+            if (HAS_E && M.E) {
+                if constexpr (CPT == 4)
+                    __stcs((float4 *)(M.E + off), make_float4(av[u][0] - d[0], av[u][1] - d[1], av[u][2] - d[2],
+                                                              av[u][3] - d[3]));
+                else
+                    __stcs((float2 *)(M.E + off), make_float2(av[u][0] - d[0], av[u][1] - d[1]));
+            }
+            if (HAS_C && M.C) {
+                if constexpr (CPT == 4)
+                    __stcs((float4 *)(M.C + off), make_float4(cv[u][0] + d[0], cv[u][1] + d[1], cv[u][2] + d[2],
+                                                              cv[u][3] + d[3]));
+                else
+                    __stcs((float2 *)(M.C + off), make_float2(cv[u][0] + d[0], cv[u][1] + d[1]));
+            }
         }
     }
 }
@@ -594,12 +683,28 @@ bool make_map(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 tensor map over `count` equally spaced [outer x inner] blocks
+// (pitch in elements, block stride in elements), box {bx, by, 1}.
+bool make_map3(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t count, uint64_t pitch_elems,
+               uint64_t block_elems, uint32_t bx, uint32_t by)
+{
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {inner, outer, count};
+    cuuint64_t strides[2] = {pitch_elems * 4, block_elems * 4};
+    cuuint32_t box[3] = {bx, by, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int64_t rup(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
     int rp;
     int64_t mp, np;                       // padded leading dims (multiples of 32)
-    size_t qt, pt, pe, z, g, total;       // per-matrix byte offsets inside the workspace
+    size_t qt, pt, pe, z, g, total;       // byte offsets inside the workspace
 };
 
 WsLayout layout(int nmat, int64_t m, int64_t n, int r)
@@ -637,7 +742,7 @@ cudaError_t gemm_launch(GemmParams &gp, int total_tiles, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-// out_i = A_i Q_i (mn_major = 0) or A_i^T P_i (mn_major = 1) for a chunk of matrices.
+// out_i = A_i Q_i (mn_major = 0) or A_i^T P_i (mn_major = 1) for every matrix.
 cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLayout &L, int mn_major, int out_mode,
                       cudaStream_t stream)
 {
@@ -654,37 +759,41 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
         gp->out_mode = out_mode;
         gp->status = pl.status;
         gp->wait_ns = kWaitNs;
+        bool ok;
         if (!mn_major) {
             gp->tiles_per_mat = (int)((m + kBM - 1) / kBM);
             gp->ktiles = (int)((n + kBK - 1) / kBK);
             gp->out_rows = (int)m;
             gp->out_ld = (int)L.mp;
+            ok = make_map3(&gp->tb, ws + L.qt + (size_t)first * L.rp * L.np * 4, n, L.rp, cnt, L.np, L.rp * L.np,
+                           kBK, L.rp);
+            if (out_mode == 0) {
+                gp->out = (float *)(ws + L.pt) + (size_t)first * L.rp * L.mp;
+                gp->out_stride = L.rp * L.mp;
+            } else {
+                gp->out = (float *)(ws + L.pe) + (size_t)first * m * L.rp;
+                gp->out_stride = m * L.rp;
+            }
         } else {
             gp->tiles_per_mat = (int)((n + kBM - 1) / kBM);
             gp->ktiles = (int)((m + kBK - 1) / kBK);
             gp->out_rows = (int)n;
             gp->out_ld = 0;
+            ok = make_map3(&gp->tb, ws + L.pt + (size_t)first * L.rp * L.mp * 4, m, L.rp, cnt, L.mp, L.rp * L.mp,
+                           kBK, L.rp);
+            gp->out = (float *)(ws + L.z) + (size_t)first * n * L.rp;
+            gp->out_stride = n * L.rp;
         }
-        for (int k = 0; k < cnt; ++k) {
-            const int i = first + k;
-            GemmMat &g = gp->mat[k];
-            bool ok;
-            if (!mn_major) {
-                ok = make_map(&g.ta, mats[i].A, n, m, n, kBK, kBM) &&
-                     make_map(&g.tb, ws + L.qt + (size_t)i * L.rp * L.np * 4, n, L.rp, L.np, kBK, L.rp);
-                g.out = out_mode == 0 ? (float *)(ws + L.pt + (size_t)i * L.rp * L.mp * 4)
-                                      : (float *)(ws + L.pe + (size_t)i * m * L.rp * 4);
-            } else {
-                ok = make_map(&g.ta, mats[i].A, n, m, n, 32, kBK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
-                     make_map(&g.tb, ws + L.pt + (size_t)i * L.rp * L.mp * 4, m, L.rp, L.mp, kBK, L.rp);
-                g.out = (float *)(ws + L.z + (size_t)i * n * L.rp * 4);
-            }
-            if (!ok) {
-                err = cudaErrorInvalidValue;
-                break;
-            }
+        for (int k = 0; k < cnt && ok; ++k) {
+            const LowrankMat &s = mats[first + k];
+            ok = !mn_major ? make_map(&gp->mat[k].ta, s.A, n, m, n, kBK, kBM)
+                           : make_map(&gp->mat[k].ta, s.A, n, m, n, 32, kBK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
         }
-        if (err == cudaSuccess) err = gemm_launch(*gp, cnt * gp->tiles_per_mat, stream);
+        if (!ok) {
+            err = cudaErrorInvalidValue;
+            break;
+        }
+        err = gemm_launch(*gp, cnt * gp->tiles_per_mat, stream);
     }
     delete gp;
     return err;
@@ -729,8 +838,7 @@ cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsL
         k_gram<<<ggrid, kGramThreads, 0, stream>>>(*cp);
         err = cudaGetLastError();
         if (err != cudaSuccess) break;
-        const int per = (int)((rows + kSolveThreads - 1) / kSolveThreads);
-        dim3 sgrid((unsigned)(per < 8 ? per : 8), (unsigned)cnt);
+        dim3 sgrid((unsigned)((rows + kSolveThreads - 1) / kSolveThreads), (unsigned)cnt);
         if (mode == 0)
             k_chol_solve<0><<<sgrid, kSolveThreads, 0, stream>>>(*cp);
         else
@@ -745,6 +853,8 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
 {
     ApplyParams *ap = new ApplyParams;
     cudaError_t err = cudaSuccess;
+    const int rmax = pl.r <= 16 ? 16 : 32;
+    const int cols = 32 * (64 / rmax);
     for (int first = 0; first < pl.nmat && err == cudaSuccess; first += kMaxApplyMats) {
         const int cnt = pl.nmat - first < kMaxApplyMats ? pl.nmat - first : kMaxApplyMats;
         memset(ap, 0, sizeof *ap);
@@ -753,8 +863,8 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
         ap->n = (int)pl.n;
         ap->r = pl.r;
         ap->row_tiles = (int)((pl.m + kApplyRows - 1) / kApplyRows);
-        ap->col_tiles = (int)((pl.n + kApplyCols - 1) / kApplyCols);
-        bool any = false;
+        ap->col_tiles = (int)((pl.n + cols - 1) / cols);
+        bool has_e = false, has_c = false;
         for (int k = 0; k < cnt; ++k) {
             const LowrankMat &s = mats[first + k];
             ApplyMat &a = ap->mat[k];
@@ -764,11 +874,18 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
             a.V = s.V;
             a.E = sender ? s.E : nullptr;
             a.C = s.C;
-            any = any || a.E || a.C;
+            has_e = has_e || a.E;
+            has_c = has_c || a.C;
         }
-        if (!any) continue;
-        const int64_t blocks = (int64_t)cnt * ap->row_tiles * ap->col_tiles;
-        k_apply<<<(unsigned)blocks, kApplyThreads, 0, stream>>>(*ap);
+        if (!has_e && !has_c) continue;
+        const unsigned blocks = (unsigned)((int64_t)cnt * ap->row_tiles * ap->col_tiles);
+        using Fn = void (*)(ApplyParams);
+        Fn fn;
+        if (rmax == 16)
+            fn = has_e ? (has_c ? k_apply<16, true, true> : k_apply<16, true, false>) : k_apply<16, false, true>;
+        else
+            fn = has_e ? (has_c ? k_apply<32, true, true> : k_apply<32, true, false>) : k_apply<32, false, true>;
+        fn<<<blocks, kApplyThreads, 0, stream>>>(*ap);
         err = cudaGetLastError();
     }
     delete ap;
