@@ -22,7 +22,8 @@ CF_MODE_QUANT, CF_MODE_LOWRANK = 0, 1
 
 EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
             "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
-            "cf_destroy"]
+            "cf_destroy", "cf_lowrank_noalloc"]
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class cf_config(ctypes.Structure):
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.cf_last_error.restype = ctypes.c_char_p
         L.cf_destroy.argtypes = [P]
         L.cf_destroy.restype = I
+        L.cf_lowrank_noalloc.argtypes = [ctypes.POINTER(cf_config), I, I64, I64, PP, PP, PP, PP, PP, PP, PP, P]
+        L.cf_lowrank_noalloc.restype = I
         _lib = L
     return _lib
 
@@ -215,6 +218,18 @@ def cf_decompress(ctx: Context, slots, step, stream=None):
 
 def cf_lowrank(ctx: Context, A, Q0, U, R, V, E=None, C=None, stream=None):
     ctx.lowrank(A, Q0, U, R, V, E, C, stream)
+
+
+def cf_lowrank_noalloc(A, Q0, U, R, V, E=None, C=None, rank: int = 16, iters: int = 2, stream=None) -> int:
+    """cf_lowrank without a context or workspace, for callers that cannot
+    allocate device memory: the scratch is a fixed 8 MiB device array inside
+    libcf.  Synchronous; returns the C status (CF_OK, CF_E_NOMEM when the call
+    does not fit the scratch, ...)."""
+    cfg = cf_config(CF_MODE_LOWRANK, 0, 0, 0, rank, iters)
+    nmat = len(A)
+    m, n = (A[0].shape[0], A[0].shape[1]) if nmat else (0, 0)
+    return int(lib().cf_lowrank_noalloc(ctypes.byref(cfg), nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R),
+                                        _parr(V), _parr(E), _parr(C), _stream_handle(stream)))
 
 
 def cf_check(ctx: Context, stream=None) -> int:

@@ -181,6 +181,45 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
                      const float *const *Q0, float *const *U, float *const *R, float *const *V,
                      float *const *E_opt, float *const *C_opt, void *cuda_stream);
 
+/* Bytes of device scratch that the library keeps on every GPU it is loaded
+ * on, for cf_lowrank_noalloc (status word plus the Algorithm 3 buffers). */
+#define CF_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* cf_lowrank for callers that cannot allocate device memory.  (The paper has
+ * no counterpart: this is an integration aid of this library.)
+ *
+ * Who needs it: code that must not call cudaMalloc or any allocating library
+ * routine at the point where it compresses -- work running inside a caller's
+ * pre-reserved memory pool, a plug-in that is handed only the tensors it may
+ * touch, or a step that must not change the device's allocation state while
+ * other work is in flight.  cf_lowrank needs a context (cf_create allocates
+ * its status word) and a caller-allocated workspace; this entry point needs
+ * neither.  Its scratch is a fixed CF_NOALLOC_SCRATCH_BYTES (8 MiB) device
+ * array inside the library, which every GPU that loads the library holds
+ * until the process exits.  It calls no device allocator.
+ *
+ * Arguments and results are those of cf_lowrank, with the rank r and the
+ * iteration count T taken from `config` (mode must be CF_MODE_LOWRANK);
+ * A, Q0, U, R, V, E_opt, C_opt are host arrays of nmat device pointers.
+ * Limits: the Algorithm 3 buffers of the call -- cf_lowrank_workspace_bytes
+ * for the same nmat, m, n and r, about 4*rp*(2m + 2n) + 8 KB per matrix with
+ * rp = 16 (r <= 16) or 32 -- must fit in CF_NOALLOC_SCRATCH_BYTES - 256
+ * bytes, and nmat <= 512; otherwise the call returns CF_E_NOMEM and launches
+ * nothing.  Eight 4608 x 3072 matrices at r = 16 fit in one call.
+ *
+ * The call is synchronous: it enqueues the work on `cuda_stream`, waits for
+ * it and returns the device status (CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or
+ * CF_E_CUDA).  The first call on a device looks up the scratch's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call shares the one scratch array,
+ * which keeps the previous call's contents (the call clears what must start
+ * at zero), so calls that overlap on the GPU -- on two streams or from two
+ * host threads -- race and must be serialised by the caller.  Errors before
+ * launch: CF_E_ARG, CF_E_SHAPE, CF_E_ALIGN, CF_E_NOMEM. */
+cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64_t m, int64_t n, const float *const *A,
+                             const float *const *Q0, float *const *U, float *const *R, float *const *V,
+                             float *const *E_opt, float *const *C_opt, void *cuda_stream);
+
 /* Synchronise `cuda_stream`, read and clear the device status word.
  * Returns CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or CF_E_CUDA (an asynchronous
  * CUDA error, e.g. from an earlier launch). */
