@@ -14,7 +14,7 @@
 // butterfly shuffles.  One launch covers every slot of a step: the slot table
 // is a __grid_constant__ parameter and persistent CTAs walk a flat tile
 // index.  The work is a pure stream (no reuse), so the design goal is bytes
-// in flight: each thread issues all loads of kUnroll vectors before it
+// in flight: each thread issues all loads of its kUnroll vectors before it
 // computes.
 //
 // Bit-exactness: every floating-point step is an explicit round-to-nearest
@@ -35,9 +35,37 @@
 namespace cf {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
-constexpr int kTileVec = kThreads * kUnroll;  // vectors of 8 elements per tile
+// Launch shape per operation: threads per CTA, vectors (of 8 elements) each
+// thread keeps in flight (a tile is threads * unroll vectors), and a cap on
+// resident CTAs per SM (0: as many as fit).  Chosen by sweeps on the B200
+// over 128..1024 threads, 1..8 vectors and 1..4 CTAs per SM on the 57-slot
+// FLUX-shaped step: compress wants many warps to hide its ~150 instructions
+// per vector (1024 x 1: 93.5% of the measured copy bandwidth, against 88% for
+// 256 x 4 at 2 CTAs/SM); decompress wants about 512 resident threads per SM
+// with 4 vectors each (94.5%, against 84% at 4 CTAs/SM).
+template <QuantOp OP>
+struct QShape {
+    static constexpr int kThreads = 256;
+    static constexpr int kUnroll = 4;
+    static constexpr int kMaxPerSm = 0;
+};
+template <>
+struct QShape<QuantOp::Compress> {
+    static constexpr int kThreads = 1024;
+    static constexpr int kUnroll = 1;
+    static constexpr int kMaxPerSm = 0;
+};
+template <>
+struct QShape<QuantOp::Decompress> {
+    static constexpr int kThreads = 512;
+    static constexpr int kUnroll = 4;
+    static constexpr int kMaxPerSm = 1;
+};
+template <QuantOp OP>
+constexpr int64_t qtile_vec()
+{
+    return (int64_t)QShape<OP>::kThreads * QShape<OP>::kUnroll;
+}
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kAbsMask = 0x7fffffffu;
 constexpr uint32_t kInfBits = 0x7f800000u;
@@ -106,8 +134,11 @@ __device__ __forceinline__ float group_scale(const float (&a)[8], bool &nonfinit
 }
 
 template <QuantOp OP, int K, int G, int SS>
-__global__ void __launch_bounds__(kThreads) k_quant(const __grid_constant__ QuantLaunch p)
+__global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
 {
+    constexpr int kThreads = QShape<OP>::kThreads;
+    constexpr int kUnroll = QShape<OP>::kUnroll;
+    constexpr int kTileVec = kThreads * kUnroll;
     constexpr int LPG = G / 8;
     constexpr int L = (K >= 2) ? (1 << (K - 1)) - 1 : 1;
     using Word = typename CodeWord<K>::T;
@@ -555,7 +586,26 @@ Shape launch_shape(KernelFn fn, bool tma, QuantOp op)
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find((const void *)fn);
     if (it != cache.end()) return it->second;
-    Shape sh{kThreads, 0, 1};
+    Shape sh{0, 0, 1};
+    int cap = 0;
+    switch (op) {
+    case QuantOp::WarmupSender:
+        sh.threads = QShape<QuantOp::WarmupSender>::kThreads;
+        cap = QShape<QuantOp::WarmupSender>::kMaxPerSm;
+        break;
+    case QuantOp::WarmupReceiver:
+        sh.threads = QShape<QuantOp::WarmupReceiver>::kThreads;
+        cap = QShape<QuantOp::WarmupReceiver>::kMaxPerSm;
+        break;
+    case QuantOp::Compress:
+        sh.threads = QShape<QuantOp::Compress>::kThreads;
+        cap = QShape<QuantOp::Compress>::kMaxPerSm;
+        break;
+    case QuantOp::Decompress:
+        sh.threads = QShape<QuantOp::Decompress>::kThreads;
+        cap = QShape<QuantOp::Decompress>::kMaxPerSm;
+        break;
+    }
     if (tma) {
         sh.threads = kTmaThreads;
         sh.smem = op == QuantOp::Compress ? tma_smem_bytes<QuantOp::Compress>() : tma_smem_bytes<QuantOp::Decompress>();
@@ -563,7 +613,7 @@ Shape launch_shape(KernelFn fn, bool tma, QuantOp op)
     }
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, sh.threads, sh.smem) != cudaSuccess || nb < 1) nb = 1;
-    sh.per_sm = nb;
+    sh.per_sm = (!tma && cap > 0 && nb > cap) ? cap : nb;
     cache[(const void *)fn] = sh;
     return sh;
 }
@@ -600,7 +650,15 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, QuantL
     KernelFn fn = tma ? pick<true>(op, bits, group, sign_scale) : pick<false>(op, bits, group, sign_scale);
     if (!fn) return cudaErrorInvalidValue;
     // tile prefix of every slot, in this kernel's tile size
-    const int64_t tile_vec = tma ? kTmaVec : kTileVec;
+    int64_t tile_vec = kTmaVec;
+    if (!tma) {
+        switch (op) {
+        case QuantOp::WarmupSender: tile_vec = qtile_vec<QuantOp::WarmupSender>(); break;
+        case QuantOp::WarmupReceiver: tile_vec = qtile_vec<QuantOp::WarmupReceiver>(); break;
+        case QuantOp::Compress: tile_vec = qtile_vec<QuantOp::Compress>(); break;
+        case QuantOp::Decompress: tile_vec = qtile_vec<QuantOp::Decompress>(); break;
+        }
+    }
     int64_t tiles = 0;
     for (int k = 0; k < lp.nslots; ++k) {
         lp.slot[k].tile0 = tiles;

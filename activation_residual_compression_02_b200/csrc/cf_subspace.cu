@@ -511,12 +511,12 @@ __global__ void __launch_bounds__(kSolveThreads) k_chol_solve(const __grid_const
 // -------------------------------------------------------------- apply ----
 // D = U (R V^T) with E = A - D and/or C += D.  W = R V^T is held in
 // registers: a thread owns CPT adjacent columns (4 for r <= 16, 2 for
-// r <= 32) for all RMAX rows of W, and walks a long strip of rows; the U
-// rows of the CTA's strip are staged in shared memory (zero-padded to
-// RMAX) and read as broadcasts.  A and C are streamed with 4 rows in flight
-// per thread.
+// r <= 32) for all RMAX rows of W and walks a long strip of rows; warp w
+// takes rows w, w + 8, ... of the strip, RF rows at a time, so that every
+// thread keeps RF rows of A (and C) in flight.  The U row of each step is
+// the same for all lanes of a warp (a broadcast load through L1).
 constexpr int kApplyThreads = 256;
-constexpr int kApplyRows = 256;     // rows per CTA strip (8 warps x 32 rows)
+constexpr int kApplyRows = 1024;    // rows per CTA strip
 
 struct ApplyMat {
     const float *A;   // [m x n] or null
@@ -536,12 +536,38 @@ struct ApplyParams {
     int row_tiles, col_tiles;
 };
 
+template <int CPT>
+struct Vec;
+template <> struct Vec<4> {
+    using T = float4;
+    static __device__ __forceinline__ void load(const float *p, float (&v)[4])
+    {
+        const float4 x = __ldcs((const float4 *)p);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[4])
+    {
+        __stcs((float4 *)p, make_float4(v[0], v[1], v[2], v[3]));
+    }
+};
+template <> struct Vec<2> {
+    static __device__ __forceinline__ void load(const float *p, float (&v)[2])
+    {
+        const float2 x = __ldcs((const float2 *)p);
+        v[0] = x.x; v[1] = x.y;
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[2])
+    {
+        __stcs((float2 *)p, make_float2(v[0], v[1]));
+    }
+};
+
 template <int RMAX, bool HAS_E, bool HAS_C>
 __global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constant__ ApplyParams p)
 {
-    constexpr int CPT = 64 / RMAX;           // columns per thread
-    constexpr int COLS = 32 * CPT;           // columns per CTA
-    constexpr int RPW = kApplyRows / 8;      // rows per warp
+    constexpr int CPT = 64 / RMAX;                     // columns per thread
+    constexpr int COLS = 32 * CPT;                     // columns per CTA
+    constexpr int RF = (HAS_E && HAS_C) ? 3 : 6;       // rows in flight per thread
     const int per_mat = p.row_tiles * p.col_tiles;
     const int mi = blockIdx.x / per_mat;
     const int t = blockIdx.x - mi * per_mat;
@@ -550,11 +576,11 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constan
     const int r = p.r, n = p.n, m = p.m;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int row0 = rt * kApplyRows;
+    const int row_end = min(m, row0 + kApplyRows);
     const int col = ct * COLS + lane * CPT;
 
     __shared__ float Rs[32 * 33];
     __shared__ float Vs[COLS * (RMAX + 1)];
-    __shared__ __align__(16) float Us[kApplyRows * RMAX];
     for (int i = threadIdx.x; i < 32 * 33; i += kApplyThreads) {
         const int a = i / 33, b = i - a * 33;
         Rs[i] = (a < r && b < r) ? M.R[a * r + b] : 0.0f;
@@ -564,12 +590,8 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constan
         const int gc = ct * COLS + j;
         Vs[j * (RMAX + 1) + c] = (gc < n && c < r) ? M.V[(int64_t)gc * r + c] : 0.0f;
     }
-    for (int i = threadIdx.x; i < kApplyRows * RMAX; i += kApplyThreads) {
-        const int a = i / RMAX, c = i - a * RMAX;
-        Us[i] = (row0 + a < m && c < r) ? M.U[(int64_t)(row0 + a) * r + c] : 0.0f;
-    }
     __syncthreads();
-    // W[k][col + c] = sum_{q >= k} R[k][q] V[col + c][q], in registers
+    // W[k][col + c] = sum_{q >= k} R[k][q] V[col + c][q]
     float w[RMAX][CPT];
 #pragma unroll
     for (int k = 0; k < RMAX; ++k)
@@ -581,69 +603,47 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constan
             for (int q = 0; q < RMAX; ++q) acc = fmaf(Rs[k * 33 + q], Vs[j * (RMAX + 1) + q], acc);
             w[k][c] = acc;
         }
-    if (col >= n) return;   // n % 4 == 0 and CPT divides 4: a thread's columns are all in or all out
+    if (col >= n) return;   // n % 4 == 0: a thread's columns are all in or all out
 
-    const int rbeg = warp * RPW;
-    for (int a0 = rbeg; a0 < rbeg + RPW; a0 += 4) {
-        float av[4][CPT], cv[4][CPT];
+    for (int base = row0 + warp; base < row_end; base += 8 * RF) {
+        float av[RF][CPT], cv[RF][CPT];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int row = row0 + a0 + u;
-            const int64_t off = (int64_t)row * n + col;
-            if (row < m) {
-                if (HAS_E && M.E) {
-                    if constexpr (CPT == 4) {
-                        const float4 v = __ldcs((const float4 *)(M.A + off));
-                        av[u][0] = v.x; av[u][1] = v.y; av[u][2] = v.z; av[u][3] = v.w;
-                    } else {
-                        const float2 v = __ldcs((const float2 *)(M.A + off));
-                        av[u][0] = v.x; av[u][1] = v.y;
-                    }
-                }
-                if (HAS_C && M.C) {
-                    if constexpr (CPT == 4) {
-                        const float4 v = __ldcs((const float4 *)(M.C + off));
-                        cv[u][0] = v.x; cv[u][1] = v.y; cv[u][2] = v.z; cv[u][3] = v.w;
-                    } else {
-                        const float2 v = __ldcs((const float2 *)(M.C + off));
-                        cv[u][0] = v.x; cv[u][1] = v.y;
-                    }
-                }
+        for (int u = 0; u < RF; ++u) {
+            const int row = base + 8 * u;
+            if (row < row_end) {
+                const int64_t off = (int64_t)row * n + col;
+                if (HAS_E && M.E) Vec<CPT>::load(M.A + off, av[u]);
+                if (HAS_C && M.C) Vec<CPT>::load(M.C + off, cv[u]);
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int row = row0 + a0 + u;
-            if (row >= m) break;
+        for (int u = 0; u < RF; ++u) {
+            const int row = base + 8 * u;
+            if (row >= row_end) break;
+            float ur[RMAX];
+            const float *urow = M.U + (int64_t)row * r;
+#pragma unroll
+            for (int k = 0; k < RMAX; ++k) ur[k] = (k < r) ? __ldg(urow + k) : 0.0f;
             float d[CPT];
 #pragma unroll
-            for (int c = 0; c < CPT; ++c) d[c] = 0.0f;
-            const float *urow = Us + (a0 + u) * RMAX;
+            for (int c = 0; c < CPT; ++c) {
+                float acc = 0.0f;
 #pragma unroll
-            for (int k = 0; k < RMAX; k += 4) {
-                const float4 uk = *(const float4 *)(urow + k);
-#pragma unroll
-                for (int c = 0; c < CPT; ++c) {
-                    d[c] = fmaf(uk.x, w[k][c], d[c]);
-                    d[c] = fmaf(uk.y, w[k + 1][c], d[c]);
-                    d[c] = fmaf(uk.z, w[k + 2][c], d[c]);
-                    d[c] = fmaf(uk.w, w[k + 3][c], d[c]);
-                }
+                for (int k = 0; k < RMAX; ++k) acc = fmaf(ur[k], w[k][c], acc);
+                d[c] = acc;
             }
             const int64_t off = (int64_t)row * n + col;
             if (HAS_E && M.E) {
-                if constexpr (CPT == 4)
-                    __stcs((float4 *)(M.E + off), make_float4(av[u][0] - d[0], av[u][1] - d[1], av[u][2] - d[2],
-                                                              av[u][3] - d[3]));
-                else
-                    __stcs((float2 *)(M.E + off), make_float2(av[u][0] - d[0], av[u][1] - d[1]));
+                float e[CPT];
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) e[c] = av[u][c] - d[c];
+                Vec<CPT>::store(M.E + off, e);
             }
             if (HAS_C && M.C) {
-                if constexpr (CPT == 4)
-                    __stcs((float4 *)(M.C + off), make_float4(cv[u][0] + d[0], cv[u][1] + d[1], cv[u][2] + d[2],
-                                                              cv[u][3] + d[3]));
-                else
-                    __stcs((float2 *)(M.C + off), make_float2(cv[u][0] + d[0], cv[u][1] + d[1]));
+                float o[CPT];
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) o[c] = cv[u][c] + d[c];
+                Vec<CPT>::store(M.C + off, o);
             }
         }
     }

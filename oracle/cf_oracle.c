@@ -8,9 +8,9 @@
  *
  * Sources (page title, then section):
  *  - "Accelerating Parallel Diffusion Model Serving with Residual Compression"
- *    (arXiv 2507.17511), abstract: the codec transmits compressed residuals,
- *    i.e. step-wise activation differences, and adds lightweight error
- *    feedback so that compression error does not accumulate.
+ *    (arXiv 2507.17511), abstract: only the compressed difference between an
+ *    activation and its value at the previous denoising step is sent, and a
+ *    cheap error-feedback term keeps compression error from building up.
  *  - Same paper, reproducibility table, "Dataset Splits" row (Appendix D,
  *    Figure 8): a 1-step uncompressed warmup initialises the base tensor used
  *    for later residuals.
