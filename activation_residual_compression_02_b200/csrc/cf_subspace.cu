@@ -31,6 +31,8 @@
 // MMAs, frees TMEM and returns.
 #include <cuda.h>
 
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "cf_internal.h"
@@ -69,6 +71,7 @@ struct GemmParams {
     int out_ld;        // leading dimension of the transposed output
     uint32_t *status;
     unsigned long long wait_ns;
+    int starve;        // fault-injection hook for tests: the producer issues no loads
 };
 
 // ------------------------------------------------------- PTX wrappers ----
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             uint32_t it = 0;
-            bool ok = true;
+            bool ok = !p.starve;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 const int mi = tile / p.tiles_per_mat;
                 const int mt = tile - mi * p.tiles_per_mat;
@@ -759,6 +762,15 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
         gp->out_mode = out_mode;
         gp->status = pl.status;
         gp->wait_ns = kWaitNs;
+        // Fault injection for the failure-detection test: with
+        // CF_TEST_STARVE_GEMM=1 the producer loads nothing, so the consumers'
+        // bounded waits on the "tile landed" barriers run out (after 20 ms) and
+        // the kernel returns with the timeout bit set in the status word.
+        const char *starve = getenv("CF_TEST_STARVE_GEMM");
+        if (starve && starve[0] == '1') {
+            gp->starve = 1;
+            gp->wait_ns = 20000000ull;
+        }
         bool ok;
         if (!mn_major) {
             gp->tiles_per_mat = (int)((m + kBM - 1) / kBM);

@@ -165,6 +165,7 @@ def test_argument_errors_launch_nothing(cf):
 FULL = [
     ("flux", synth.FLUX, 3),
     ("cogvideox", synth.COGVIDEOX, 3),
+    ("stress", synth.STRESS, 2),
 ]
 
 
