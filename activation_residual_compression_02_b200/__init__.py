@@ -15,4 +15,4 @@ from ._cf import (  # noqa: F401
     CF_MODE_LOWRANK, CF_MODE_QUANT, CF_OK, EXPORTED, CfError, Context, Slot, cf_check, cf_compress, cf_create,
     cf_decompress, cf_destroy, cf_lowrank, cf_lowrank_noalloc, cf_payload_bytes, lib, NOALLOC_SCRATCH_BYTES,
 )
-from .state import QuantState, alloc_quant_state  # noqa: F401
+from .state import HostStreamCodec, QuantState, alloc_quant_state  # noqa: F401

@@ -335,41 +335,51 @@ def run_cf(args, w):
     ach_pair = (bc + bd) * n_elem / (ms_per_step * 1e-3) / 1e9
 
     # ---- end to end through the public API, host buffers -----------------
+    # Pinned host activations in, payload (codes + scales) back to pinned host
+    # memory, every step; HostStreamCodec overlaps the host-to-device copy of
+    # step t+1 and the device-to-host copy of step t-1 with the codec on step t.
     e2e = None
     if not args.no_e2e:
-        n_host = min(4, len(slot_lists))
-        host_x = [[X[1 + j][s].cpu().pin_memory() for s in range(w.slots)] for j in range(n_host)]
-        dev_x = [torch.empty_like(X[0][s]) for s in range(w.slots)]
-        host_codes = [torch.empty(st.codes[s].numel(), dtype=torch.uint8).pin_memory() for s in range(w.slots)]
-        host_scales = [torch.empty(st.scales[s].numel(), dtype=torch.float32).pin_memory() for s in range(w.slots)]
-        e2e_slots = st.slots(dev_x)
-        e2e_steps = max(3, min(args.steps, 20))
+        hc = cf.HostStreamCodec(shapes, bits=w.bits, group=w.group, device=dev)
+        n_host = min(4, nsteps)
+        host_x = []
+        for j in range(n_host):
+            buf, views = hc.st.activation_buffer(pin=True)
+            for s_, v in enumerate(views):
+                v.copy_(X[j][s_])
+            host_x.append(buf)
+        host_pay = [hc.st.payload_buffers(pin=True) for _ in range(2)]
         h2d = x_bytes
-        d2h = sum(c.numel() for c in host_codes) + 4 * sum(s_.numel() for s_ in host_scales)
+        d2h = host_pay[0][0].numel() + 4 * host_pay[0][2].numel()
+        e2e_steps = max(3, min(args.steps, 30))
 
-        def e2e_step(i):
-            hx = host_x[i % n_host]
-            for s in range(w.slots):
-                dev_x[s].copy_(hx[s], non_blocking=True)
-            ctx.compress(e2e_slots, i + 1, stream)
-            ctx.decompress(e2e_slots, i + 1, stream)
-            for s in range(w.slots):
-                host_codes[s].copy_(st.codes[s], non_blocking=True)
-                host_scales[s].copy_(st.scales[s], non_blocking=True)
+        def e2e_step(t):
+            hp = host_pay[t % 2]
+            hc.step(t, host_x[t % n_host], hp[0], hp[2])
 
         e2e_step(0)
-        torch.cuda.synchronize()
+        for t in range(1, 3):
+            e2e_step(t)
+        hc.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(e2e_steps):
-            e2e_step(i + 1)
-        e1.record(stream)
-        torch.cuda.synchronize()
+        e0.record(hc.s_h2d)
+        for t in range(3, 3 + e2e_steps):
+            e2e_step(t)
+        for s_ in (hc.s_codec, hc.s_d2h):
+            ev = torch.cuda.Event()
+            ev.record(s_)
+            hc.s_h2d.wait_event(ev)
+        e1.record(hc.s_h2d)
+        hc.synchronize()
+        if hc.check() != 0:
+            raise RuntimeError("device status after the e2e run")
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
         e2e = {"value": world * x_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
-               "host_inputs": f"{n_host} pinned host copies of the step inputs, cycled"}
+               "host_inputs": f"{n_host} pinned host copies of the step inputs, cycled; copies overlapped with "
+                              "the codec on three streams"}
+        del hc
     status = ctx.check()
     if status != 0:
         raise RuntimeError(f"device status {status}")
@@ -482,7 +492,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cf", "reference"], default="cf")
     ap.add_argument("--workload", default="flux", choices=["flux", "cogvideox", "stress", "tiny", "lowrank"])
-    ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--cpu-steps", type=int, default=8)
     ap.add_argument("--slots", type=int, default=None, help="override the slot count (profiling a smaller case)")
     ap.add_argument("--budget", type=float, default=120.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-e2e", action="store_true")

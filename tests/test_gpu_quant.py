@@ -208,3 +208,34 @@ def test_full_size_sampled_rows_bit_exact(cf, oracle, name, w, steps):
         rel = torch.linalg.vector_norm(st.cache[s] + st.err[s] - x) / torch.linalg.vector_norm(x)
         assert rel.item() <= 1e-6
     assert ctx.check() == cf.CF_OK
+
+
+def test_host_stream_codec_matches_oracle(cf, oracle):
+    """Host-fed pipeline (copies on their own streams, double-buffered inputs
+    and payloads): the payload that reaches the host each step is bit-exact."""
+    shapes = [(64, 512), (37, 256), (128, 768)]
+    bits, group = 2, 128
+    hc = cf.HostStreamCodec(shapes, bits=bits, group=group)
+    ors = [oracle.QuantSlot(bits, group) for _ in shapes]
+    streams = [synth.SlotStream(synth.FLUX.scaled(rows=r, cols=c), slot=i) for i, (r, c) in enumerate(shapes)]
+    steps = 6
+    xs = [[s.next() for s in streams] for _ in range(steps)]
+    host_x, host_pay = [], []
+    for t in range(steps):
+        buf, views = hc.st.activation_buffer(pin=True)
+        for v, x in zip(views, xs[t]):
+            v.copy_(x.reshape(-1))
+        host_x.append(buf)
+        host_pay.append(hc.st.payload_buffers(pin=True))
+    for t in range(steps):
+        hc.step(t, host_x[t], host_pay[t][0], host_pay[t][2])
+    assert hc.check() == cf.CF_OK
+    for t in range(steps):
+        for i, x in enumerate(xs[t]):
+            ors[i].step(t, u16(x))
+            if t > 0:
+                assert np.array_equal(host_pay[t][1][i].numpy(), ors[i].codes), (t, i)
+                assert np.array_equal(host_pay[t][3][i].numpy(), ors[i].scales), (t, i)
+    for i in range(len(shapes)):
+        assert np.array_equal(hc.st.cache[i].cpu().numpy(), ors[i].cache)
+        assert np.array_equal(hc.st.err[i].cpu().numpy(), ors[i].err)
