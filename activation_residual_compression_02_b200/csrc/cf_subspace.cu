@@ -652,6 +652,154 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constan
     }
 }
 
+// Apply for r <= 16 with r % 4 == 0: the same arithmetic as k_apply<16>, but
+// the rows of A (and C) and U travel through a per-thread ring of cp.async
+// copies in shared memory, kAsyncStages deep, so that each thread keeps
+// (kAsyncStages - 1) * kAsyncRF rows in flight without holding them in
+// registers.  A thread only reads its own A/C copies; the U row of a warp is
+// copied by lanes 0..r/4-1 and shared after __syncwarp.
+constexpr int kAsyncRF = 4;
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <bool HAS_E, bool HAS_C>
+__host__ __device__ constexpr int async_stages()
+{
+    return (HAS_E && HAS_C) ? 3 : 4;
+}
+
+template <bool HAS_E, bool HAS_C>
+constexpr size_t async_smem_bytes()
+{
+    return (size_t)async_stages<HAS_E, HAS_C>() * kAsyncRF *
+           ((HAS_E ? kApplyThreads * 16 : 0) + (HAS_C ? kApplyThreads * 16 : 0) + 8 * 64);
+}
+
+template <bool HAS_E, bool HAS_C>
+__global__ void __launch_bounds__(kApplyThreads, 2) k_apply_async(const __grid_constant__ ApplyParams p)
+{
+    constexpr int S = async_stages<HAS_E, HAS_C>();
+    constexpr int RF = kAsyncRF;
+    constexpr int CPT = 4, COLS = 128, RMAX = 16;
+    const int per_mat = p.row_tiles * p.col_tiles;
+    const int mi = blockIdx.x / per_mat;
+    const int t = blockIdx.x - mi * per_mat;
+    const int ct = t % p.col_tiles, rt = t / p.col_tiles;
+    const ApplyMat &M = p.mat[mi];
+    const int r = p.r, n = p.n, m = p.m;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row0 = rt * kApplyRows;
+    const int row_end = min(m, row0 + kApplyRows);
+    const int col = ct * COLS + lane * CPT;
+    const bool col_ok = col < n;    // n % 4 == 0: a thread's 4 columns are all in or all out
+
+    extern __shared__ __align__(16) uint8_t apply_smem[];
+    float4 *ringA = reinterpret_cast<float4 *>(apply_smem);
+    float4 *ringC = ringA + (HAS_E ? S * RF * kApplyThreads : 0);
+    float *ringU = reinterpret_cast<float *>(ringC + (HAS_C ? S * RF * kApplyThreads : 0));
+    __shared__ float Rs[32 * 33];
+    __shared__ float Vs[COLS * (RMAX + 1)];
+    for (int i = tid; i < 32 * 33; i += kApplyThreads) {
+        const int a = i / 33, b = i - a * 33;
+        Rs[i] = (a < r && b < r) ? M.R[a * r + b] : 0.0f;
+    }
+    for (int i = tid; i < COLS * RMAX; i += kApplyThreads) {
+        const int j = i / RMAX, c = i - j * RMAX;
+        const int gc = ct * COLS + j;
+        Vs[j * (RMAX + 1) + c] = (gc < n && c < r) ? M.V[(int64_t)gc * r + c] : 0.0f;
+    }
+    // U slots past column r are never copied: they must read as zero
+    for (int i = tid; i < S * RF * 8 * 16; i += kApplyThreads) ringU[i] = 0.0f;
+    __syncthreads();
+    float w[RMAX][CPT];
+#pragma unroll
+    for (int k = 0; k < RMAX; ++k)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            float acc = 0.0f;
+            const int j = lane * CPT + c;
+#pragma unroll
+            for (int q = 0; q < RMAX; ++q) acc = fmaf(Rs[k * 33 + q], Vs[j * (RMAX + 1) + q], acc);
+            w[k][c] = acc;
+        }
+
+    const int nrows = row_end - row0;
+    const int ngroups = nrows > 0 ? (nrows + 8 * RF - 1) / (8 * RF) : 0;
+    const int uchunks = r / 4;
+    auto issue = [&](int g, int slot) {
+#pragma unroll
+        for (int u = 0; u < RF; ++u) {
+            const int row = row0 + g * 8 * RF + warp + 8 * u;
+            const bool valid = row < row_end;
+            const int safe_row = valid ? row : row0;
+            const int64_t off = (int64_t)safe_row * n + (col_ok ? col : 0);
+            // a matrix without E (or C) reads nothing: zero bytes from a valid address
+            if (HAS_E)
+                cp_async16(&ringA[(slot * RF + u) * kApplyThreads + tid], M.E ? M.A + off : M.U,
+                           valid && col_ok && M.E != nullptr);
+            if (HAS_C)
+                cp_async16(&ringC[(slot * RF + u) * kApplyThreads + tid], M.C ? M.C + off : M.U,
+                           valid && col_ok && M.C != nullptr);
+            if (lane < uchunks)
+                cp_async16(&ringU[((slot * RF + u) * 8 + warp) * 16 + lane * 4], M.U + (int64_t)safe_row * r + lane * 4,
+                           valid);
+        }
+    };
+#pragma unroll
+    for (int s = 0; s < S - 1; ++s) {
+        if (s < ngroups) issue(s, s);
+        cp_async_commit();
+    }
+    for (int g = 0; g < ngroups; ++g) {
+        const int gi = g + S - 1;
+        if (gi < ngroups) issue(gi, gi % S);
+        cp_async_commit();
+        cp_async_wait<S - 1>();
+        __syncwarp();
+        const int slot = g % S;
+#pragma unroll
+        for (int u = 0; u < RF; ++u) {
+            const int row = row0 + g * 8 * RF + warp + 8 * u;
+            if (row >= row_end || !col_ok) continue;
+            const float4 *urow4 = reinterpret_cast<const float4 *>(&ringU[((slot * RF + u) * 8 + warp) * 16]);
+            float d[CPT] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k4 = 0; k4 < RMAX / 4; ++k4) {
+                const float4 uk = urow4[k4];
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    d[c] = fmaf(uk.x, w[4 * k4][c], d[c]);
+                    d[c] = fmaf(uk.y, w[4 * k4 + 1][c], d[c]);
+                    d[c] = fmaf(uk.z, w[4 * k4 + 2][c], d[c]);
+                    d[c] = fmaf(uk.w, w[4 * k4 + 3][c], d[c]);
+                }
+            }
+            const int64_t off = (int64_t)row * n + col;
+            if (HAS_E && M.E) {
+                const float4 a = ringA[(slot * RF + u) * kApplyThreads + tid];
+                __stcs((float4 *)(M.E + off), make_float4(a.x - d[0], a.y - d[1], a.z - d[2], a.w - d[3]));
+            }
+            if (HAS_C && M.C) {
+                const float4 c = ringC[(slot * RF + u) * kApplyThreads + tid];
+                __stcs((float4 *)(M.C + off), make_float4(c.x + d[0], c.y + d[1], c.z + d[2], c.w + d[3]));
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+}
+
 // ----------------------------------------------------------- host side ---
 using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                               const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -893,6 +1041,24 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
         const unsigned blocks = (unsigned)((int64_t)cnt * ap->row_tiles * ap->col_tiles);
         using Fn = void (*)(ApplyParams);
         Fn fn;
+        if (rmax == 16 && pl.r % 4 == 0) {
+            // copies through a cp.async ring (U rows are 16-byte chunks when r % 4 == 0)
+            size_t smem;
+            if (has_e && has_c) {
+                fn = k_apply_async<true, true>;
+                smem = async_smem_bytes<true, true>();
+            } else if (has_e) {
+                fn = k_apply_async<true, false>;
+                smem = async_smem_bytes<true, false>();
+            } else {
+                fn = k_apply_async<false, true>;
+                smem = async_smem_bytes<false, true>();
+            }
+            cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            fn<<<blocks, kApplyThreads, smem, stream>>>(*ap);
+            err = cudaGetLastError();
+            continue;
+        }
         if (rmax == 16)
             fn = has_e ? (has_c ? k_apply<16, true, true> : k_apply<16, true, false>) : k_apply<16, false, true>;
         else

@@ -464,7 +464,32 @@ def run_lowrank_bench(args, w):
     elems = k * m * n
     peak, peak_kind = hbm_peak()
     alg_bytes = elems * (4 + 4)          # A read once, E written once
+    sched_bytes = elems * (4 * (2 * T + 2) + 4)   # A read by each of the 2T+1 products and the apply, E written
     flops = 2.0 * (2 * T + 1) * m * n * r * k + 2.0 * m * n * r * k
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import concurrent.futures
+
+        import oracle
+
+        oracle.build()
+        nsample = min(8, k)
+        Ah = [A[i].cpu().numpy() for i in range(nsample)]
+        Qh = [Q0[i].cpu().numpy() for i in range(nsample)]
+
+        def work(i):
+            Uo, Ro, Vo = oracle.subspace_iteration(Ah[i], Qh[i], T)
+            oracle.lowrank_apply(Ah[i], Uo, Ro, Vo)
+
+        threads = min(cpu_cores(), nsample)
+        t0 = time.perf_counter()
+        with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(work, range(nsample)))
+        dt = time.perf_counter() - t0
+        cpu = {"value": nsample * m * n * 4 / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{nsample} of the {k} matrices (Algorithm 3 in fp64 plus the apply), one matrix per host "
+                         f"thread, {threads} threads, {dt:.1f} s wall"}
     line = {
         "metric": "low-rank codec GB/s of fp32 residual input (Algorithm 3 + apply)", "value":
             world * elems * 4 / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -476,8 +501,13 @@ def run_lowrank_bench(args, w):
         "roofline": {"bound": "hbm", "kernel": "whole cf_lowrank call", "achieved": alg_bytes / (ms * 1e-3) / 1e9,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": alg_bytes / (ms * 1e-3) / 1e9 / peak, "traffic": None,
-                     "alg_bytes_per_step": alg_bytes, "tflops": flops / (ms * 1e-3) / 1e12},
-        "gpu_launches": None, "e2e": None, "cpu_baseline": None, "clocks": clk.summary(),
+                     "alg_bytes_per_step": alg_bytes, "tflops": flops / (ms * 1e-3) / 1e12,
+                     "schedule_bytes_per_step": sched_bytes,
+                     "schedule_frac": sched_bytes / (ms * 1e-3) / 1e9 / peak,
+                     "note": "alg bytes count A once and E once; the schedule reads A from HBM in each of the "
+                             "2T+1 products and in the apply"},
+        "gpu_launches": args.steps * (2 * (T + 2) + (2 * T + 1) + 1), "e2e": None, "cpu_baseline": cpu,
+        "clocks": clk.summary(),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
