@@ -22,7 +22,7 @@ CF_MODE_QUANT, CF_MODE_LOWRANK = 0, 1
 
 EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
             "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
-            "cf_destroy", "cf_lowrank_noalloc"]
+            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback"]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.cf_compress.restype = I
         L.cf_decompress.argtypes = [P, ctypes.POINTER(cf_slot), I, P]
         L.cf_decompress.restype = I
+        L.cf_loopback.argtypes = [P, ctypes.POINTER(cf_slot), I, P]
+        L.cf_loopback.restype = I
         L.cf_lowrank_workspace_bytes.argtypes = [P, I, I64, I64]
         L.cf_lowrank_workspace_bytes.restype = SZ
         PP = ctypes.POINTER(P)
@@ -190,6 +192,9 @@ class Context:
     def decompress(self, slots: Sequence[Slot], step: int, stream: Optional[torch.cuda.Stream] = None):
         self._raise(lib().cf_decompress(self._h, self._slots(slots), step, _stream_handle(stream)), "cf_decompress")
 
+    def loopback(self, slots: Sequence[Slot], step: int, stream: Optional[torch.cuda.Stream] = None):
+        self._raise(lib().cf_loopback(self._h, self._slots(slots), step, _stream_handle(stream)), "cf_loopback")
+
     def lowrank(self, A: List[torch.Tensor], Q0: List[torch.Tensor], U: List[torch.Tensor], R: List[torch.Tensor],
                 V: List[torch.Tensor], E: Optional[List[torch.Tensor]] = None, C: Optional[List[torch.Tensor]] = None,
                 stream: Optional[torch.cuda.Stream] = None):
@@ -214,6 +219,10 @@ def cf_compress(ctx: Context, slots, step, stream=None):
 
 def cf_decompress(ctx: Context, slots, step, stream=None):
     ctx.decompress(slots, step, stream)
+
+
+def cf_loopback(ctx: Context, slots, step, stream=None):
+    ctx.loopback(slots, step, stream)
 
 
 def cf_lowrank(ctx: Context, A, Q0, U, R, V, E=None, C=None, stream=None):

@@ -341,6 +341,29 @@ cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_
     return codec_call(ctx, slots, step, cuda_stream, false);
 }
 
+cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream)
+{
+    if (!ctx) return CF_E_ARG;
+    if (step == 0 || ctx->cfg.mode != CF_MODE_QUANT) {
+        cf_status st = codec_call(ctx, slots, step, cuda_stream, true);
+        if (st != CF_OK) return st;
+        return codec_call(ctx, slots, step, cuda_stream, false);
+    }
+    if (!(ctx->warm_sender && ctx->warm_receiver))
+        return fail(ctx, CF_E_STATE, "step %d before the warmup step (step 0) on this context", step);
+    const int n = (int)ctx->shapes.size();
+    if (n > 0 && !slots) return fail(ctx, CF_E_ARG, "slots is NULL");
+    for (int i = 0; i < n; ++i) {
+        if (ctx->shapes[i].rows == 0) continue;
+        cf_status st = check_quant_slot(ctx, slots[i], i, true, step);
+        if (st == CF_OK) st = check_quant_slot(ctx, slots[i], i, false, step);
+        if (st != CF_OK) return st;
+    }
+    cf_status st = run_quant(ctx, slots, cf::QuantOp::Loopback, (cudaStream_t)cuda_stream);
+    if (st == CF_OK) ctx->err.clear();
+    return st;
+}
+
 size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_t n)
 {
     if (!ctx || ctx->cfg.mode != CF_MODE_LOWRANK || nmat < 0 || m < ctx->cfg.rank || n < ctx->cfg.rank) return 0;

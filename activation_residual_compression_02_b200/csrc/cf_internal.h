@@ -40,7 +40,7 @@ struct QuantLaunch {
     QuantSlotDesc slot[kMaxSlotsPerLaunch];
 };
 
-enum class QuantOp { WarmupSender, WarmupReceiver, Compress, Decompress };
+enum class QuantOp { WarmupSender, WarmupReceiver, Compress, Decompress, Loopback };
 
 // Launch one grouped quantised kernel over `lp` (host-built slot table;
 // tile0/ntiles are filled in here for the chosen kernel's tile size).

@@ -323,6 +323,29 @@ def run_cf(args, w):
         raise RuntimeError(f"device status {status}")
     ms_local = start.elapsed_time(end)
     ms = max_over_ranks(ms_local, world)
+
+    # ---- the same steps through cf_loopback (sender and receiver fused) ---
+    lb = None
+    if not args.no_loopback:
+        for i in range(1, args.warmup + 1):
+            if L.cf_loopback(h, c_slots[(i - 1) % len(c_slots)], i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+        barrier(world)
+        torch.cuda.synchronize()
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        l0.record(stream)
+        for k in range(args.steps):
+            i = args.warmup + 1 + k
+            if L.cf_loopback(h, c_slots[(i - 1) % len(c_slots)], i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+        l1.record(stream)
+        torch.cuda.synchronize()
+        lb_ms = max_over_ranks(l0.elapsed_time(l1), world) / args.steps
+        lb_bytes = (22.0 + w.bits / 8 + 4 / w.group) * n_elem
+        lb = {"ms_per_step": lb_ms, "value": world * x_bytes / (lb_ms * 1e-3) / 1e9, "unit": "GB/s",
+              "alg_bytes_per_step": lb_bytes, "achieved": lb_bytes / (lb_ms * 1e-3) / 1e9,
+              "frac": lb_bytes / (lb_ms * 1e-3) / 1e9 / hbm_peak()[0],
+              "note": "cf_loopback: compress and decompress of a step in one launch (both sides on this GPU)"}
     comp_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     deco_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     ms_per_step = ms / args.steps
@@ -412,6 +435,7 @@ def run_cf(args, w):
                                 "alg_bytes_per_launch": bd * n_elem, "ms_per_launch": deco_ms},
         "roofline_step": {"achieved": ach_pair, "frac": ach_pair / peak, "frac_of_8tbs": ach_pair / 8000.0,
                           "alg_bytes_per_step": (bc + bd) * n_elem},
+        "loopback": lb,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
@@ -527,6 +551,7 @@ def main():
     ap.add_argument("--budget", type=float, default=120.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-loopback", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

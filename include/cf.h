@@ -157,6 +157,18 @@ cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
  * Errors as cf_compress (CF_E_STATE: step >= 1 before a receiver warmup). */
 cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
 
+/* Sender and receiver of step `step` in one pass, for when both sides of a
+ * slot live on this device (e.g. the local shard of an all-gather).  The
+ * results are bit-identical to cf_compress followed by cf_decompress: the
+ * receiver's C += deq reuses the values the sender dequantised, and the
+ * payload is still written (for transmission) but not read back.  In
+ * quantised mode a step >= 1 is one fused grouped launch moving k/8 + 4/G
+ * bytes per element less than the pair; step 0, and every step in low-rank
+ * mode, run the two sides one after the other.  Uses x, base, err, cache,
+ * codes, scales (and q0, U, R, V in low-rank mode).  Errors as cf_compress
+ * (CF_E_STATE: step >= 1 before the warmup). */
+cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
+
 /* Workspace cf_lowrank needs for nmat matrices of m x n at this context's
  * rank: the r-column blocks of Algorithm 3 (Q^T, P^T, P, Z, padded to 16 or
  * 32 columns) and their fp64 Gram matrices, about 4*rp*(2m + 2n) + 8 KB

@@ -27,7 +27,8 @@ def u16(t):
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16).ravel()
 
 
-def run_case(cf, oracle, shapes, steps, bits, group, ss=0, seed=0, w=synth.TINY, check_every_step=True):
+def run_case(cf, oracle, shapes, steps, bits, group, ss=0, seed=0, w=synth.TINY, check_every_step=True,
+             loopback=False):
     """Run the codec on the GPU and the oracle on the CPU for `steps` steps."""
     ctx = cf.Context(shapes, bits=bits, group=group, sign_scale=ss)
     st = cf.QuantState(shapes, bits, group)
@@ -37,8 +38,11 @@ def run_case(cf, oracle, shapes, steps, bits, group, ss=0, seed=0, w=synth.TINY,
         xs_cpu = [s.next() for s in streams]
         xs = [x.cuda() for x in xs_cpu]
         slots = st.slots(xs)
-        ctx.compress(slots, t)
-        ctx.decompress(slots, t)
+        if loopback:
+            ctx.loopback(slots, t)
+        else:
+            ctx.compress(slots, t)
+            ctx.decompress(slots, t)
         for i, x in enumerate(xs_cpu):
             ors[i].step(t, u16(x))
         if check_every_step or t == steps - 1:
@@ -68,6 +72,15 @@ def test_ragged_multi_slot_grouped_launch(cf, oracle, bits, group):
     shapes = [(37, 512), (1, 256), (0, 256), (300, 768), (5, 1024), (129, 256)]
     shapes = [(r, c) for r, c in shapes if c % group == 0]
     run_case(cf, oracle, shapes, 4, bits, group, w=synth.COGVIDEOX)
+
+
+@pytest.mark.parametrize("bits,group,ss", [(2, 128, 0), (4, 64, 0), (1, 128, 0), (1, 256, 1), (2, 8, 0), (4, 256, 0)])
+def test_loopback_bit_exact(cf, oracle, bits, group, ss):
+    """cf_loopback (sender and receiver fused in one pass) equals the oracle's
+    compress + decompress bit for bit, on ragged multi-slot launches."""
+    shapes = [(37, 512), (1, 256), (0, 256), (300, 768), (129, 256)]
+    shapes = [(r, c) for r, c in shapes if c % group == 0]
+    run_case(cf, oracle, shapes, 4, bits, group, ss, w=synth.FLUX, loopback=True)
 
 
 def test_grouped_equals_per_slot(cf):
@@ -239,3 +252,18 @@ def test_host_stream_codec_matches_oracle(cf, oracle):
     for i in range(len(shapes)):
         assert np.array_equal(hc.st.cache[i].cpu().numpy(), ors[i].cache)
         assert np.array_equal(hc.st.err[i].cpu().numpy(), ors[i].err)
+
+
+def test_tma_staged_variant_bit_exact():
+    """The TMA-staged compress/decompress variant (CF_QUANT_STAGING=tma, read
+    once per process) passes the same bit-exact parity, in a fresh process."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CF_QUANT_STAGING="tma")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+                        os.path.join(root, "tests", "test_gpu_quant.py"), "-k", "tiny_workload or ragged or stress"],
+                       capture_output=True, text=True, env=env, cwd=root, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
