@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
         _lib.cfo_cholqr.argtypes = [I64, I, P, P, P]
         _lib.cfo_subspace_iteration.argtypes = [I64, I64, I, I, P, P, P, P, P]
         _lib.cfo_lowrank_apply.argtypes = [I64, I64, I, P, P, P, P, P, P, P, P]
+        _lib.cfo_warmup_sender_lean.argtypes = [I64, P, P, P]
+        _lib.cfo_warmup_receiver_lean.argtypes = [I64, P, P]
+        _lib.cfo_compress_lean.argtypes = [I64, I, I, I, P, P, P, P, P, U32P]
+        _lib.cfo_decompress_lean.argtypes = [I64, I, I, P, P, P]
     return _lib
 
 
@@ -154,16 +158,54 @@ def get_code(stream: np.ndarray, i: int, bits: int) -> int:
     return int(c.value)
 
 
-class QuantSlot:
-    """Sender + receiver state of one slot, stepped by the oracle."""
+def compress_lean(x_bits: np.ndarray, base: np.ndarray, err_bits: np.ndarray, bits: int, group: int,
+                  sign_scale: int = 0) -> Tuple[np.ndarray, np.ndarray, int]:
+    """Sender step with bf16 E (raw bits, updated in place)."""
+    x = _u16(x_bits).ravel()
+    n = x.size
+    assert base.dtype == np.uint16 and err_bits.dtype == np.uint16 and err_bits.size == n
+    codes = np.zeros(n * bits // 8, np.uint8)
+    scales = np.empty(n // group, np.float32)
+    flags = ctypes.c_uint32(0)
+    _check(lib().cfo_compress_lean(n, bits, group, sign_scale, _ptr(x), _ptr(base), _ptr(err_bits), _ptr(codes),
+                                   _ptr(scales), ctypes.byref(flags)), "compress_lean")
+    return codes, scales, int(flags.value)
 
-    def __init__(self, bits: int, group: int, sign_scale: int = 0):
-        self.bits, self.group, self.sign_scale = bits, group, sign_scale
+
+def decompress_lean(codes: np.ndarray, scales: np.ndarray, cache_bits: np.ndarray, bits: int, group: int) -> None:
+    """Receiver step with a bf16 cache (raw bits, updated in place)."""
+    assert cache_bits.dtype == np.uint16 and cache_bits.flags["C_CONTIGUOUS"]
+    _check(lib().cfo_decompress_lean(cache_bits.size, bits, group, _ptr(np.ascontiguousarray(codes)),
+                                     _ptr(np.ascontiguousarray(scales)), _ptr(cache_bits)), "decompress_lean")
+
+
+class QuantSlot:
+    """Sender + receiver state of one slot, stepped by the oracle.
+
+    ``lean=True`` keeps E and C in bf16 (raw 16-bit patterns) instead of fp32.
+    """
+
+    def __init__(self, bits: int, group: int, sign_scale: int = 0, lean: bool = False):
+        self.bits, self.group, self.sign_scale, self.lean = bits, group, sign_scale, lean
         self.base = self.err = self.cache = None
         self.codes = self.scales = None
         self.flags = 0
 
     def step(self, t: int, x_bits: np.ndarray) -> None:
+        if self.lean:
+            x = _u16(x_bits).ravel()
+            if t == 0:
+                self.base = np.empty_like(x)
+                self.err = np.empty_like(x)
+                self.cache = np.empty_like(x)
+                _check(lib().cfo_warmup_sender_lean(x.size, _ptr(x), _ptr(self.base), _ptr(self.err)), "warmup")
+                _check(lib().cfo_warmup_receiver_lean(x.size, _ptr(x), _ptr(self.cache)), "warmup")
+                return
+            self.codes, self.scales, fl = compress_lean(x, self.base, self.err, self.bits, self.group,
+                                                        self.sign_scale)
+            self.flags |= fl
+            decompress_lean(self.codes, self.scales, self.cache, self.bits, self.group)
+            return
         if t == 0:
             self.base, self.err = warmup_sender(x_bits)
             self.cache = warmup_receiver(x_bits)

@@ -58,11 +58,15 @@ static float bf16_to_float(uint16_t h)
     return f;
 }
 
-static uint32_t float_bits(float f)
+/* Round a float to bf16 with round-to-nearest-even on the 16 dropped bits
+ * (a NaN stays a quiet NaN). */
+static uint16_t float_to_bf16(float f)
 {
     uint32_t u;
     memcpy(&u, &f, sizeof u);
-    return u;
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u);
+    const uint32_t lsb = (u >> 16) & 1u;
+    return (uint16_t)((u + 0x7fffu + lsb) >> 16);
 }
 
 /* ------------------------------------------------------- bit stream ----- */
@@ -409,5 +413,64 @@ int cfo_lowrank_apply(int64_t m, int64_t n, int r, const float *A, const double 
             if (C_out) C_out[i * n + j] = (double)C_in[i * n + j] + dv;
         }
     free(W);
+    return CFO_OK;
+}
+
+/* ======================================== lean state (bf16 E and C) ==== */
+/* The same codec with the error-feedback buffer E and the receiver cache C
+ * kept in bf16: every arithmetic step stays one binary32 operation, and the
+ * new E and C are rounded to bf16 (RNE) when they are stored.  The payload
+ * (codes, scales) is the same as in the fp32-state codec for the same A. */
+
+int cfo_warmup_sender_lean(int64_t n, const uint16_t *x, uint16_t *base, uint16_t *err)
+{
+    if (n < 0) return CFO_E_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        base[i] = x[i];
+        err[i] = 0;
+    }
+    return CFO_OK;
+}
+
+int cfo_warmup_receiver_lean(int64_t n, const uint16_t *x, uint16_t *cache)
+{
+    if (n < 0) return CFO_E_ARG;
+    for (int64_t i = 0; i < n; ++i) cache[i] = x[i];
+    return CFO_OK;
+}
+
+int cfo_compress_lean(int64_t n, int k, int G, int sign_scale, const uint16_t *x, uint16_t *base, uint16_t *err,
+                      uint8_t *codes, float *scales, uint32_t *flags_out)
+{
+    if (!valid_quant(n, k, G) || (sign_scale != 0 && sign_scale != 1)) return CFO_E_ARG;
+    uint32_t flags = 0;
+    float a[256], d[256];
+    for (int64_t g = 0; g < n / G; ++g) {
+        const int64_t i0 = g * G;
+        for (int j = 0; j < G; ++j) {
+            float diff = bf16_to_float(x[i0 + j]) - bf16_to_float(base[i0 + j]);
+            a[j] = diff + bf16_to_float(err[i0 + j]);
+            base[i0 + j] = x[i0 + j];
+        }
+        scales[g] = quantise_group(a, G, k, sign_scale, codes, i0, d, &flags);
+        for (int j = 0; j < G; ++j) err[i0 + j] = float_to_bf16(a[j] - d[j]);
+    }
+    if (flags_out) *flags_out = flags;
+    return CFO_OK;
+}
+
+int cfo_decompress_lean(int64_t n, int k, int G, const uint8_t *codes, const float *scales, uint16_t *cache)
+{
+    if (!valid_quant(n, k, G)) return CFO_E_ARG;
+    const int L = half_levels(k);
+    for (int64_t g = 0; g < n / G; ++g) {
+        const float s = scales[g];
+        for (int j = 0; j < G; ++j) {
+            const int64_t i = g * G + j;
+            const unsigned c = get_code(codes, i, k);
+            const float dv = (k == 1) ? (c ? s : -s) : level(c, L) * s;
+            cache[i] = float_to_bf16(bf16_to_float(cache[i]) + dv);
+        }
+    }
     return CFO_OK;
 }

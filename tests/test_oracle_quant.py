@@ -54,6 +54,17 @@ def test_hand_worked_group(oracle, name):
     bits, group, ss = int(c["bits"]), int(c["group"]), int(c["sign_scale"])
     x = bf16([float(v) for v in c["x"].split(",")])
     base = bf16([float(v) for v in c["base"].split(",")])
+    if c.get("state") == "bf16":
+        err = bf16([float(v) for v in c["e"].split(",")])
+        cache = bf16([float(v) for v in c["cache"].split(",")])
+        codes, scales, flags = oracle.compress_lean(x, base, err, bits, group, ss)
+        assert flags == 0
+        assert codes.tobytes() == bytes(int(b, 16) for b in c["bytes"].split(","))
+        assert scales.tolist() == [float(c["scale"])]
+        assert np.array_equal(err, bf16([float(v) for v in c["e_new"].split(",")]))
+        oracle.decompress_lean(codes, scales, cache, bits, group)
+        assert np.array_equal(cache, bf16([float(v) for v in c["cache_new"].split(",")]))
+        return
     err = floats(c["e"])
     cache = floats(c["cache"])
     codes, scales, flags = oracle.compress(x, base, err, bits, group, ss)
@@ -268,3 +279,48 @@ def test_bad_arguments_rejected(oracle):
         oracle.compress(x, x.copy(), np.zeros(24, np.float32), 3, 8)
     with pytest.raises(ValueError):
         oracle.compress(x, x.copy(), np.zeros(24, np.float32), 2, 16)  # 24 % 16 != 0
+
+
+def _bits_to_f32(b):
+    return torch.from_numpy(b.view(np.int16).copy()).view(torch.bfloat16).float().numpy()
+
+
+def _f32_to_bf16_bits(f):
+    return torch.from_numpy(np.ascontiguousarray(f, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(
+        np.uint16)
+
+
+@pytest.mark.parametrize("bits,group", [(2, 128), (4, 64), (1, 128)])
+def test_lean_state_is_the_fp32_step_rounded_to_bf16(oracle, bits, group):
+    """From a common state (E, C exact in bf16), one lean step sends the same
+    payload as the fp32-state step, and its new E and C are the fp32-state
+    results rounded to bf16 by torch (an independent round-to-nearest-even)."""
+    w = synth.FLUX.scaled(rows=24, cols=512, outlier_frac=0.01)
+    xs = synth.activations(w, 0, 4)
+    lean = oracle.QuantSlot(bits, group, lean=True)
+    for t in range(3):
+        lean.step(t, synth.bf16_bits(xs[t]).numpy().view(np.uint16).ravel().copy())
+    x3 = synth.bf16_bits(xs[3]).numpy().view(np.uint16).ravel().copy()
+    base32, err32, cache32 = lean.base.copy(), _bits_to_f32(lean.err), _bits_to_f32(lean.cache)
+    codes32, scales32, _ = oracle.compress(x3, base32, err32, bits, group)
+    oracle.decompress(codes32, scales32, cache32, bits, group)
+    lean.step(3, x3)
+    assert np.array_equal(lean.codes, codes32)
+    assert np.array_equal(lean.scales, scales32)
+    assert np.array_equal(lean.err, _f32_to_bf16_bits(err32))
+    assert np.array_equal(lean.cache, _f32_to_bf16_bits(cache32))
+    assert np.array_equal(lean.base, x3)
+
+
+def test_lean_state_error_feedback_identity(oracle):
+    """With bf16 E and C the identity C + E = X holds up to the bf16 rounding of
+    E and C at each step (a few 2^-9 relative over a handful of steps)."""
+    w = synth.COGVIDEOX.scaled(rows=32, cols=640)
+    xs = synth.activations(w, 1, 6)
+    st = oracle.QuantSlot(4, 64, lean=True)
+    for t, x in enumerate(xs):
+        st.step(t, synth.bf16_bits(x).numpy().view(np.uint16).ravel().copy())
+        x64 = x.float().numpy().ravel().astype(np.float64)
+        rec = _bits_to_f32(st.cache).astype(np.float64) + _bits_to_f32(st.err).astype(np.float64)
+        rel = np.linalg.norm(rec - x64) / np.linalg.norm(x64)
+        assert rel <= (t + 1) * 2.0 ** -9, (t, rel)
