@@ -57,9 +57,11 @@ cf_status validate_config(const cf_config *c, std::string &why)
         if (c->bits != 1 && c->bits != 2 && c->bits != 4) { why = "bits must be 1, 2 or 4"; return CF_E_ARG; }
         if (!pow2(c->group) || c->group < 8 || c->group > 256) { why = "group must be a power of two in [8, 256]"; return CF_E_ARG; }
         if (c->sign_scale != 0 && c->sign_scale != 1) { why = "sign_scale must be 0 or 1"; return CF_E_ARG; }
+        if (c->state_bf16 != 0 && c->state_bf16 != 1) { why = "state_bf16 must be 0 or 1"; return CF_E_ARG; }
         return CF_OK;
     }
     if (c->mode == CF_MODE_LOWRANK) {
+        if (c->state_bf16 != 0) { why = "the lean bf16 state is a quantised-mode option"; return CF_E_ARG; }
         if (c->rank < 1 || c->rank > 32) { why = "rank must be in [1, 32]"; return CF_E_ARG; }
         if (c->iters < 0 || c->iters > 1000) { why = "iters must be in [0, 1000]"; return CF_E_ARG; }
         return CF_OK;
@@ -152,7 +154,8 @@ cf_status run_quant(cf_ctx *ctx, const cf_slot *slots, cf::QuantOp op, cudaStrea
             d.scales = s.scales;
             d.nvec = elems / 8;
         }
-        cudaError_t e = cf::launch_quant(op, ctx->cfg.bits, ctx->cfg.group, ctx->cfg.sign_scale, *lp, stream);
+        cudaError_t e = cf::launch_quant(op, ctx->cfg.bits, ctx->cfg.group, ctx->cfg.sign_scale, ctx->cfg.state_bf16 != 0,
+                                         *lp, stream);
         if (e != cudaSuccess) {
             delete lp;
             return cuda_fail(ctx, e, "quantised codec launch");
@@ -203,7 +206,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
         for (int i = 0; i < n; ++i) {
             xs[i] = slots[i].x;
             bs[i] = slots[i].base;
-            es[i] = slots[i].err;
+            es[i] = static_cast<const float *>(slots[i].err);
             ns[i] = ctx->shapes[i].rows * ctx->shapes[i].cols;
         }
         cudaError_t e = cf::launch_residual_f32(xs.data(), bs.data(), es.data(), a_ptr.data(), ns.data(), n, stream);
@@ -223,8 +226,8 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
             m.U = slots[k].U;
             m.R = slots[k].R;
             m.V = slots[k].V;
-            m.E = sender ? slots[k].err : nullptr;
-            m.C = sender ? nullptr : slots[k].cache;
+            m.E = sender ? static_cast<float *>(slots[k].err) : nullptr;
+            m.C = sender ? nullptr : static_cast<float *>(slots[k].cache);
         }
         cf::LowrankPlan plan{};
         plan.nmat = (int)(j - i);

@@ -24,8 +24,8 @@ constexpr int kMaxSlotsPerLaunch = 128;
 struct QuantSlotDesc {
     const void *x;     // bf16
     void *base;        // bf16
-    float *err;        // fp32
-    float *cache;      // fp32
+    void *err;         // fp32, or bf16 with the lean state
+    void *cache;       // fp32, or bf16 with the lean state
     uint8_t *codes;    // packed codes
     float *scales;     // fp32 group scales
     int64_t nvec;      // elements / 8
@@ -46,7 +46,8 @@ enum class QuantOp { WarmupSender, WarmupReceiver, Compress, Decompress, Loopbac
 // tile0/ntiles are filled in here for the chosen kernel's tile size).
 // bits/group/sign_scale select the template instance.  Returns cudaSuccess or
 // the launch error.
-cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, QuantLaunch &lp, cudaStream_t stream);
+cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool lean, QuantLaunch &lp,
+                         cudaStream_t stream);
 
 // ---------------------------------------------------------------- low rank
 

@@ -23,14 +23,10 @@
 // magnitude bits (exact, and a NaN or infinity is seen as non-finite).
 #include <cuda_bf16.h>
 
-#include <stdlib.h>
-#include <string.h>
-
 #include <mutex>
 #include <unordered_map>
 
 #include "cf_internal.h"
-#include "cf_ptx.cuh"
 
 namespace cf {
 namespace {
@@ -43,20 +39,20 @@ namespace {
 // per vector (1024 x 1: 93.5% of the measured copy bandwidth, against 88% for
 // 256 x 4 at 2 CTAs/SM); decompress wants about 512 resident threads per SM
 // with 4 vectors each (94.5%, against 84% at 4 CTAs/SM).
-template <QuantOp OP>
+template <QuantOp OP, bool LEAN = false>
 struct QShape {
     static constexpr int kThreads = 256;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 0;
 };
 template <>
-struct QShape<QuantOp::Compress> {
+struct QShape<QuantOp::Compress, false> {
     static constexpr int kThreads = 1024;
     static constexpr int kUnroll = 1;
-    static constexpr int kMaxPerSm = 0;
+    static constexpr int kMaxPerSm = 1;   // 2 CTAs of 1024 fit at 32 registers, and are slower
 };
 template <>
-struct QShape<QuantOp::Loopback> {
+struct QShape<QuantOp::Loopback, false> {
     // fused sender + receiver: 9 streams per tile; best of the sweep (90.6%
     // of the copy peak), still below the separate pair (94.3%)
     static constexpr int kThreads = 256;
@@ -64,15 +60,35 @@ struct QShape<QuantOp::Loopback> {
     static constexpr int kMaxPerSm = 1;
 };
 template <>
-struct QShape<QuantOp::Decompress> {
+struct QShape<QuantOp::Decompress, false> {
     static constexpr int kThreads = 512;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 1;
 };
-template <QuantOp OP>
+// Lean state (bf16 E and C): half the state bytes per vector, so each thread
+// wants more vectors in flight (sweep on the same workload).
+template <>
+struct QShape<QuantOp::Compress, true> {
+    static constexpr int kThreads = 1024;
+    static constexpr int kUnroll = 2;
+    static constexpr int kMaxPerSm = 1;
+};
+template <>
+struct QShape<QuantOp::Loopback, true> {
+    static constexpr int kThreads = 256;
+    static constexpr int kUnroll = 8;
+    static constexpr int kMaxPerSm = 1;
+};
+template <>
+struct QShape<QuantOp::Decompress, true> {
+    static constexpr int kThreads = 1024;
+    static constexpr int kUnroll = 4;
+    static constexpr int kMaxPerSm = 1;
+};
+template <QuantOp OP, bool LEAN>
 constexpr int64_t qtile_vec()
 {
-    return (int64_t)QShape<OP>::kThreads * QShape<OP>::kUnroll;
+    return (int64_t)QShape<OP, LEAN>::kThreads * QShape<OP, LEAN>::kUnroll;
 }
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kAbsMask = 0x7fffffffu;
@@ -110,6 +126,53 @@ template <> struct CodeWord<1> { using T = uint8_t; };
 template <> struct CodeWord<2> { using T = uint16_t; };
 template <> struct CodeWord<4> { using T = uint32_t; };
 
+// State vectors (E or C) of 8 elements: fp32 (32 bytes) or, with the lean
+// state, bf16 (16 bytes, rounded to nearest even on store).
+struct F8 {
+    float4 a, b;
+};
+template <bool LEAN>
+struct StateVec {
+    using T = F8;
+    static __device__ __forceinline__ T load(const void *base, int64_t v)
+    {
+        const float4 *p = static_cast<const float4 *>(base) + 2 * v;
+        return F8{__ldcs(p), __ldcs(p + 1)};
+    }
+    static __device__ __forceinline__ void unpack(const T &s, float (&f)[8])
+    {
+        f[0] = s.a.x; f[1] = s.a.y; f[2] = s.a.z; f[3] = s.a.w;
+        f[4] = s.b.x; f[5] = s.b.y; f[6] = s.b.z; f[7] = s.b.w;
+    }
+    static __device__ __forceinline__ T zero() { return F8{make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)}; }
+    static __device__ __forceinline__ void store(void *base, int64_t v, const float (&f)[8])
+    {
+        float4 *p = static_cast<float4 *>(base) + 2 * v;
+        __stcs(p, make_float4(f[0], f[1], f[2], f[3]));
+        __stcs(p + 1, make_float4(f[4], f[5], f[6], f[7]));
+    }
+};
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+template <>
+struct StateVec<true> {
+    using T = uint4;
+    static __device__ __forceinline__ T load(const void *base, int64_t v)
+    {
+        return __ldcs(static_cast<const uint4 *>(base) + v);
+    }
+    static __device__ __forceinline__ void unpack(const T &s, float (&f)[8]) { unpack8(s, f); }
+    static __device__ __forceinline__ T zero() { return make_uint4(0, 0, 0, 0); }
+    static __device__ __forceinline__ void store(void *base, int64_t v, const float (&f)[8])
+    {
+        __stcs(static_cast<uint4 *>(base) + v, make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                          pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
+    }
+};
+
 // Per-group scale: absmax (k >= 2, or k = 1 with sign_scale 1) as an integer
 // max of the magnitude bits, or for k = 1 the mean of |a| by a perfect
 // binary-tree sum (three levels in the lane, then butterfly levels across the
@@ -141,11 +204,12 @@ __device__ __forceinline__ float group_scale(const float (&a)[8], bool &nonfinit
     }
 }
 
-template <QuantOp OP, int K, int G, int SS>
-__global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
+template <QuantOp OP, int K, int G, int SS, bool LEAN>
+__global__ void __launch_bounds__(QShape<OP, LEAN>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
 {
-    constexpr int kThreads = QShape<OP>::kThreads;
-    constexpr int kUnroll = QShape<OP>::kUnroll;
+    using SV = StateVec<LEAN>;
+    constexpr int kThreads = QShape<OP, LEAN>::kThreads;
+    constexpr int kUnroll = QShape<OP, LEAN>::kUnroll;
     constexpr int kTileVec = kThreads * kUnroll;
     constexpr int LPG = G / 8;
     constexpr int L = (K >= 2) ? (1 << (K - 1)) - 1 : 1;
@@ -167,26 +231,23 @@ __global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_con
         if constexpr (OP == QuantOp::WarmupSender) {
             const uint4 *X = static_cast<const uint4 *>(S.x);
             uint4 *B = static_cast<uint4 *>(S.base);
-            float4 *E = reinterpret_cast<float4 *>(S.err);
             uint4 xv[kUnroll];
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int64_t v = v0 + (int64_t)u * kThreads;
                 if (v < nvec) xv[u] = __ldcs(X + v);
             }
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int64_t v = v0 + (int64_t)u * kThreads;
                 if (v < nvec) {
                     __stcs(B + v, xv[u]);
-                    __stcs(E + 2 * v, z);
-                    __stcs(E + 2 * v + 1, z);
+                    SV::store(S.err, v, z);
                 }
             }
         } else if constexpr (OP == QuantOp::WarmupReceiver) {
             const uint4 *X = static_cast<const uint4 *>(S.x);
-            float4 *C = reinterpret_cast<float4 *>(S.cache);
             uint4 xv[kUnroll];
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
@@ -199,8 +260,7 @@ __global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_con
                 if (v < nvec) {
                     float f[8];
                     unpack8(xv[u], f);
-                    __stcs(C + 2 * v, make_float4(f[0], f[1], f[2], f[3]));
-                    __stcs(C + 2 * v + 1, make_float4(f[4], f[5], f[6], f[7]));
+                    SV::store(S.cache, v, f);   // bf16 -> fp32 is exact; fp32 -> bf16 of a bf16 value too
                 }
             }
         } else if constexpr (OP == QuantOp::Compress || OP == QuantOp::Loopback) {
@@ -210,30 +270,24 @@ __global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_con
             constexpr bool LB = OP == QuantOp::Loopback;
             const uint4 *X = static_cast<const uint4 *>(S.x);
             uint4 *B = static_cast<uint4 *>(S.base);
-            float4 *E = reinterpret_cast<float4 *>(S.err);
-            float4 *C = reinterpret_cast<float4 *>(S.cache);
             Word *codes = reinterpret_cast<Word *>(S.codes);
             float *scales = S.scales;
 
             uint4 xv[kUnroll], bv[kUnroll];
-            float4 ea[kUnroll], eb[kUnroll];
-            float4 ca[LB ? kUnroll : 1], cb[LB ? kUnroll : 1];
+            typename SV::T ev[kUnroll];
+            typename SV::T cv[LB ? kUnroll : 1];
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int64_t v = v0 + (int64_t)u * kThreads;
                 if (v < nvec) {
                     xv[u] = __ldcs(X + v);
                     bv[u] = __ldcs(B + v);
-                    ea[u] = __ldcs(E + 2 * v);
-                    eb[u] = __ldcs(E + 2 * v + 1);
-                    if constexpr (LB) {
-                        ca[u] = __ldcs(C + 2 * v);
-                        cb[u] = __ldcs(C + 2 * v + 1);
-                    }
+                    ev[u] = SV::load(S.err, v);
+                    if constexpr (LB) cv[u] = SV::load(S.cache, v);
                 } else {
                     xv[u] = bv[u] = make_uint4(0, 0, 0, 0);
-                    ea[u] = eb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if constexpr (LB) ca[u] = cb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    ev[u] = SV::zero();
+                    if constexpr (LB) cv[u] = SV::zero();
                 }
             }
 #pragma unroll
@@ -241,10 +295,10 @@ __global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_con
                 const int64_t v = v0 + (int64_t)u * kThreads;
                 const bool valid = v < nvec;
                 // residual against the base tensor plus the carried error
-                float xf[8], bf[8], a[8];
+                float xf[8], bf[8], a[8], e[8];
                 unpack8(xv[u], xf);
                 unpack8(bv[u], bf);
-                const float e[8] = {ea[u].x, ea[u].y, ea[u].z, ea[u].w, eb[u].x, eb[u].y, eb[u].z, eb[u].w};
+                SV::unpack(ev[u], e);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(__fsub_rn(xf[j], bf[j]), e[j]);
 
@@ -278,23 +332,22 @@ __global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_con
                 for (int j = 0; j < 8; ++j) a[j] = __fsub_rn(a[j], d[j]);  // new carried error
                 if (valid) {
                     __stcs(B + v, xv[u]);
-                    __stcs(E + 2 * v, make_float4(a[0], a[1], a[2], a[3]));
-                    __stcs(E + 2 * v + 1, make_float4(a[4], a[5], a[6], a[7]));
+                    SV::store(S.err, v, a);
                     codes[v] = (Word)word;
                     if ((lane & (LPG - 1)) == 0) scales[v / LPG] = s;
                     if constexpr (LB) {
-                        const float4 c0 = ca[u], c1 = cb[u];
-                        __stcs(C + 2 * v, make_float4(__fadd_rn(c0.x, d[0]), __fadd_rn(c0.y, d[1]),
-                                                      __fadd_rn(c0.z, d[2]), __fadd_rn(c0.w, d[3])));
-                        __stcs(C + 2 * v + 1, make_float4(__fadd_rn(c1.x, d[4]), __fadd_rn(c1.y, d[5]),
-                                                          __fadd_rn(c1.z, d[6]), __fadd_rn(c1.w, d[7])));
+                        float c[8];
+                        SV::unpack(cv[u], c);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) c[j] = __fadd_rn(c[j], d[j]);
+                        SV::store(S.cache, v, c);
                     }
                 }
             }
-        } else {  // Decompress
+        } else if constexpr (!LEAN) {  // Decompress, fp32 cache
             const Word *codes = reinterpret_cast<const Word *>(S.codes);
             const float *scales = S.scales;
-            float4 *C = reinterpret_cast<float4 *>(S.cache);
+            float4 *C = static_cast<float4 *>(S.cache);
             Word cw[kUnroll];
             float sv[kUnroll];
             float4 ca[kUnroll], cb[kUnroll];
@@ -330,232 +383,41 @@ __global__ void __launch_bounds__(QShape<OP>::kThreads) k_quant(const __grid_con
                                                       __fadd_rn(b.z, d[6]), __fadd_rn(b.w, d[7])));
                 }
             }
-        }
-    }
-}
-
-// ------------------------------------------------ TMA-staged variant ----
-// The same arithmetic as k_quant, but the input streams are staged through
-// shared memory by one producer thread with bulk-async copies (TMA,
-// cp.async.bulk, no tensor map), so that a CTA always has kTmaStages - 1
-// tiles in flight without spending registers on them.  Compress stages x,
-// base and err (64 B per vector); decompress stages the cache (32 B per
-// vector) and loads the small codes/scales directly before it waits.
-constexpr int kTmaConsumers = 256;               // 8 consumer warps
-constexpr int kTmaThreads = kTmaConsumers + 32;  // + 1 producer warp
-constexpr int kTmaVec = 512;                     // vectors per tile (= one stage)
-constexpr int kTmaStages = 3;
-constexpr unsigned long long kQuantWaitNs = 2000000000ull;
-
-template <QuantOp OP>
-__host__ __device__ constexpr int tma_bytes_per_vec()
-{
-    return OP == QuantOp::Compress ? 64 : 32;
-}
-
-struct TmaBarriers {
-    uint64_t full[kTmaStages];
-    uint64_t empty[kTmaStages];
-    int abort_flag;
-};
-
-template <QuantOp OP>
-constexpr size_t tma_smem_bytes()
-{
-    return (size_t)kTmaStages * kTmaVec * tma_bytes_per_vec<OP>() + sizeof(TmaBarriers);
-}
-
-template <QuantOp OP, int K, int G, int SS>
-__global__ void __launch_bounds__(kTmaThreads) k_quant_tma(const __grid_constant__ QuantLaunch p)
-{
-    using namespace ptx;
-    constexpr int LPG = G / 8;
-    constexpr int L = (K >= 2) ? (1 << (K - 1)) - 1 : 1;
-    constexpr int BPV = tma_bytes_per_vec<OP>();
-    constexpr int kStageBytes = kTmaVec * BPV;
-    using Word = typename CodeWord<K>::T;
-
-    extern __shared__ __align__(128) uint8_t tma_smem[];
-    TmaBarriers *bar = reinterpret_cast<TmaBarriers *>(tma_smem + kTmaStages * kStageBytes);
-    __shared__ float lut[16];
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    if (tid < 16) lut[tid] = (K >= 2) ? __fdiv_rn((float)(tid - L), (float)L) : 0.0f;
-    if (tid == 0) {
-        for (int s = 0; s < kTmaStages; ++s) {
-            mbar_init(&bar->full[s], 1);
-            mbar_init(&bar->empty[s], kTmaConsumers / 32);
-        }
-        bar->abort_flag = 0;
-        mbar_init_fence();
-    }
-    __syncthreads();
-    volatile int *abort_flag = &bar->abort_flag;
-
-    if (warp == kTmaConsumers / 32) {
-        // ---------------------------------------------------- producer --
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            uint32_t it = 0;
-            for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
-                const int s = it % kTmaStages;
-                const uint32_t ph = (it / kTmaStages) & 1u;
-                if (!wait_bounded(&bar->empty[s], ph ^ 1u, abort_flag, p.status, kQuantWaitNs)) break;
-                const QuantSlotDesc &S = p.slot[find_slot(p, tile)];
-                const int64_t v0 = (tile - S.tile0) * kTmaVec;
-                const int64_t left = S.nvec - v0;
-                const uint32_t nv = (uint32_t)(left < kTmaVec ? left : kTmaVec);
-                uint8_t *st = tma_smem + s * kStageBytes;
-                mbar_expect_tx(&bar->full[s], nv * BPV);
-                if constexpr (OP == QuantOp::Compress) {
-                    bulk_g2s(st, static_cast<const uint4 *>(S.x) + v0, nv * 16, &bar->full[s], pol);
-                    bulk_g2s(st + kTmaVec * 16, static_cast<const uint4 *>(S.base) + v0, nv * 16, &bar->full[s], pol);
-                    bulk_g2s(st + kTmaVec * 32, S.err + v0 * 8, nv * 32, &bar->full[s], pol);
-                } else {
-                    bulk_g2s(st, S.cache + v0 * 8, nv * 32, &bar->full[s], pol);
-                }
-            }
-            // every copy this thread issued has landed before the CTA exits
-            const uint32_t out = it < (uint32_t)kTmaStages ? it : (uint32_t)kTmaStages;
-            for (uint32_t j = it - out; j < it; ++j) {
-                volatile int no_abort = 0;
-                wait_bounded(&bar->full[j % kTmaStages], (j / kTmaStages) & 1u, &no_abort, p.status, kQuantWaitNs);
-            }
-        }
-        return;
-    }
-
-    // ------------------------------------------------------- consumers --
-    uint32_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
-        const int s = it % kTmaStages;
-        const uint32_t ph = (it / kTmaStages) & 1u;
-        const QuantSlotDesc &S = p.slot[find_slot(p, tile)];
-        const int64_t v0 = (tile - S.tile0) * kTmaVec;
-        const int64_t left = S.nvec - v0;
-        const int nv = (int)(left < kTmaVec ? left : kTmaVec);
-        const uint8_t *st = tma_smem + s * kStageBytes;
-
-        if constexpr (OP == QuantOp::Compress) {
-            bool ok = wait_bounded(&bar->full[s], ph, abort_flag, p.status, kQuantWaitNs);
-            if (!__all_sync(kFull, ok)) break;
-            uint4 xv[2], bv[2];
-            float4 ea[2], eb[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int vl = tid + u * kTmaConsumers;
-                if (vl < nv) {
-                    xv[u] = reinterpret_cast<const uint4 *>(st)[vl];
-                    bv[u] = reinterpret_cast<const uint4 *>(st + kTmaVec * 16)[vl];
-                    const float4 *e = reinterpret_cast<const float4 *>(st + kTmaVec * 32);
-                    ea[u] = e[2 * vl];
-                    eb[u] = e[2 * vl + 1];
-                } else {
-                    xv[u] = bv[u] = make_uint4(0, 0, 0, 0);
-                    ea[u] = eb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->empty[s]);
-
-            uint4 *B = static_cast<uint4 *>(S.base);
-            float4 *E = reinterpret_cast<float4 *>(S.err);
-            Word *codes = reinterpret_cast<Word *>(S.codes);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int vl = tid + u * kTmaConsumers;
-                const bool valid = vl < nv;
-                const int64_t v = v0 + vl;
-                float xf[8], bf[8], a[8];
-                unpack8(xv[u], xf);
-                unpack8(bv[u], bf);
-                const float e[8] = {ea[u].x, ea[u].y, ea[u].z, ea[u].w, eb[u].x, eb[u].y, eb[u].z, eb[u].w};
-#pragma unroll
-                for (int j = 0; j < 8; ++j) a[j] = __fadd_rn(__fsub_rn(xf[j], bf[j]), e[j]);
-                bool nonfinite;
-                float sc = group_scale<K, G, SS>(a, nonfinite);
-                const bool zero = nonfinite || !(sc >= kScaleMin);
-                if (zero) sc = 0.0f;
-                if (nonfinite && valid) atomicOr(p.status, kStatusNonfinite);
-                uint32_t word = 0;
-                if constexpr (K >= 2) {
-                    const float inv = __fdiv_rn((float)L, zero ? 1.0f : sc);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        int q = __float2int_rn(__fmul_rn(a[j], inv));
-                        q = min(max(q, -L), L);
-                        const int c = zero ? L : q + L;
-                        word |= (uint32_t)c << (K * j);
-                        a[j] = __fsub_rn(a[j], __fmul_rn(lut[c], sc));
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const bool pos = zero || (a[j] >= 0.0f);
-                        word |= (uint32_t)pos << j;
-                        a[j] = __fsub_rn(a[j], pos ? sc : -sc);
-                    }
-                }
-                if (valid) {
-                    __stcs(B + v, xv[u]);
-                    __stcs(E + 2 * v, make_float4(a[0], a[1], a[2], a[3]));
-                    __stcs(E + 2 * v + 1, make_float4(a[4], a[5], a[6], a[7]));
-                    codes[v] = (Word)word;
-                    if ((lane & (LPG - 1)) == 0) S.scales[v / LPG] = sc;
-                }
-            }
-        } else {
-            // codes and scales do not go through the stage: load them first
+        } else {  // Decompress, bf16 cache (lean state)
             const Word *codes = reinterpret_cast<const Word *>(S.codes);
-            Word cw[2];
-            float sv[2];
+            const float *scales = S.scales;
+            Word cw[kUnroll];
+            float sv[kUnroll];
+            typename SV::T cv[kUnroll];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int vl = tid + u * kTmaConsumers;
-                if (vl < nv) {
-                    cw[u] = __ldcs(codes + v0 + vl);
-                    sv[u] = __ldcs(S.scales + (v0 + vl) / LPG);
-                } else {
-                    cw[u] = 0;
-                    sv[u] = 0.0f;
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t v = v0 + (int64_t)u * kThreads;
+                if (v < nvec) {
+                    cw[u] = __ldcs(codes + v);
+                    sv[u] = __ldcs(scales + v / LPG);
+                    cv[u] = SV::load(S.cache, v);
                 }
             }
-            bool ok = wait_bounded(&bar->full[s], ph, abort_flag, p.status, kQuantWaitNs);
-            if (!__all_sync(kFull, ok)) break;
-            float4 ca[2], cb[2];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int vl = tid + u * kTmaConsumers;
-                if (vl < nv) {
-                    const float4 *c = reinterpret_cast<const float4 *>(st);
-                    ca[u] = c[2 * vl];
-                    cb[u] = c[2 * vl + 1];
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->empty[s]);
-            float4 *C = reinterpret_cast<float4 *>(S.cache);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int vl = tid + u * kTmaConsumers;
-                if (vl < nv) {
-                    const int64_t v = v0 + vl;
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t v = v0 + (int64_t)u * kThreads;
+                if (v < nvec) {
                     const uint32_t w = cw[u];
-                    const float sc = sv[u];
+                    const float s = sv[u];
                     float d[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const uint32_t c = (w >> (K * j)) & ((1u << K) - 1u);
                         if constexpr (K >= 2)
-                            d[j] = __fmul_rn(lut[c], sc);
+                            d[j] = __fmul_rn(lut[c], s);
                         else
-                            d[j] = c ? sc : -sc;
+                            d[j] = c ? s : -s;
                     }
-                    const float4 a = ca[u], b = cb[u];
-                    __stcs(C + 2 * v, make_float4(__fadd_rn(a.x, d[0]), __fadd_rn(a.y, d[1]), __fadd_rn(a.z, d[2]),
-                                                  __fadd_rn(a.w, d[3])));
-                    __stcs(C + 2 * v + 1, make_float4(__fadd_rn(b.x, d[4]), __fadd_rn(b.y, d[5]),
-                                                      __fadd_rn(b.z, d[6]), __fadd_rn(b.w, d[7])));
+                    float c[8];
+                    SV::unpack(cv[u], c);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) c[j] = __fadd_rn(c[j], d[j]);
+                    SV::store(S.cache, v, c);
                 }
             }
         }
@@ -564,70 +426,87 @@ __global__ void __launch_bounds__(kTmaThreads) k_quant_tma(const __grid_constant
 
 using KernelFn = void (*)(QuantLaunch);
 
-template <QuantOp OP, int K, int SS, bool TMA>
+template <QuantOp OP, int K, int SS, bool LEAN>
 KernelFn pick_group(int group)
 {
-    if constexpr (TMA) {
-        static_assert(OP == QuantOp::Compress || OP == QuantOp::Decompress, "TMA staging covers compress/decompress");
-        switch (group) {
-        case 8: return k_quant_tma<OP, K, 8, SS>;
-        case 16: return k_quant_tma<OP, K, 16, SS>;
-        case 32: return k_quant_tma<OP, K, 32, SS>;
-        case 64: return k_quant_tma<OP, K, 64, SS>;
-        case 128: return k_quant_tma<OP, K, 128, SS>;
-        case 256: return k_quant_tma<OP, K, 256, SS>;
-        default: return nullptr;
-        }
-    } else {
-        switch (group) {
-        case 8: return k_quant<OP, K, 8, SS>;
-        case 16: return k_quant<OP, K, 16, SS>;
-        case 32: return k_quant<OP, K, 32, SS>;
-        case 64: return k_quant<OP, K, 64, SS>;
-        case 128: return k_quant<OP, K, 128, SS>;
-        case 256: return k_quant<OP, K, 256, SS>;
-        default: return nullptr;
-        }
+    switch (group) {
+    case 8: return k_quant<OP, K, 8, SS, LEAN>;
+    case 16: return k_quant<OP, K, 16, SS, LEAN>;
+    case 32: return k_quant<OP, K, 32, SS, LEAN>;
+    case 64: return k_quant<OP, K, 64, SS, LEAN>;
+    case 128: return k_quant<OP, K, 128, SS, LEAN>;
+    case 256: return k_quant<OP, K, 256, SS, LEAN>;
+    default: return nullptr;
     }
 }
 
-template <bool TMA>
+template <QuantOp OP, bool LEAN>
+KernelFn pick_bits(int bits, int group, int ss)
+{
+    if (bits == 1) {
+        if constexpr (OP == QuantOp::Compress || OP == QuantOp::Loopback)
+            if (ss) return pick_group<OP, 1, 1, LEAN>(group);
+        return pick_group<OP, 1, 0, LEAN>(group);
+    }
+    if (bits == 2) return pick_group<OP, 2, 0, LEAN>(group);
+    if (bits == 4) return pick_group<OP, 4, 0, LEAN>(group);
+    return nullptr;
+}
+
+template <bool LEAN>
 KernelFn pick(QuantOp op, int bits, int group, int ss)
 {
     switch (op) {
-    case QuantOp::WarmupSender: return k_quant<QuantOp::WarmupSender, 2, 8, 0>;
-    case QuantOp::WarmupReceiver: return k_quant<QuantOp::WarmupReceiver, 2, 8, 0>;
-    case QuantOp::Compress:
-        if (bits == 1)
-            return ss ? pick_group<QuantOp::Compress, 1, 1, TMA>(group) : pick_group<QuantOp::Compress, 1, 0, TMA>(group);
-        if (bits == 2) return pick_group<QuantOp::Compress, 2, 0, TMA>(group);
-        if (bits == 4) return pick_group<QuantOp::Compress, 4, 0, TMA>(group);
-        return nullptr;
-    case QuantOp::Loopback:
-        if (bits == 1)
-            return ss ? pick_group<QuantOp::Loopback, 1, 1, false>(group) : pick_group<QuantOp::Loopback, 1, 0, false>(group);
-        if (bits == 2) return pick_group<QuantOp::Loopback, 2, 0, false>(group);
-        if (bits == 4) return pick_group<QuantOp::Loopback, 4, 0, false>(group);
-        return nullptr;
-    case QuantOp::Decompress:
-        if (bits == 1) return pick_group<QuantOp::Decompress, 1, 0, TMA>(group);
-        if (bits == 2) return pick_group<QuantOp::Decompress, 2, 0, TMA>(group);
-        if (bits == 4) return pick_group<QuantOp::Decompress, 4, 0, TMA>(group);
-        return nullptr;
+    case QuantOp::WarmupSender: return k_quant<QuantOp::WarmupSender, 2, 8, 0, LEAN>;
+    case QuantOp::WarmupReceiver: return k_quant<QuantOp::WarmupReceiver, 2, 8, 0, LEAN>;
+    case QuantOp::Compress: return pick_bits<QuantOp::Compress, LEAN>(bits, group, ss);
+    case QuantOp::Decompress: return pick_bits<QuantOp::Decompress, LEAN>(bits, group, ss);
+    case QuantOp::Loopback: return pick_bits<QuantOp::Loopback, LEAN>(bits, group, ss);
     }
     return nullptr;
 }
 
 // Launch shape of one kernel instance: threads, dynamic shared memory and
-// resident CTAs per SM (cached; the attribute call raises the dynamic shared
-// memory limit of the TMA-staged instances once).
+// resident CTAs per SM (cached per instance).
 struct Shape {
     int threads;
     size_t smem;
     int per_sm;
 };
 
-Shape launch_shape(KernelFn fn, bool tma, QuantOp op)
+template <bool LEAN>
+void shape_of(QuantOp op, int &threads, int &cap, int64_t &tile_vec)
+{
+    switch (op) {
+    case QuantOp::WarmupSender:
+        threads = QShape<QuantOp::WarmupSender, LEAN>::kThreads;
+        cap = QShape<QuantOp::WarmupSender, LEAN>::kMaxPerSm;
+        tile_vec = qtile_vec<QuantOp::WarmupSender, LEAN>();
+        break;
+    case QuantOp::WarmupReceiver:
+        threads = QShape<QuantOp::WarmupReceiver, LEAN>::kThreads;
+        cap = QShape<QuantOp::WarmupReceiver, LEAN>::kMaxPerSm;
+        tile_vec = qtile_vec<QuantOp::WarmupReceiver, LEAN>();
+        break;
+    case QuantOp::Compress:
+        threads = QShape<QuantOp::Compress, LEAN>::kThreads;
+        cap = QShape<QuantOp::Compress, LEAN>::kMaxPerSm;
+        tile_vec = qtile_vec<QuantOp::Compress, LEAN>();
+        break;
+    case QuantOp::Decompress:
+        threads = QShape<QuantOp::Decompress, LEAN>::kThreads;
+        cap = QShape<QuantOp::Decompress, LEAN>::kMaxPerSm;
+        tile_vec = qtile_vec<QuantOp::Decompress, LEAN>();
+        break;
+    case QuantOp::Loopback:
+        threads = QShape<QuantOp::Loopback, LEAN>::kThreads;
+        cap = QShape<QuantOp::Loopback, LEAN>::kMaxPerSm;
+        tile_vec = qtile_vec<QuantOp::Loopback, LEAN>();
+        break;
+    }
+}
+
+Shape launch_shape(KernelFn fn, bool lean, QuantOp op)
 {
     static std::mutex mu;
     static std::unordered_map<const void *, Shape> cache;
@@ -636,50 +515,16 @@ Shape launch_shape(KernelFn fn, bool tma, QuantOp op)
     if (it != cache.end()) return it->second;
     Shape sh{0, 0, 1};
     int cap = 0;
-    switch (op) {
-    case QuantOp::WarmupSender:
-        sh.threads = QShape<QuantOp::WarmupSender>::kThreads;
-        cap = QShape<QuantOp::WarmupSender>::kMaxPerSm;
-        break;
-    case QuantOp::WarmupReceiver:
-        sh.threads = QShape<QuantOp::WarmupReceiver>::kThreads;
-        cap = QShape<QuantOp::WarmupReceiver>::kMaxPerSm;
-        break;
-    case QuantOp::Compress:
-        sh.threads = QShape<QuantOp::Compress>::kThreads;
-        cap = QShape<QuantOp::Compress>::kMaxPerSm;
-        break;
-    case QuantOp::Decompress:
-        sh.threads = QShape<QuantOp::Decompress>::kThreads;
-        cap = QShape<QuantOp::Decompress>::kMaxPerSm;
-        break;
-    case QuantOp::Loopback:
-        sh.threads = QShape<QuantOp::Loopback>::kThreads;
-        cap = QShape<QuantOp::Loopback>::kMaxPerSm;
-        break;
-    }
-    if (tma) {
-        sh.threads = kTmaThreads;
-        sh.smem = op == QuantOp::Compress ? tma_smem_bytes<QuantOp::Compress>() : tma_smem_bytes<QuantOp::Decompress>();
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh.smem);
-    }
+    int64_t tile_vec = 0;
+    if (lean)
+        shape_of<true>(op, sh.threads, cap, tile_vec);
+    else
+        shape_of<false>(op, sh.threads, cap, tile_vec);
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, sh.threads, sh.smem) != cudaSuccess || nb < 1) nb = 1;
-    sh.per_sm = (!tma && cap > 0 && nb > cap) ? cap : nb;
+    sh.per_sm = (cap > 0 && nb > cap) ? cap : nb;
     cache[(const void *)fn] = sh;
     return sh;
-}
-
-// Staging of the compress / decompress streams: "tma" (bulk-async copies
-// through shared memory) or "reg" (vector loads straight into registers).
-bool use_tma_staging()
-{
-    static int v = -1;
-    if (v < 0) {
-        const char *e = getenv("CF_QUANT_STAGING");
-        v = (e && strcmp(e, "tma") == 0) ? 1 : 0;
-    }
-    return v == 1;
 }
 
 }  // namespace
@@ -696,22 +541,18 @@ int num_sms()
     return sms;
 }
 
-cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, QuantLaunch &lp, cudaStream_t stream)
+cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool lean, QuantLaunch &lp,
+                         cudaStream_t stream)
 {
-    const bool tma = use_tma_staging() && (op == QuantOp::Compress || op == QuantOp::Decompress);
-    KernelFn fn = tma ? pick<true>(op, bits, group, sign_scale) : pick<false>(op, bits, group, sign_scale);
+    KernelFn fn = lean ? pick<true>(op, bits, group, sign_scale) : pick<false>(op, bits, group, sign_scale);
     if (!fn) return cudaErrorInvalidValue;
     // tile prefix of every slot, in this kernel's tile size
-    int64_t tile_vec = kTmaVec;
-    if (!tma) {
-        switch (op) {
-        case QuantOp::WarmupSender: tile_vec = qtile_vec<QuantOp::WarmupSender>(); break;
-        case QuantOp::WarmupReceiver: tile_vec = qtile_vec<QuantOp::WarmupReceiver>(); break;
-        case QuantOp::Compress: tile_vec = qtile_vec<QuantOp::Compress>(); break;
-        case QuantOp::Decompress: tile_vec = qtile_vec<QuantOp::Decompress>(); break;
-        case QuantOp::Loopback: tile_vec = qtile_vec<QuantOp::Loopback>(); break;
-        }
-    }
+    int threads = 0, cap = 0;
+    int64_t tile_vec = 0;
+    if (lean)
+        shape_of<true>(op, threads, cap, tile_vec);
+    else
+        shape_of<false>(op, threads, cap, tile_vec);
     int64_t tiles = 0;
     for (int k = 0; k < lp.nslots; ++k) {
         lp.slot[k].tile0 = tiles;
@@ -719,9 +560,9 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, QuantL
     }
     lp.ntiles = tiles;
     if (tiles <= 0) return cudaSuccess;
-    const Shape sh = launch_shape(fn, tma, op);
-    const int64_t cap = (int64_t)num_sms() * sh.per_sm;
-    const int grid = (int)(tiles < cap ? tiles : cap);
+    const Shape sh = launch_shape(fn, lean, op);
+    const int64_t cap_blocks = (int64_t)num_sms() * sh.per_sm;
+    const int grid = (int)(tiles < cap_blocks ? tiles : cap_blocks);
     fn<<<grid, sh.threads, sh.smem, stream>>>(lp);
     return cudaGetLastError();
 }

@@ -30,19 +30,21 @@ class QuantState:
     """Sender state (base, err), receiver state (cache) and payload of each slot.
 
     Each array family is one contiguous allocation with per-slot views, so the
-    payload of a step can leave the device in one copy.
+    payload of a step can leave the device in one copy.  ``lean=True`` holds
+    err and cache in bf16 (the context's state_bf16 option).
     """
 
-    def __init__(self, shapes: Sequence[Sequence[int]], bits: int, group: int, device="cuda"):
+    def __init__(self, shapes: Sequence[Sequence[int]], bits: int, group: int, device="cuda", lean: bool = False):
         self.shapes = [tuple(s) for s in shapes]
-        self.bits, self.group = bits, group
+        self.bits, self.group, self.lean = bits, group, lean
         n = [r * c for r, c in self.shapes]
         self.elems = n
         nb = _aligned_sizes(n, 2)
-        nf = _aligned_sizes(n, 4)
+        sdt = torch.bfloat16 if lean else torch.float32
+        nf = _aligned_sizes(n, 2 if lean else 4)
         self.base_all = torch.empty(sum(nb), dtype=torch.bfloat16, device=device)
-        self.err_all = torch.empty(sum(nf), dtype=torch.float32, device=device)
-        self.cache_all = torch.empty(sum(nf), dtype=torch.float32, device=device)
+        self.err_all = torch.empty(sum(nf), dtype=sdt, device=device)
+        self.cache_all = torch.empty(sum(nf), dtype=sdt, device=device)
         self.base = [v[:k] for v, k in zip(_split(self.base_all, nb), n)]
         self.err = [v[:k] for v, k in zip(_split(self.err_all, nf), n)]
         self.cache = [v[:k] for v, k in zip(_split(self.cache_all, nf), n)]

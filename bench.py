@@ -357,6 +357,42 @@ def run_cf(args, w):
     ach_d = bd * n_elem / (deco_ms * 1e-3) / 1e9
     ach_pair = (bc + bd) * n_elem / (ms_per_step * 1e-3) / 1e9
 
+    # ---- the lean state (E and C in bf16), same inputs -------------------
+    lean = None
+    if not args.no_lean:
+        lctx = cf.Context(shapes, bits=w.bits, group=w.group, state_bf16=1)
+        lst = cf.QuantState(shapes, w.bits, w.group, device=dev, lean=True)
+        l_arrays = [lctx._slots(lst.slots(x_at(i))) for i in range(1, min(nsteps, 1 + args.warmup + args.steps))]
+        l0_arr = lctx._slots(lst.slots(X[0]))
+        lh = lctx.handle
+
+        def lean_step(i, arr):
+            if L.cf_compress(lh, arr, i, sh) != 0 or L.cf_decompress(lh, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(lh).decode())
+
+        lean_step(0, l0_arr)
+        for i in range(1, args.warmup + 1):
+            lean_step(i, l_arrays[(i - 1) % len(l_arrays)])
+        barrier(world)
+        torch.cuda.synchronize()
+        q0e, q1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0e.record(stream)
+        for k in range(args.steps):
+            i = args.warmup + 1 + k
+            lean_step(i, l_arrays[(i - 1) % len(l_arrays)])
+        q1e.record(stream)
+        torch.cuda.synchronize()
+        if lctx.check() != 0:
+            raise RuntimeError("device status in the lean run")
+        lean_ms = max_over_ranks(q0e.elapsed_time(q1e), world) / args.steps
+        pay = w.bits / 8 + 4 / w.group
+        lean_bytes = (2 + 2 + 2 + 2 + 2 + pay + pay + 2 + 2) * n_elem
+        lean = {"ms_per_step": lean_ms, "value": world * x_bytes / (lean_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "alg_bytes_per_step": lean_bytes, "achieved": lean_bytes / (lean_ms * 1e-3) / 1e9,
+                "frac": lean_bytes / (lean_ms * 1e-3) / 1e9 / peak,
+                "note": "state_bf16=1: E and C kept in bf16 (14.56 B/elt for compress + decompress)"}
+        del lctx, lst, l_arrays
+
     # ---- end to end through the public API, host buffers -----------------
     # Pinned host activations in, payload (codes + scales) back to pinned host
     # memory, every step; HostStreamCodec overlaps the host-to-device copy of
@@ -435,7 +471,7 @@ def run_cf(args, w):
                                 "alg_bytes_per_launch": bd * n_elem, "ms_per_launch": deco_ms},
         "roofline_step": {"achieved": ach_pair, "frac": ach_pair / peak, "frac_of_8tbs": ach_pair / 8000.0,
                           "alg_bytes_per_step": (bc + bd) * n_elem},
-        "loopback": lb,
+        "loopback": lb, "lean_state": lean,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
@@ -552,6 +588,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-loopback", action="store_true")
+    ap.add_argument("--no-lean", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

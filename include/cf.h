@@ -96,6 +96,9 @@ typedef struct cf_config {
     int sign_scale;  /* k = 1: 0 = mean |A| scale (default), 1 = absmax scale */
     int rank;        /* low-rank: r, 1..32 */
     int iters;       /* low-rank: T >= 0 subspace iterations */
+    int state_bf16;  /* quant: 0 = E and C in fp32 (default); 1 = lean state, E and C in bf16
+                        (each new E and C rounded to nearest even when stored; 14.3 instead of
+                        22.6 bytes per element for compress + decompress at k = 2, G = 128) */
 } cf_config;
 
 typedef struct cf_shape {
@@ -109,8 +112,8 @@ typedef struct cf_shape {
 typedef struct cf_slot {
     const void *x;   /* bf16 [rows*cols]  activation X_t (read only) */
     void *base;      /* bf16 [rows*cols]  sender's base tensor X_{t-1} */
-    float *err;      /* fp32 [rows*cols]  sender's error-feedback buffer E */
-    float *cache;    /* fp32 [rows*cols]  receiver's reconstruction C */
+    void *err;       /* fp32 [rows*cols]  sender's error-feedback buffer E (bf16 with state_bf16) */
+    void *cache;     /* fp32 [rows*cols]  receiver's reconstruction C (bf16 with state_bf16) */
     uint8_t *codes;  /* quant payload codes, rows*cols*k/8 bytes */
     float *scales;   /* quant payload scales, rows*cols/G */
     const float *q0; /* low-rank: Gaussian start block [cols x r] for this call */

@@ -254,16 +254,44 @@ def test_host_stream_codec_matches_oracle(cf, oracle):
         assert np.array_equal(hc.st.err[i].cpu().numpy(), ors[i].err)
 
 
-def test_tma_staged_variant_bit_exact():
-    """The TMA-staged compress/decompress variant (CF_QUANT_STAGING=tma, read
-    once per process) passes the same bit-exact parity, in a fresh process."""
-    import os
-    import subprocess
-    import sys
+def run_lean(cf, oracle, shapes, steps, bits, group, ss=0, loopback=False, w=synth.FLUX):
+    ctx = cf.Context(shapes, bits=bits, group=group, sign_scale=ss, state_bf16=1)
+    st = cf.QuantState(shapes, bits, group, lean=True)
+    streams = [synth.SlotStream(w.scaled(rows=r, cols=c), slot=i) for i, (r, c) in enumerate(shapes)]
+    ors = [oracle.QuantSlot(bits, group, ss, lean=True) for _ in shapes]
+    for t in range(steps):
+        xs = [s.next() for s in streams]
+        slots = st.slots([x.cuda() for x in xs])
+        if loopback:
+            ctx.loopback(slots, t)
+        else:
+            ctx.compress(slots, t)
+            ctx.decompress(slots, t)
+        for i, x in enumerate(xs):
+            ors[i].step(t, u16(x))
+        torch.cuda.synchronize()
+        for i in range(len(shapes)):
+            o = ors[i]
+            assert np.array_equal(u16(st.err[i]), o.err), (t, i, "err")
+            assert np.array_equal(u16(st.cache[i]), o.cache), (t, i, "cache")
+            assert np.array_equal(u16(st.base[i]), o.base), (t, i, "base")
+            if t > 0:
+                assert np.array_equal(st.codes[i].cpu().numpy(), o.codes), (t, i, "codes")
+                assert np.array_equal(st.scales[i].cpu().numpy(), o.scales), (t, i, "scales")
+    assert ctx.check() == cf.CF_OK
 
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, CF_QUANT_STAGING="tma")
-    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
-                        os.path.join(root, "tests", "test_gpu_quant.py"), "-k", "tiny_workload or ragged or stress"],
-                       capture_output=True, text=True, env=env, cwd=root, timeout=900)
-    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+@pytest.mark.parametrize("bits,group,ss", [(2, 128, 0), (4, 64, 0), (1, 128, 0), (1, 128, 1), (2, 8, 0), (4, 256, 0)])
+@pytest.mark.parametrize("loopback", [False, True])
+def test_lean_state_bit_exact(cf, oracle, bits, group, ss, loopback):
+    """Lean state (E and C in bf16): codes, scales, E, C and base bit-exact to
+    the oracle's lean codec, for the pair and for the fused loopback."""
+    shapes = [(37, 512), (1, 256), (0, 256), (129, 768)]
+    shapes = [(r, c) for r, c in shapes if c % group == 0]
+    run_lean(cf, oracle, shapes, 4, bits, group, ss, loopback)
+
+
+def test_lean_state_rejected_in_lowrank_mode(cf):
+    with pytest.raises(cf.CfError) as e:
+        cf.Context([(64, 64)], mode=cf.CF_MODE_LOWRANK, rank=4, iters=1, state_bf16=1)
+    assert e.value.status == cf.CF_E_ARG
