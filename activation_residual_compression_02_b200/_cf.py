@@ -29,7 +29,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 class cf_config(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("bits", ctypes.c_int), ("group", ctypes.c_int),
                 ("sign_scale", ctypes.c_int), ("rank", ctypes.c_int), ("iters", ctypes.c_int),
-                ("state_bf16", ctypes.c_int)]
+                ("state_bf16", ctypes.c_int), ("warm_start", ctypes.c_int)]
 
 
 class cf_shape(ctypes.Structure):
@@ -133,9 +133,9 @@ class Context:
     """A libcf context (``cf_create`` ... ``cf_destroy``)."""
 
     def __init__(self, shapes: Sequence[Sequence[int]], mode: int = CF_MODE_QUANT, bits: int = 2, group: int = 128,
-                 sign_scale: int = 0, rank: int = 16, iters: int = 2, state_bf16: int = 0):
+                 sign_scale: int = 0, rank: int = 16, iters: int = 2, state_bf16: int = 0, warm_start: int = 0):
         L = lib()
-        self.cfg = cf_config(mode, bits, group, sign_scale, rank, iters, state_bf16)
+        self.cfg = cf_config(mode, bits, group, sign_scale, rank, iters, state_bf16, warm_start)
         self.shapes = [tuple(int(v) for v in s) for s in shapes]
         arr = (cf_shape * max(1, len(self.shapes)))(*[cf_shape(r, c) for r, c in self.shapes])
         h = ctypes.c_void_p()
@@ -235,7 +235,7 @@ def cf_lowrank_noalloc(A, Q0, U, R, V, E=None, C=None, rank: int = 16, iters: in
     allocate device memory: the scratch is a fixed 8 MiB device array inside
     libcf.  Synchronous; returns the C status (CF_OK, CF_E_NOMEM when the call
     does not fit the scratch, ...)."""
-    cfg = cf_config(CF_MODE_LOWRANK, 0, 0, 0, rank, iters, 0)
+    cfg = cf_config(CF_MODE_LOWRANK, 0, 0, 0, rank, iters, 0, 0)
     nmat = len(A)
     m, n = (A[0].shape[0], A[0].shape[1]) if nmat else (0, 0)
     return int(lib().cf_lowrank_noalloc(ctypes.byref(cfg), nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R),

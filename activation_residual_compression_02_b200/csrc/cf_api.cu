@@ -23,6 +23,7 @@ struct cf_ctx {
     size_t ws_bytes = 0;
     bool warm_sender = false;
     bool warm_receiver = false;
+    int64_t lowrank_steps = 0;   // compressed low-rank steps done (for warm_start)
     int device = 0;
     std::string err;
 };
@@ -58,10 +59,12 @@ cf_status validate_config(const cf_config *c, std::string &why)
         if (!pow2(c->group) || c->group < 8 || c->group > 256) { why = "group must be a power of two in [8, 256]"; return CF_E_ARG; }
         if (c->sign_scale != 0 && c->sign_scale != 1) { why = "sign_scale must be 0 or 1"; return CF_E_ARG; }
         if (c->state_bf16 != 0 && c->state_bf16 != 1) { why = "state_bf16 must be 0 or 1"; return CF_E_ARG; }
+        if (c->warm_start != 0) { why = "warm_start is a low-rank-mode option"; return CF_E_ARG; }
         return CF_OK;
     }
     if (c->mode == CF_MODE_LOWRANK) {
         if (c->state_bf16 != 0) { why = "the lean bf16 state is a quantised-mode option"; return CF_E_ARG; }
+        if (c->warm_start != 0 && c->warm_start != 1) { why = "warm_start must be 0 or 1"; return CF_E_ARG; }
         if (c->rank < 1 || c->rank > 32) { why = "rank must be in [1, 32]"; return CF_E_ARG; }
         if (c->iters < 0 || c->iters > 1000) { why = "iters must be in [0, 1000]"; return CF_E_ARG; }
         return CF_OK;
@@ -172,6 +175,9 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
         return fail(ctx, CF_E_NOMEM, "low-rank mode needs %zu bytes of workspace (cf_set_workspace)", need);
     const int n = (int)ctx->shapes.size();
     const int r = ctx->cfg.rank;
+    // warm start: from the second compressed step on, Algorithm 3 starts from
+    // the V each slot received in the previous step
+    const bool warm = sender && ctx->cfg.warm_start && ctx->lowrank_steps > 0;
     for (int i = 0; i < n; ++i) {
         const cf_slot &s = slots[i];
         if (ctx->shapes[i].rows == 0) continue;  // an empty slot is never touched
@@ -179,7 +185,8 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
         if (!aligned16(s.U) || !aligned16(s.R) || !aligned16(s.V))
             return fail(ctx, CF_E_ALIGN, "slot %d: U/R/V must be 16-byte aligned", i);
         if (sender) {
-            if (!s.x || !s.base || !s.err || !s.q0) return fail(ctx, CF_E_ARG, "slot %d: x/base/err/q0 must be non-NULL", i);
+            if (!s.x || !s.base || !s.err || (!s.q0 && !warm))
+                return fail(ctx, CF_E_ARG, "slot %d: x/base/err/q0 must be non-NULL", i);
             if (!aligned16(s.x) || !aligned16(s.base) || !aligned16(s.err) || !aligned16(s.q0))
                 return fail(ctx, CF_E_ALIGN, "slot %d: x/base/err/q0 must be 16-byte aligned", i);
             if (ctx->shapes[i].rows > 0 && (ctx->shapes[i].rows < r || ctx->shapes[i].cols < r))
@@ -222,7 +229,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
         for (size_t k = i; k < j; ++k) {
             cf::LowrankMat &m = mats[k - i];
             m.A = a_ptr[k];
-            m.Q0 = slots[k].q0;
+            m.Q0 = warm ? slots[k].V : slots[k].q0;
             m.U = slots[k].U;
             m.R = slots[k].R;
             m.V = slots[k].V;
@@ -242,6 +249,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
                                : cf::run_lowrank_decompress(plan, mats.data(), stream);
         if (e != cudaSuccess) st = cuda_fail(ctx, e, sender ? "low-rank compress" : "low-rank decompress");
     });
+    if (st == CF_OK && sender) ++ctx->lowrank_steps;
     return st;
 }
 

@@ -495,6 +495,8 @@ def run_lowrank_bench(args, w):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     m, n, r, T, k = w.rows, w.cols, w.rank, w.iters, w.slots
+    if args.warm_start:
+        T = 1      # each call starts from the previous call's V
     ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
     ws = torch.empty(ctx.lowrank_workspace_bytes(k, m, n), dtype=torch.uint8, device=dev)
     ctx.set_workspace(ws)
@@ -505,8 +507,10 @@ def run_lowrank_bench(args, w):
     V = [torch.empty(n, r, device=dev) for _ in range(k)]
     E = [torch.empty(m, n, device=dev) for _ in range(k)]
     stream = torch.cuda.current_stream()
+    ctx.lowrank(A, Q0, U, R, V, E)
+    start_block = V if args.warm_start else Q0   # warm start: V doubles as the next start block
     for _ in range(args.warmup):
-        ctx.lowrank(A, Q0, U, R, V, E)
+        ctx.lowrank(A, start_block, U, R, V, E)
     torch.cuda.synchronize()
     assert ctx.check() == 0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -514,7 +518,7 @@ def run_lowrank_bench(args, w):
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for _ in range(args.steps):
-            ctx.lowrank(A, Q0, U, R, V, E)
+            ctx.lowrank(A, start_block, U, R, V, E)
         end.record(stream)
         torch.cuda.synchronize()
     status = ctx.check()
@@ -556,7 +560,8 @@ def run_lowrank_bench(args, w):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "tf32/f64", "data": "synthetic",
         "config": {"workload": f"lowrank: {k} matrices x {m} x {n} fp32, rank-{r} signal + 0.01 noise, r={r}, "
-                               f"T={T}, Gaussian Q0, E = A - U R V^T written",
+                               f"T={T}, " + ("warm start from the previous V" if args.warm_start else "Gaussian Q0")
+                               + ", E = A - U R V^T written",
                    "l2": "inputs larger than L2 (3.2 GB of A per step)"},
         "roofline": {"bound": "hbm", "kernel": "whole cf_lowrank call", "achieved": alg_bytes / (ms * 1e-3) / 1e9,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
@@ -589,6 +594,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-loopback", action="store_true")
     ap.add_argument("--no-lean", action="store_true")
+    ap.add_argument("--warm-start", action="store_true", help="low-rank: T = 1 from the previous call's V")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -99,6 +99,10 @@ typedef struct cf_config {
     int state_bf16;  /* quant: 0 = E and C in fp32 (default); 1 = lean state, E and C in bf16
                         (each new E and C rounded to nearest even when stored; 14.3 instead of
                         22.6 bytes per element for compress + decompress at k = 2, G = 128) */
+    int warm_start;  /* low-rank cf_compress: 0 = start Algorithm 3 from the slot's q0 every step
+                        (default); 1 = from the second compressed step on, start from the slot's V
+                        of the previous step (q0 may then be NULL), so that a small `iters`
+                        (e.g. 1) tracks a slowly moving subspace with fewer passes over A */
 } cf_config;
 
 typedef struct cf_shape {
@@ -144,7 +148,8 @@ cf_status cf_set_workspace(cf_ctx *ctx, void *dev_ptr, size_t bytes);
  *   step >= 1, quantised: A = (x - base) + err; codes, scales = Q(A);
  *           err = A - deq; base = x.  Uses x, base, err, codes, scales.
  *   step >= 1, low-rank: A as above into the workspace; Algorithm 3 with
- *           start block q0 gives U, R, V; err = A - U R V^T; base = x.
+ *           start block q0 (or, with warm_start, the V of the previous
+ *           compressed step) gives U, R, V; err = A - U R V^T; base = x.
  *           Uses x, base, err, q0, U, R, V.
  * `slots` is a host array of nslots entries; `cuda_stream` a cudaStream_t
  * (NULL = legacy default stream).  Errors before launch: CF_E_ARG,

@@ -197,3 +197,50 @@ def test_lowrank_mode_through_slots(cf, oracle):
     for i in range(2):
         x = xs[i][2].float().reshape(-1).cuda()
         assert (torch.linalg.vector_norm(cache[i] + err[i] - x) / torch.linalg.vector_norm(x)).item() < 1e-5
+
+
+def test_lowrank_warm_start_through_slots(cf, oracle):
+    """warm_start: from the second compressed step on, Algorithm 3 starts from
+    the previous step's V (T = 1 here).  Each step matches the oracle run from
+    the same start block, and the error feedback keeps C + E = X."""
+    rows, cols, r, T = 192, 256, 16, 1
+    shapes = [(rows, cols)]
+    ctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T, warm_start=1)
+    ws = torch.empty(max(ctx.workspace_bytes(), 16), dtype=torch.uint8, device="cuda")
+    ctx.set_workspace(ws)
+    x = synth.gaussian((rows, cols), 0, 7, 99)
+    # a slowly rotating rank-r increment: the subspace moves a little per step
+    Ub = synth.gaussian((rows, r), 0, 7, 98)
+    Vb = synth.gaussian((cols, r), 0, 7, 97)
+    seq = [x.to(torch.bfloat16)]
+    for t in range(1, 6):
+        Ut = Ub + 0.05 * t * synth.gaussian((rows, r), 0, 7, t)
+        Vt = Vb + 0.05 * t * synth.gaussian((cols, r), 0, 7, 100 + t)
+        L = (Ut * (1.0 / torch.arange(1, r + 1))) @ Vt.T
+        seq.append((seq[-1].float() + 0.5 * L / L.pow(2).mean().sqrt()).to(torch.bfloat16))
+    base = torch.empty(rows * cols, dtype=torch.bfloat16, device="cuda")
+    err = torch.empty(rows * cols, device="cuda")
+    cache = torch.empty(rows * cols, device="cuda")
+    U, R, V = torch.empty(rows, r, device="cuda"), torch.empty(r, r, device="cuda"), torch.empty(cols, r, device="cuda")
+    q0 = synth.q0(cols, r, seed=0, mat=7).cuda()
+    ob = oe = None
+    for t, xt in enumerate(seq):
+        start = q0 if t <= 1 else V.clone()
+        slot = cf.Slot(x=xt.reshape(-1).cuda(), base=base, err=err, cache=cache, q0=q0 if t <= 1 else None,
+                       U=U, R=R, V=V)
+        ctx.compress([slot], t)
+        ctx.decompress([slot], t)
+        xb = xt.view(torch.int16).numpy().view(np.uint16).ravel().copy()
+        if t == 0:
+            ob, oe = oracle.warmup_sender(xb)
+            continue
+        a = oracle.residual(xb, ob, oe).reshape(rows, cols)
+        Uo, Ro, Vo = oracle.subspace_iteration(a, start.cpu().numpy(), T)
+        Do, Eo, _ = oracle.lowrank_apply(a, Uo, Ro, Vo)
+        torch.cuda.synchronize()
+        eg = err.cpu().double().numpy().reshape(rows, cols)
+        assert rel(eg, Eo, Do) <= TOL, t
+        oe = err.cpu().numpy().copy()
+    assert ctx.check() == cf.CF_OK
+    xl = seq[-1].float().reshape(-1).cuda()
+    assert (torch.linalg.vector_norm(cache + err - xl) / torch.linalg.vector_norm(xl)).item() < 1e-5
