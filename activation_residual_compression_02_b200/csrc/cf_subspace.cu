@@ -12,8 +12,8 @@
 //    Z = A^T P (A read as an MN-major operand straight from its row-major
 //    storage, staged with the 128-byte/32-byte-atom swizzle that MN-major
 //    32-bit operands require).  A warp-specialised persistent tcgen05 kernel: one TMA warp
-//    streams 128x32 fp32 tiles of A (128-byte swizzle) plus the matching
-//    r-column slice of Q^T / P^T; four warps round each A tile to TF32 in
+//    streams stages of two or three 128x32 fp32 boxes of A (128-byte swizzle)
+//    plus the matching r-column slices of Q^T / P^T; four warps round each A tile to TF32 in
 //    shared memory (round to nearest: the tensor core would otherwise drop the
 //    low mantissa bits, a bias of about 2^-11 that alone costs ~7e-4 of the
 //    reconstruction); one thread issues tcgen05.mma (M=128, N=16/32, K=8)
@@ -43,12 +43,27 @@ namespace {
 
 // ------------------------------------------------------------ constants --
 constexpr int kBM = 128;            // MMA M: rows of an output tile
-constexpr int kBK = 32;             // K per pipeline stage (fp32: 128 bytes)
-constexpr int kStages = 8;
+constexpr int kBoxK = 32;           // K of one TMA box: 32 fp32 = 128 bytes, the swizzle span
+constexpr int kBoxBytes = kBM * kBoxK * 4;   // one 128 x 32 box of A: 16 KB
 constexpr int kGemmThreads = 320;   // 10 warps: TMA, MMA, 4 convert, 4 epilogue
-constexpr int kATileBytes = kBM * kBK * 4;   // 16 KB
-constexpr int kBTileBytes = 32 * kBK * 4;    // room for N = 32
 constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parameters
+
+// Pipeline shape per padded rank RP (the MMA's N).  A stage holds NB boxes of
+// A side by side in K, so each row of A is read NB x 128 contiguous bytes at
+// a time and the per-stage handshakes (barrier, TF32 rounding, fence, MMA
+// batch) are paid once per NB boxes.  Measured on the 57 x 4608 x 3072 pass:
+// one box per stage with 8 stages ran at 5.2-5.6 TB/s; three boxes with four
+// stages at 6.6 TB/s, bit-identical.  RP = 32 needs twice the B space and
+// keeps two boxes with five stages to stay within 227 KB of shared memory.
+template <int RP>
+struct GemmCfg {
+    static constexpr int NB = RP == 16 ? 3 : 2;         // boxes of A per stage
+    static constexpr int ST = RP == 16 ? 4 : 5;         // pipeline stages
+    static constexpr int BK = NB * kBoxK;               // K per stage
+    static constexpr int ATile = NB * kBoxBytes;        // A bytes per stage
+    static constexpr int BBox = RP * kBoxK * 4;         // one RP x 32 box of Q^T / P^T
+    static constexpr int BTile = NB * BBox;
+};
 constexpr int kTmemCols = 64;       // two accumulators of up to 32 columns
 constexpr uint64_t kWaitNs = 2000000000ull;
 
@@ -161,10 +176,11 @@ __device__ __forceinline__ uint32_t instr_desc_tf32(int rp, int a_mn_major)
            ((uint32_t)(kBM >> 4) << 24);
 }
 
+template <int ST>
 struct GemmSmem {
-    uint64_t full[kStages];
-    uint64_t conv[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[ST];
+    uint64_t conv[ST];
+    uint64_t empty[ST];
     uint64_t accf[2];
     uint64_t acce[2];
     uint64_t drain;
@@ -173,13 +189,16 @@ struct GemmSmem {
 };
 
 // ------------------------------------------------------------ the GEMM ----
+template <int RP>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_constant__ GemmParams p)
 {
+    using C = GemmCfg<RP>;
+    constexpr int kStages = C::ST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sA = base;                                   // kStages x 16 KB
-    uint8_t *sB = base + kStages * kATileBytes;           // kStages x 4 KB
-    GemmSmem *S = (GemmSmem *)(sB + kStages * kBTileBytes);
+    uint8_t *sA = base;                                   // kStages x NB boxes of A
+    uint8_t *sB = base + kStages * C::ATile;              // kStages x NB boxes of Q^T / P^T
+    GemmSmem<kStages> *S = (GemmSmem<kStages> *)(sB + kStages * C::BTile);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -211,8 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
     const uint32_t tmem = S->tmem_base;
     volatile int *abort_flag = &S->abort_flag;
     const unsigned long long wait_ns = p.wait_ns;
-    const int rp = p.rp;
-    const uint32_t stage_bytes = (uint32_t)kATileBytes + (uint32_t)rp * kBK * 4;
+    const uint32_t stage_bytes = (uint32_t)(C::ATile + C::BTile);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -231,15 +249,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
                         break;
                     }
                     mbar_expect_tx(&S->full[s], stage_bytes);
-                    uint8_t *a = sA + s * kATileBytes;
-                    if (!p.mn_major) {
-                        tma_load_2d(a, &M.ta, kt * kBK, mt * kBM, &S->full[s]);
-                    } else {
+                    // NB boxes side by side in K; boxes past the end of K
+                    // are zero-filled by the TMA unit and still count their
+                    // full bytes.
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            tma_load_2d(a + j * 4096, &M.ta, mt * kBM + 32 * j, kt * kBK, &S->full[s]);
+                    for (int h = 0; h < C::NB; ++h) {
+                        uint8_t *a = sA + s * C::ATile + h * kBoxBytes;
+                        const int k0 = kt * C::BK + h * kBoxK;
+                        if (!p.mn_major) {
+                            tma_load_2d(a, &M.ta, k0, mt * kBM, &S->full[s]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                tma_load_2d(a + j * 4096, &M.ta, mt * kBM + 32 * j, k0, &S->full[s]);
+                        }
+                        tma_load_3d(sB + s * C::BTile + h * C::BBox, &p.tb, k0, 0, mi, &S->full[s]);
                     }
-                    tma_load_3d(sB + s * kBTileBytes, &p.tb, kt * kBK, 0, mi, &S->full[s]);
                 }
             }
             // Drain: every load this thread issued has landed before exit.
@@ -251,7 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
         }
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
-        const uint32_t idesc = instr_desc_tf32(rp, p.mn_major);
+        const uint32_t idesc = instr_desc_tf32(RP, p.mn_major);
         uint32_t it = 0, lt = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++lt) {
@@ -269,13 +294,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t a0 = smem_u32(sA + s * kATileBytes);
-                    const uint32_t b0 = smem_u32(sB + s * kBTileBytes);
+                    const uint32_t a0 = smem_u32(sA + s * C::ATile);
+                    const uint32_t b0 = smem_u32(sB + s * C::BTile);
 #pragma unroll
-                    for (int k = 0; k < kBK / 8; ++k) {
-                        const uint64_t ad = p.mn_major ? smem_desc(a0 + k * 1024, 4096, 512, kLayoutSw128Atom32)
-                                                       : smem_desc(a0 + k * 32, 16, 1024, kLayoutSw128);
-                        const uint64_t bd = smem_desc(b0 + k * 32, 16, 1024, kLayoutSw128);
+                    for (int k = 0; k < C::BK / 8; ++k) {
+                        // K step k: box k / 4, 8-element slice k % 4 of it
+                        const uint32_t ah = a0 + (k / 4) * kBoxBytes, bh = b0 + (k / 4) * C::BBox;
+                        const uint32_t kk = (uint32_t)(k % 4);
+                        const uint64_t ad = p.mn_major ? smem_desc(ah + kk * 1024, 4096, 512, kLayoutSw128Atom32)
+                                                       : smem_desc(ah + kk * 32, 16, 1024, kLayoutSw128);
+                        const uint64_t bd = smem_desc(bh + kk * 32, 16, 1024, kLayoutSw128);
                         tc_mma_tf32(dtm, ad, bd, idesc, (kt > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(&S->empty[s]);
@@ -305,9 +333,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
                     ok = false;
                     break;
                 }
-                float4 *a = (float4 *)(sA + s * kATileBytes);
+                float4 *a = (float4 *)(sA + s * C::ATile);
 #pragma unroll
-                for (int i = 0; i < kATileBytes / 16 / 128; ++i) {
+                for (int i = 0; i < C::ATile / 16 / 128; ++i) {
                     float4 v = a[ct + 128 * i];
                     v.x = round_tf32(v.x);
                     v.y = round_tf32(v.y);
@@ -336,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
 #pragma unroll
                 for (int c = 0; c < 16; ++c) v[c] = lo[c];
             }
-            if (rp > 16) {
+            if (RP > 16) {
                 uint32_t hi[16];
                 tc_ld16(taddr + 16, hi);
 #pragma unroll
@@ -352,11 +380,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
             float *out = p.out + (int64_t)mi * p.out_stride;
             if (row < p.out_rows) {
                 if (p.out_mode == 0) {
-                    for (int c = 0; c < rp; ++c)
+#pragma unroll
+                    for (int c = 0; c < RP; ++c)
                         out[(int64_t)c * p.out_ld + row] = round_tf32(__uint_as_float(v[c]));
                 } else {
-                    float4 *o = (float4 *)(out + (int64_t)row * rp);
-                    for (int c = 0; c < rp; c += 4)
+                    float4 *o = (float4 *)(out + (int64_t)row * RP);
+#pragma unroll
+                    for (int c = 0; c < RP; c += 4)
                         o[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
                                                __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
                 }
@@ -372,7 +402,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
     }
 }
 
-constexpr size_t kGemmSmemBytes = 1024 + kStages * (kATileBytes + kBTileBytes) + sizeof(GemmSmem);
+template <int RP>
+constexpr size_t gemm_smem_bytes()
+{
+    using C = GemmCfg<RP>;
+    return 1024 + (size_t)C::ST * (C::ATile + C::BTile) + sizeof(GemmSmem<C::ST>);
+}
+static_assert(gemm_smem_bytes<16>() <= 227 * 1024, "GEMM shared memory (RP = 16) exceeds 227 KB");
+static_assert(gemm_smem_bytes<32>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
 
 // ------------------------------------------------------ CholeskyQR -------
 constexpr int kGramThreads = 256;
@@ -879,19 +916,28 @@ WsLayout layout(int nmat, int64_t m, int64_t n, int r)
     return L;
 }
 
-cudaError_t gemm_launch(GemmParams &gp, int total_tiles, cudaStream_t stream)
+template <int RP>
+cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
 {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(k_gemm_tf32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes);
+        attr_err = cudaFuncSetAttribute(k_gemm_tf32<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)gemm_smem_bytes<RP>());
     });
     if (attr_err != cudaSuccess) return attr_err;
-    const int grid = total_tiles < num_sms() ? total_tiles : num_sms();
-    if (grid <= 0) return cudaSuccess;
-    k_gemm_tf32<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(gp);
+    k_gemm_tf32<RP><<<grid, kGemmThreads, gemm_smem_bytes<RP>(), stream>>>(gp);
     return cudaGetLastError();
 }
+
+cudaError_t gemm_launch(GemmParams &gp, int total_tiles, cudaStream_t stream)
+{
+    const int grid = total_tiles < num_sms() ? total_tiles : num_sms();
+    if (grid <= 0) return cudaSuccess;
+    return gp.rp == 16 ? gemm_launch_rp<16>(gp, grid, stream) : gemm_launch_rp<32>(gp, grid, stream);
+}
+
+int gemm_bk(int rp) { return rp == 16 ? GemmCfg<16>::BK : GemmCfg<32>::BK; }
 
 // out_i = A_i Q_i (mn_major = 0) or A_i^T P_i (mn_major = 1) for every matrix.
 cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLayout &L, int mn_major, int out_mode,
@@ -922,11 +968,11 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
         bool ok;
         if (!mn_major) {
             gp->tiles_per_mat = (int)((m + kBM - 1) / kBM);
-            gp->ktiles = (int)((n + kBK - 1) / kBK);
+            gp->ktiles = (int)((n + gemm_bk(L.rp) - 1) / gemm_bk(L.rp));
             gp->out_rows = (int)m;
             gp->out_ld = (int)L.mp;
             ok = make_map3(&gp->tb, ws + L.qt + (size_t)first * L.rp * L.np * 4, n, L.rp, cnt, L.np, L.rp * L.np,
-                           kBK, L.rp);
+                           kBoxK, L.rp);
             if (out_mode == 0) {
                 gp->out = (float *)(ws + L.pt) + (size_t)first * L.rp * L.mp;
                 gp->out_stride = L.rp * L.mp;
@@ -936,18 +982,18 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             }
         } else {
             gp->tiles_per_mat = (int)((n + kBM - 1) / kBM);
-            gp->ktiles = (int)((m + kBK - 1) / kBK);
+            gp->ktiles = (int)((m + gemm_bk(L.rp) - 1) / gemm_bk(L.rp));
             gp->out_rows = (int)n;
             gp->out_ld = 0;
             ok = make_map3(&gp->tb, ws + L.pt + (size_t)first * L.rp * L.mp * 4, m, L.rp, cnt, L.mp, L.rp * L.mp,
-                           kBK, L.rp);
+                           kBoxK, L.rp);
             gp->out = (float *)(ws + L.z) + (size_t)first * n * L.rp;
             gp->out_stride = n * L.rp;
         }
         for (int k = 0; k < cnt && ok; ++k) {
             const LowrankMat &s = mats[first + k];
-            ok = !mn_major ? make_map(&gp->mat[k].ta, s.A, n, m, n, kBK, kBM)
-                           : make_map(&gp->mat[k].ta, s.A, n, m, n, 32, kBK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+            ok = !mn_major ? make_map(&gp->mat[k].ta, s.A, n, m, n, kBoxK, kBM)
+                           : make_map(&gp->mat[k].ta, s.A, n, m, n, 32, kBoxK, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
         }
         if (!ok) {
             err = cudaErrorInvalidValue;
