@@ -84,9 +84,13 @@ def check(oracle, As, Q0s, out, T, idx=None):
 # gives 1.6e-3 there for one of three seeds, against 1.7e-4 at T = 4.  The
 # cases below keep the iteration well posed; the 1e-3 bar is the one stated
 # for the low-rank workload (4608 x 3072, r = 16, T = 2: about 3e-5).
+# Ragged shapes in both dimensions (m and n not multiples of the 128-row
+# tile or the 32-column box), full-width rows (n = 3072) and wider (3200),
+# r from 1 to 32 (padded to 16 or 32 columns), T from 0 to 4.
 @pytest.mark.parametrize("m,n,r,T", [(256, 256, 16, 2), (300, 200, 16, 2), (4444 // 4, 1920 // 4, 16, 2),
                                      (200, 72, 8, 2), (160, 96, 24, 1), (320, 256, 32, 2), (192, 128, 32, 4),
-                                     (130, 64, 16, 0), (128, 128, 1, 3)])
+                                     (130, 64, 16, 0), (128, 128, 1, 3), (700, 1000, 16, 2), (300, 3072, 16, 2),
+                                     (256, 3200, 8, 1)])
 def test_lowrank_matches_oracle(cf, oracle, m, n, r, T):
     k = 3
     As = [synth.lowrank_matrix(m, n, r, mat=i, noise=0.01) for i in range(k)]
@@ -95,14 +99,26 @@ def test_lowrank_matches_oracle(cf, oracle, m, n, r, T):
     check(oracle, As, Q0s, out, T)
 
 
+@pytest.mark.parametrize("k,m,n,r,T", [(8, 1024, 3072, 16, 2), (80, 1000, 128, 8, 1)])
+def test_lowrank_many_tiles_and_matrices(cf, oracle, k, m, n, r, T):
+    """Many matrices of many 128-row tiles in one call: the persistent GEMM
+    walks tiles across matrix boundaries and its pipeline wraps around many
+    times (8 x 1024 x 3072), and 80 matrices of ragged 1000-row tiles."""
+    As = [synth.lowrank_matrix(m, n, r, mat=40 + i, noise=0.01) for i in range(k)]
+    Q0s = [synth.q0(n, r, seed=0, mat=40 + i) for i in range(k)]
+    out = run_gpu(cf, As, Q0s, r, T)
+    check(oracle, As, Q0s, out, T, idx=[0, k // 2 + 1, k - 1])
+
+
 def test_lowrank_many_matrices_chunked(cf, oracle):
-    """More matrices than one launch's descriptor table holds."""
+    """More matrices than one launch's parameter table holds (160 for the
+    GEMM, 192 for CholeskyQR and the apply)."""
     m, n, r, T = 128, 96, 8, 2
-    k = 45
+    k = 200
     As = [synth.lowrank_matrix(m, n, r, mat=i, noise=0.01) for i in range(k)]
     Q0s = [synth.q0(n, r, seed=0, mat=i) for i in range(k)]
     out = run_gpu(cf, As, Q0s, r, T, with_c=False)
-    check(oracle, As, Q0s, out, T, idx=[0, 39, 40, 44])
+    check(oracle, As, Q0s, out, T, idx=[0, 159, 160, 191, 192, 199])
 
 
 def test_lowrank_exact_rank_recovered(cf):
