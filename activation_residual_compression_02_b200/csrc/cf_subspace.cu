@@ -20,9 +20,9 @@
 //    into a double-buffered TMEM accumulator; four warps drain TMEM with
 //    tcgen05.ld and write the r-column result.  The work is HBM-bound (8 flop
 //    per byte of A), so the tensor cores only have to keep up with the stream.
-//  * k_gram / k_chol_solve: CholeskyQR in fp64 -- Gram partials with fp64
-//    atomics, then every CTA recomputes the r x r Cholesky factor and solves
-//    its rows (Y R^{-1}).
+//  * k_cholqr_factor / k_cholqr_apply: CholeskyQR in fp64 -- Gram matrices
+//    of 256-row chunks, summed in chunk order by the last CTA of each
+//    matrix, which factors G = R^T R and inverts R; then Y R^{-1} row by row.
 //  * k_apply: D = U (R V^T) on CUDA cores (K = r is far too thin for the
 //    tensor cores; the step is an HBM stream), fused with E = A - D and
 //    C += D.
@@ -33,6 +33,7 @@
 
 #include <stdlib.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "cf_internal.h"
@@ -330,16 +331,25 @@ static_assert(gemm_smem_bytes<16>() <= 227 * 1024, "GEMM shared memory (RP = 16)
 static_assert(gemm_smem_bytes<32>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
 
 // ------------------------------------------------------ CholeskyQR -------
-constexpr int kGramThreads = 256;
-constexpr int kGramRows = 256;   // rows per Gram CTA
+// Two launches per orthonormalisation.  k_cholqr_factor: CTA (chunk, matrix)
+// forms the Gram matrix of its kCqrRows rows in fp64 and stores it; the CTA
+// that finishes last for a matrix (a counter per matrix) sums the stored Gram
+// matrices in chunk order -- so the result does not depend on timing --,
+// factors G = R^T R with one warp and inverts R with one warp.
+// k_cholqr_apply: every row times R^{-1} in fp64 (the columns of a row are
+// independent, so each thread keeps many multiply-adds in flight).
+constexpr int kCqrThreads = 256;
+constexpr int kCqrRows = 256;   // rows per Gram CTA
 
 struct CholMat {
-    const float *Y;     // input block [rows x ld]
-    double *G;          // Gram matrix [32 x 32] (fp64, zeroed before k_gram)
-    float *Qt;          // mode Q: rounded transposed output [rp x qt_ld] (rows >= r stay zero)
-    float *Qexact;      // mode Q: optional exact output [rows x r] (V)
-    float *U;           // mode U: [rows x r]
-    float *R;           // mode U: [r x r]
+    const float *Y;       // input block [rows x ld]
+    double *Gpart;        // Gram matrix of every chunk, packed upper triangles [chunks][r (r + 1) / 2]
+    unsigned int *count;  // chunks done (zero before the launch; the last CTA resets it)
+    double *Rinv;         // R^{-1} [32 x 32], upper triangular
+    float *Qt;            // mode Q: rounded transposed output [rp x qt_ld] (rows >= r stay zero)
+    float *Qexact;        // mode Q: optional exact output [rows x r] (V)
+    float *U;             // mode U: [rows x r]
+    float *R;             // mode U: [r x r]
 };
 
 constexpr int kMaxCholMats = 192;
@@ -353,35 +363,6 @@ struct CholParams {
     int qt_ld;
     uint32_t *status;
 };
-
-// Gram partials: CTA (chunk, mat) adds Y[chunk]^T Y[chunk] (upper triangle)
-// into G in fp64.
-__global__ void __launch_bounds__(kGramThreads) k_gram(const __grid_constant__ CholParams p)
-{
-    const CholMat &M = p.mat[blockIdx.y];
-    const int r = p.r;
-    const int row0 = blockIdx.x * kGramRows;
-    const int nrows = min(kGramRows, p.rows - row0);
-    __shared__ float ys[kGramRows * 33];
-    for (int i = threadIdx.x; i < nrows * r; i += kGramThreads) {
-        const int rr = i / r, c = i - rr * r;
-        ys[rr * 33 + c] = M.Y[(int64_t)(row0 + rr) * p.ld + c];
-    }
-    __syncthreads();
-    const int npairs = r * (r + 1) / 2;
-    for (int pidx = threadIdx.x; pidx < npairs; pidx += kGramThreads) {
-        // pair index -> (i, j), i <= j
-        int i = 0, rem = pidx;
-        while (rem >= r - i) {
-            rem -= r - i;
-            ++i;
-        }
-        const int j = i + rem;
-        double acc = 0.0;
-        for (int k = 0; k < nrows; ++k) acc += (double)ys[k * 33 + i] * (double)ys[k * 33 + j];
-        atomicAdd(&M.G[i * 32 + j], acc);
-    }
-}
 
 // Upper Cholesky factor of G (G = R^T R) by one warp: lane j owns column j.
 // Step p: lane p forms the diagonal, then every lane q > p forms R[p][q].
@@ -415,54 +396,181 @@ __device__ void cholesky_upper_warp(const double *G, double *R, double *inv_diag
     }
 }
 
-constexpr int kSolveThreads = 256;
+// R^{-1} of the upper triangular R by one warp: lane j forms column j by back
+// substitution, Ri[i][j] = -(sum_{i < k <= j} R[i][k] Ri[k][j]) / R[i][i].
+__device__ void inverse_upper_warp(const double *R, const double *inv_diag, double *Ri, int r)
+{
+    const int j = threadIdx.x & 31;
+    for (int i = 0; i < 32; ++i) Ri[i * 32 + j] = 0.0;
+    if (j < r) {
+        Ri[j * 32 + j] = inv_diag[j];
+        for (int i = j - 1; i >= 0; --i) {
+            double acc = 0.0;
+            for (int k = i + 1; k <= j; ++k) acc += R[i * 32 + k] * Ri[k * 32 + j];
+            Ri[i * 32 + j] = -acc * inv_diag[i];
+        }
+    }
+    __syncwarp();
+}
 
-// Y R^{-1} row by row (forward substitution over the columns), fp64.
-// mode 0: Qt (rounded, transposed) [+ Qexact];  mode 1: U (+ R by CTA 0).
+// Copy n floats between global memory and a row-padded shared tile (row
+// stride 33, `ld` floats per row), 16 bytes at a time where the block allows:
+// a CTA's rows are one contiguous, 16-byte aligned block of n = rows * ld
+// floats.
+template <bool TO_SHARED>
+__device__ __forceinline__ void block_copy(float *gptr, float *tile, int n, int ld)
+{
+    const int n4 = n >> 2;
+    for (int i4 = threadIdx.x; i4 < n4; i4 += kCqrThreads) {
+        const int i = i4 << 2;
+        if (TO_SHARED) {
+            const float4 v = reinterpret_cast<const float4 *>(gptr)[i4];
+            const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) tile[((i + u) / ld) * 33 + (i + u) % ld] = e[u];
+        } else {
+            float e[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) e[u] = tile[((i + u) / ld) * 33 + (i + u) % ld];
+            reinterpret_cast<float4 *>(gptr)[i4] = make_float4(e[0], e[1], e[2], e[3]);
+        }
+    }
+    for (int i = (n4 << 2) + threadIdx.x; i < n; i += kCqrThreads) {
+        if (TO_SHARED)
+            tile[(i / ld) * 33 + i % ld] = gptr[i];
+        else
+            gptr[i] = tile[(i / ld) * 33 + i % ld];
+    }
+}
+
+// Gram matrix, Cholesky factor and its inverse for every matrix of the
+// launch (MODE 1 also stores R, the payload of the final step).
 template <int MODE>
-__global__ void __launch_bounds__(kSolveThreads) k_chol_solve(const __grid_constant__ CholParams p)
+__global__ void __launch_bounds__(kCqrThreads, 3) k_cholqr_factor(const __grid_constant__ CholParams p)
 {
     const CholMat &M = p.mat[blockIdx.y];
     const int r = p.r;
-    __shared__ double Gs[32 * 32];
-    __shared__ double Rs[32 * 32];
+    const int npairs = r * (r + 1) / 2;
+    const int row0 = blockIdx.x * kCqrRows;
+    const int nrows = min(kCqrRows, p.rows - row0);
+    // The staged rows (phase 1) and the r x r matrices of the last CTA
+    // (phase 2) share one buffer: 33.8 KB, of which phase 2 uses 24 KB.
+    __shared__ __align__(16) unsigned char sbuf[kCqrRows * 33 * 4];
+    static_assert(3 * 32 * 32 * sizeof(double) <= sizeof(sbuf), "phase-2 matrices exceed the staging buffer");
+    float *ys = reinterpret_cast<float *>(sbuf);
+    double *Gs = reinterpret_cast<double *>(sbuf);
+    double *Rs = Gs + 32 * 32;
+    double *Ri = Rs + 32 * 32;
     __shared__ double inv_diag[32];
-    for (int i = threadIdx.x; i < 32 * 32; i += kSolveThreads) Gs[i] = M.G[i];
+    __shared__ int is_last;
+    if (p.ld == r) {
+        block_copy<true>(const_cast<float *>(M.Y) + (int64_t)row0 * p.ld, ys, nrows * r, r);
+    } else {
+        for (int i = threadIdx.x; i < nrows * r; i += kCqrThreads) {
+            const int rr = i / r, c = i - rr * r;
+            ys[rr * 33 + c] = M.Y[(int64_t)(row0 + rr) * p.ld + c];
+        }
+    }
     __syncthreads();
-    if (threadIdx.x < 32) cholesky_upper_warp(Gs, Rs, inv_diag, r, p.status, blockIdx.x == 0);
+    for (int pidx = threadIdx.x; pidx < npairs; pidx += kCqrThreads) {
+        // pair index -> (i, j), i <= j
+        int i = 0, rem = pidx;
+        while (rem >= r - i) {
+            rem -= r - i;
+            ++i;
+        }
+        const int j = i + rem;
+        // four interleaved partial sums (rows k = 4q + u), added in a fixed
+        // order at the end: a quarter of the dependent fp64 chain
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        int k = 0;
+        for (; k + 4 <= nrows; k += 4) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] += (double)ys[(k + u) * 33 + i] * (double)ys[(k + u) * 33 + j];
+        }
+        for (; k < nrows; ++k) acc[0] += (double)ys[k * 33 + i] * (double)ys[k * 33 + j];
+        M.Gpart[(int64_t)blockIdx.x * npairs + pidx] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+    // The last CTA of this matrix to get here finishes the factorisation.
+    __threadfence();
     __syncthreads();
-    if (MODE == 1 && blockIdx.x == 0) {
-        for (int i = threadIdx.x; i < r * r; i += kSolveThreads) {
+    if (threadIdx.x == 0) is_last = atomicAdd(M.count, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int pidx = threadIdx.x; pidx < npairs; pidx += kCqrThreads) {
+        int i = 0, rem = pidx;
+        while (rem >= r - i) {
+            rem -= r - i;
+            ++i;
+        }
+        const int j = i + rem;
+        // loads of eight chunks in flight at a time, added in chunk order
+        double g = 0.0;
+        for (unsigned c0 = 0; c0 < gridDim.x; c0 += 8) {
+            double v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = c0 + u < gridDim.x ? __ldcg(M.Gpart + (int64_t)(c0 + u) * npairs + pidx) : 0.0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (c0 + u < gridDim.x) g += v[u];
+        }
+        Gs[i * 32 + j] = g;
+    }
+    if (threadIdx.x == 0) *M.count = 0u;   // ready for the next orthonormalisation
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        cholesky_upper_warp(Gs, Rs, inv_diag, r, p.status, true);
+        inverse_upper_warp(Rs, inv_diag, Ri, r);
+    }
+    __syncthreads();
+    if (MODE == 1) {
+        for (int i = threadIdx.x; i < r * r; i += kCqrThreads) {
             const int a = i / r, b = i - a * r;
             M.R[i] = (float)Rs[a * 32 + b];
         }
     }
-    const int row = blockIdx.x * kSolveThreads + threadIdx.x;
-    if (row >= p.rows) return;
-    double q[32];
-    const float *y = M.Y + (int64_t)row * p.ld;
+    for (int i = threadIdx.x; i < 32 * 32; i += kCqrThreads) M.Rinv[i] = Ri[i];
+}
+
+// Q = Y R^{-1} row by row.  MODE 0: Q into Qt (TF32-rounded, transposed)
+// [+ Qexact]; MODE 1: U.  The CTA's rows come in, and its row-major outputs
+// go out, through a shared tile with 16-byte accesses; a thread keeps its
+// row (RMAX doubles) in registers and forms one output column at a time, so
+// that several CTAs fit on an SM.
+template <int MODE, int RMAX>
+__global__ void __launch_bounds__(kCqrThreads) k_cholqr_apply(const __grid_constant__ CholParams p)
+{
+    const CholMat &M = p.mat[blockIdx.y];
+    const int r = p.r;
+    __shared__ double Ri[32 * 32];
+    __shared__ float tile[kCqrThreads * 33];
+    const int row0 = blockIdx.x * kCqrThreads;
+    const int nrows = min(kCqrThreads, p.rows - row0);
+    for (int i = threadIdx.x; i < 32 * 32; i += kCqrThreads) Ri[i] = M.Rinv[i];
+    block_copy<true>(const_cast<float *>(M.Y) + (int64_t)row0 * p.ld, tile, nrows * p.ld, p.ld);
+    __syncthreads();
+    const int t = threadIdx.x;
+    const int row = row0 + t;
+    double yv[RMAX];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
+    for (int k = 0; k < RMAX; ++k) yv[k] = (k < r && t < nrows) ? (double)tile[t * 33 + k] : 0.0;
+    __syncthreads();   // every row is in registers: the tile now collects outputs
+    float *out = MODE == 0 ? M.Qexact : M.U;
+#pragma unroll
+    for (int c = 0; c < RMAX; ++c) {
         if (c < r) {
-            double v = (double)y[c];
+            double acc = 0.0;
 #pragma unroll
-            for (int k = 0; k < c; ++k) v -= q[k] * Rs[k * 32 + c];
-            q[c] = v * inv_diag[c];
+            for (int k = 0; k <= c; ++k) acc += yv[k] * Ri[k * 32 + c];
+            if (MODE == 0 && t < nrows) M.Qt[(int64_t)c * p.qt_ld + row] = round_tf32((float)acc);
+            tile[t * 33 + c] = (float)acc;
         }
     }
-    if (MODE == 0) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-            if (c < r) M.Qt[(int64_t)c * p.qt_ld + row] = round_tf32((float)q[c]);
-        if (M.Qexact) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-                if (c < r) M.Qexact[(int64_t)row * r + c] = (float)q[c];
-        }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-            if (c < r) M.U[(int64_t)row * r + c] = (float)q[c];
+    if (out) {
+        __syncthreads();
+        block_copy<false>(out + (int64_t)row0 * r, tile, nrows * r, r);
     }
 }
 
@@ -762,7 +870,8 @@ int64_t rup(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 struct WsLayout {
     int rp;
     int64_t mp, np;                       // padded leading dims (multiples of 32)
-    size_t qt, pt, pe, z, g, total;       // byte offsets inside the workspace
+    size_t qt, pt, pe, z, cnt, gp, ri, total;   // byte offsets inside the workspace
+    int chunks;                           // Gram chunks of the tallest block
 };
 
 WsLayout layout(int nmat, int64_t m, int64_t n, int r)
@@ -781,7 +890,10 @@ WsLayout layout(int nmat, int64_t m, int64_t n, int r)
     L.pt = take((size_t)nmat * L.rp * L.mp * 4);
     L.pe = take((size_t)nmat * m * L.rp * 4);
     L.z = take((size_t)nmat * n * L.rp * 4);
-    L.g = take((size_t)nmat * 32 * 32 * 8);
+    L.cnt = take((size_t)nmat * sizeof(unsigned int));
+    L.chunks = (int)((std::max(m, n) + kCqrRows - 1) / kCqrRows);
+    L.gp = take((size_t)nmat * L.chunks * (r * (r + 1) / 2) * 8);
+    L.ri = take((size_t)nmat * 32 * 32 * 8);
     L.total = off;
     return L;
 }
@@ -876,19 +988,19 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
 }
 
 // CholeskyQR of a tall block for every matrix: mode 0 writes Qt (+ V when
-// `final_v`), mode 1 writes U and R.
+// `final_v`), mode 1 writes U and R.  Two launches (per 192 matrices).
 cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLayout &L, int src, int mode,
                         bool final_v, cudaStream_t stream)
 {
     char *ws = (char *)pl.ws;
     const int64_t m = pl.m, n = pl.n;
     const int r = pl.r;
+    const int npairs = r * (r + 1) / 2;
     // src: 0 = Q0 (n x r), 1 = Z (n x rp), 2 = P exact (m x rp)
     const int rows = (int)(src == 2 ? m : n);
     const int ld = src == 0 ? r : L.rp;
-    cudaError_t err = cudaMemsetAsync(ws + L.g, 0, (size_t)pl.nmat * 32 * 32 * 8, stream);
-    if (err != cudaSuccess) return err;
     CholParams *cp = new CholParams;
+    cudaError_t err = cudaSuccess;
     for (int first = 0; first < pl.nmat && err == cudaSuccess; first += kMaxCholMats) {
         const int cnt = pl.nmat - first < kMaxCholMats ? pl.nmat - first : kMaxCholMats;
         memset(cp, 0, sizeof *cp);
@@ -904,21 +1016,30 @@ cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsL
             c.Y = src == 0 ? mats[i].Q0
                            : (src == 1 ? (const float *)(ws + L.z + (size_t)i * n * L.rp * 4)
                                        : (const float *)(ws + L.pe + (size_t)i * m * L.rp * 4));
-            c.G = (double *)(ws + L.g + (size_t)i * 32 * 32 * 8);
+            c.Gpart = (double *)(ws + L.gp + (size_t)i * L.chunks * npairs * 8);
+            c.count = (unsigned int *)(ws + L.cnt) + i;
+            c.Rinv = (double *)(ws + L.ri + (size_t)i * 32 * 32 * 8);
             c.Qt = (float *)(ws + L.qt + (size_t)i * L.rp * L.np * 4);
             c.Qexact = final_v ? mats[i].V : nullptr;
             c.U = mats[i].U;
             c.R = mats[i].R;
         }
-        dim3 ggrid((unsigned)((rows + kGramRows - 1) / kGramRows), (unsigned)cnt);
-        k_gram<<<ggrid, kGramThreads, 0, stream>>>(*cp);
-        err = cudaGetLastError();
-        if (err != cudaSuccess) break;
-        dim3 sgrid((unsigned)((rows + kSolveThreads - 1) / kSolveThreads), (unsigned)cnt);
-        if (mode == 0)
-            k_chol_solve<0><<<sgrid, kSolveThreads, 0, stream>>>(*cp);
-        else
-            k_chol_solve<1><<<sgrid, kSolveThreads, 0, stream>>>(*cp);
+        dim3 fgrid((unsigned)((rows + kCqrRows - 1) / kCqrRows), (unsigned)cnt);
+        dim3 agrid((unsigned)((rows + kCqrThreads - 1) / kCqrThreads), (unsigned)cnt);
+        const bool r16 = r <= 16;
+        if (mode == 0) {
+            k_cholqr_factor<0><<<fgrid, kCqrThreads, 0, stream>>>(*cp);
+            if (r16)
+                k_cholqr_apply<0, 16><<<agrid, kCqrThreads, 0, stream>>>(*cp);
+            else
+                k_cholqr_apply<0, 32><<<agrid, kCqrThreads, 0, stream>>>(*cp);
+        } else {
+            k_cholqr_factor<1><<<fgrid, kCqrThreads, 0, stream>>>(*cp);
+            if (r16)
+                k_cholqr_apply<1, 16><<<agrid, kCqrThreads, 0, stream>>>(*cp);
+            else
+                k_cholqr_apply<1, 32><<<agrid, kCqrThreads, 0, stream>>>(*cp);
+        }
         err = cudaGetLastError();
     }
     delete cp;
@@ -1000,6 +1121,8 @@ cudaError_t run_lowrank(const LowrankPlan &pl, const LowrankMat *mats, cudaStrea
     // Padded rows of Q^T (rows r..rp-1) must be zero: they feed zero columns.
     cudaError_t err = cudaMemsetAsync(ws + L.qt, 0, (size_t)pl.nmat * L.rp * L.np * 4, stream);
     if (err == cudaSuccess) err = cudaMemsetAsync(ws + L.pt, 0, (size_t)pl.nmat * L.rp * L.mp * 4, stream);
+    // CholeskyQR chunk counters start at zero (each launch leaves them at zero)
+    if (err == cudaSuccess) err = cudaMemsetAsync(ws + L.cnt, 0, (size_t)pl.nmat * sizeof(unsigned int), stream);
     // Line 1: Q = orth(Q0).
     if (err == cudaSuccess) err = cholqr_pass(pl, mats, L, 0, 0, pl.T == 0, stream);
     // Lines 2-5: T times Z = A^T (A Q), Q = orth(Z).

@@ -179,8 +179,9 @@ cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
 
 /* Workspace cf_lowrank needs for nmat matrices of m x n at this context's
  * rank: the r-column blocks of Algorithm 3 (Q^T, P^T, P, Z, padded to 16 or
- * 32 columns) and their fp64 Gram matrices, about 4*rp*(2m + 2n) + 8 KB
- * bytes per matrix.  Returns 0 for a quantised-mode context or bad sizes. */
+ * 32 columns), the fp64 Gram matrices of their 256-row chunks and R^{-1},
+ * about 4*rp*(2m + 2n) + 4*r*(r+1)*ceil(max(m, n)/256) + 8 KB bytes per
+ * matrix.  Returns 0 for a quantised-mode context or bad sizes. */
 size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_t n);
 
 /* Algorithm 3 (subspace iteration, rank r = config.rank, T = config.iters
@@ -222,8 +223,9 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
  * iteration count T taken from `config` (mode must be CF_MODE_LOWRANK);
  * A, Q0, U, R, V, E_opt, C_opt are host arrays of nmat device pointers.
  * Limits: the Algorithm 3 buffers of the call -- cf_lowrank_workspace_bytes
- * for the same nmat, m, n and r, about 4*rp*(2m + 2n) + 8 KB per matrix with
- * rp = 16 (r <= 16) or 32 -- must fit in CF_NOALLOC_SCRATCH_BYTES - 256
+ * for the same nmat, m, n and r, about 4*rp*(2m + 2n) + 4*r*(r+1)*ceil(max(m,
+ * n)/256) + 8 KB per matrix with rp = 16 (r <= 16) or 32 -- must fit in
+ * CF_NOALLOC_SCRATCH_BYTES - 256
  * bytes, and nmat <= 512; otherwise the call returns CF_E_NOMEM and launches
  * nothing.  Eight 4608 x 3072 matrices at r = 16 fit in one call.
  *

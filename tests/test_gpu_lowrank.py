@@ -110,6 +110,20 @@ def test_lowrank_many_tiles_and_matrices(cf, oracle, k, m, n, r, T):
     check(oracle, As, Q0s, out, T, idx=[0, k // 2 + 1, k - 1])
 
 
+def test_lowrank_is_deterministic(cf):
+    """Every sum of the path runs in a fixed order (the GEMM's K loop, the
+    CholeskyQR Gram chunks summed in chunk order, no atomics): two calls on
+    the same inputs give bit-identical factors and error buffers."""
+    m, n, r, T, k = 1152, 3072, 16, 2, 5
+    As = [synth.lowrank_matrix(m, n, r, mat=30 + i, noise=0.01) for i in range(k)]
+    Q0s = [synth.q0(n, r, seed=0, mat=30 + i) for i in range(k)]
+    a = run_gpu(cf, As, Q0s, r, T, with_c=False)
+    b = run_gpu(cf, As, Q0s, r, T, with_c=False)
+    for key in ("U", "R", "V", "E"):
+        for i in range(k):
+            assert np.array_equal(a[key][i], b[key][i]), (key, i)
+
+
 def test_lowrank_many_matrices_chunked(cf, oracle):
     """More matrices than one launch's parameter table holds (160 for the
     GEMM, 192 for CholeskyQR and the apply)."""
