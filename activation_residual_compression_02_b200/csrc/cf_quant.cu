@@ -31,28 +31,34 @@
 namespace cf {
 namespace {
 
-// Launch shape per operation: threads per CTA, vectors (of 8 elements) each
-// thread keeps in flight (a tile is threads * unroll vectors), and a cap on
-// resident CTAs per SM (0: as many as fit).  Chosen by sweeps on the B200
-// over 128..1024 threads, 1..8 vectors and 1..4 CTAs per SM on the 57-slot
-// FLUX-shaped step: compress wants many warps to hide its ~150 instructions
-// per vector (1024 x 1: 93.5% of the measured copy bandwidth, against 88% for
-// 256 x 4 at 2 CTAs/SM); decompress wants about 512 resident threads per SM
-// with 4 vectors each (94.5%, against 84% at 4 CTAs/SM).
+// Launch shape per operation (and, for the fp32-state sender and receiver,
+// per code width k): threads per CTA, vectors (of 8 elements) each thread
+// keeps in flight (a tile is threads * unroll vectors), and a cap on resident
+// CTAs per SM (0: as many as fit).  Chosen by sweeps on the B200 over
+// 128..1024 threads, 1..16 vectors and 1..4 CTAs per SM on the 57-slot
+// FLUX-shaped (k = 2), 30-slot CogVideoX-shaped (k = 4) and 60-slot stress
+// (k = 1) steps, as a fraction of the measured copy bandwidth:
+//   compress   k = 2: 256 x 8 at 1 CTA/SM, 95.3% (1024 x 1: 93.4%)
+//              k = 4: 512 x 2, 94.0% (1024 x 1: 89.5%; 256 x 8: 91.4%)
+//              k = 1: 512 x 2, 93.3% (1024 x 1: 89.3%)
+//   decompress k = 2, 4: 512 x 4 at 1 CTA/SM, 94.5% / 93.1% (256 x 8: 90.1% / 92.1%)
+//              k = 1: 256 x 8, 98.9% (512 x 4: 89.1%)
+// More resident CTAs per SM, i.e. more concurrent streams into HBM, were
+// slower in every case.
 template <QuantOp OP, bool LEAN = false>
-struct QShape {
+struct QShapeBase {
     static constexpr int kThreads = 256;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 0;
 };
 template <>
-struct QShape<QuantOp::Compress, false> {
+struct QShapeBase<QuantOp::Compress, false> {
     static constexpr int kThreads = 1024;
     static constexpr int kUnroll = 1;
     static constexpr int kMaxPerSm = 1;   // 2 CTAs of 1024 fit at 32 registers, and are slower
 };
 template <>
-struct QShape<QuantOp::Loopback, false> {
+struct QShapeBase<QuantOp::Loopback, false> {
     // fused sender + receiver: 9 streams per tile; best of the sweep (90.6%
     // of the copy peak), still below the separate pair (94.3%)
     static constexpr int kThreads = 256;
@@ -60,7 +66,7 @@ struct QShape<QuantOp::Loopback, false> {
     static constexpr int kMaxPerSm = 1;
 };
 template <>
-struct QShape<QuantOp::Decompress, false> {
+struct QShapeBase<QuantOp::Decompress, false> {
     static constexpr int kThreads = 512;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 1;
@@ -68,27 +74,43 @@ struct QShape<QuantOp::Decompress, false> {
 // Lean state (bf16 E and C): half the state bytes per vector, so each thread
 // wants more vectors in flight (sweep on the same workload).
 template <>
-struct QShape<QuantOp::Compress, true> {
+struct QShapeBase<QuantOp::Compress, true> {
     static constexpr int kThreads = 1024;
     static constexpr int kUnroll = 2;
     static constexpr int kMaxPerSm = 1;
 };
 template <>
-struct QShape<QuantOp::Loopback, true> {
+struct QShapeBase<QuantOp::Loopback, true> {
     static constexpr int kThreads = 256;
     static constexpr int kUnroll = 8;
     static constexpr int kMaxPerSm = 1;
 };
 template <>
-struct QShape<QuantOp::Decompress, true> {
+struct QShapeBase<QuantOp::Decompress, true> {
     static constexpr int kThreads = 1024;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 1;
 };
-template <QuantOp OP, bool LEAN>
+template <QuantOp OP, bool LEAN, int K>
+struct QShape : QShapeBase<OP, LEAN> {};
+template <int T, int U>
+struct QShapeOne {
+    static constexpr int kThreads = T;
+    static constexpr int kUnroll = U;
+    static constexpr int kMaxPerSm = 1;
+};
+template <>
+struct QShape<QuantOp::Compress, false, 2> : QShapeOne<256, 8> {};
+template <>
+struct QShape<QuantOp::Compress, false, 4> : QShapeOne<512, 2> {};
+template <>
+struct QShape<QuantOp::Compress, false, 1> : QShapeOne<512, 2> {};
+template <>
+struct QShape<QuantOp::Decompress, false, 1> : QShapeOne<256, 8> {};
+template <QuantOp OP, bool LEAN, int K>
 constexpr int64_t qtile_vec()
 {
-    return (int64_t)QShape<OP, LEAN>::kThreads * QShape<OP, LEAN>::kUnroll;
+    return (int64_t)QShape<OP, LEAN, K>::kThreads * QShape<OP, LEAN, K>::kUnroll;
 }
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kAbsMask = 0x7fffffffu;
@@ -205,11 +227,11 @@ __device__ __forceinline__ float group_scale(const float (&a)[8], bool &nonfinit
 }
 
 template <QuantOp OP, int K, int G, int SS, bool LEAN>
-__global__ void __launch_bounds__(QShape<OP, LEAN>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
+__global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
 {
     using SV = StateVec<LEAN>;
-    constexpr int kThreads = QShape<OP, LEAN>::kThreads;
-    constexpr int kUnroll = QShape<OP, LEAN>::kUnroll;
+    constexpr int kThreads = QShape<OP, LEAN, K>::kThreads;
+    constexpr int kUnroll = QShape<OP, LEAN, K>::kUnroll;
     constexpr int kTileVec = kThreads * kUnroll;
     constexpr int LPG = G / 8;
     constexpr int L = (K >= 2) ? (1 << (K - 1)) - 1 : 1;
@@ -474,39 +496,40 @@ struct Shape {
     int per_sm;
 };
 
+template <QuantOp OP, bool LEAN, int K>
+void shape_is(int &threads, int &cap, int64_t &tile_vec)
+{
+    threads = QShape<OP, LEAN, K>::kThreads;
+    cap = QShape<OP, LEAN, K>::kMaxPerSm;
+    tile_vec = qtile_vec<OP, LEAN, K>();
+}
+
+template <QuantOp OP, bool LEAN>
+void shape_bits(int bits, int &threads, int &cap, int64_t &tile_vec)
+{
+    if (bits == 1)
+        shape_is<OP, LEAN, 1>(threads, cap, tile_vec);
+    else if (bits == 4)
+        shape_is<OP, LEAN, 4>(threads, cap, tile_vec);
+    else
+        shape_is<OP, LEAN, 2>(threads, cap, tile_vec);
+}
+
+// The shape of the instance pick() returns: the warmup kernels are the k = 2
+// instances.
 template <bool LEAN>
-void shape_of(QuantOp op, int &threads, int &cap, int64_t &tile_vec)
+void shape_of(QuantOp op, int bits, int &threads, int &cap, int64_t &tile_vec)
 {
     switch (op) {
-    case QuantOp::WarmupSender:
-        threads = QShape<QuantOp::WarmupSender, LEAN>::kThreads;
-        cap = QShape<QuantOp::WarmupSender, LEAN>::kMaxPerSm;
-        tile_vec = qtile_vec<QuantOp::WarmupSender, LEAN>();
-        break;
-    case QuantOp::WarmupReceiver:
-        threads = QShape<QuantOp::WarmupReceiver, LEAN>::kThreads;
-        cap = QShape<QuantOp::WarmupReceiver, LEAN>::kMaxPerSm;
-        tile_vec = qtile_vec<QuantOp::WarmupReceiver, LEAN>();
-        break;
-    case QuantOp::Compress:
-        threads = QShape<QuantOp::Compress, LEAN>::kThreads;
-        cap = QShape<QuantOp::Compress, LEAN>::kMaxPerSm;
-        tile_vec = qtile_vec<QuantOp::Compress, LEAN>();
-        break;
-    case QuantOp::Decompress:
-        threads = QShape<QuantOp::Decompress, LEAN>::kThreads;
-        cap = QShape<QuantOp::Decompress, LEAN>::kMaxPerSm;
-        tile_vec = qtile_vec<QuantOp::Decompress, LEAN>();
-        break;
-    case QuantOp::Loopback:
-        threads = QShape<QuantOp::Loopback, LEAN>::kThreads;
-        cap = QShape<QuantOp::Loopback, LEAN>::kMaxPerSm;
-        tile_vec = qtile_vec<QuantOp::Loopback, LEAN>();
-        break;
+    case QuantOp::WarmupSender: shape_is<QuantOp::WarmupSender, LEAN, 2>(threads, cap, tile_vec); break;
+    case QuantOp::WarmupReceiver: shape_is<QuantOp::WarmupReceiver, LEAN, 2>(threads, cap, tile_vec); break;
+    case QuantOp::Compress: shape_bits<QuantOp::Compress, LEAN>(bits, threads, cap, tile_vec); break;
+    case QuantOp::Decompress: shape_bits<QuantOp::Decompress, LEAN>(bits, threads, cap, tile_vec); break;
+    case QuantOp::Loopback: shape_bits<QuantOp::Loopback, LEAN>(bits, threads, cap, tile_vec); break;
     }
 }
 
-Shape launch_shape(KernelFn fn, bool lean, QuantOp op)
+Shape launch_shape(KernelFn fn, bool lean, QuantOp op, int bits)
 {
     static std::mutex mu;
     static std::unordered_map<const void *, Shape> cache;
@@ -517,9 +540,9 @@ Shape launch_shape(KernelFn fn, bool lean, QuantOp op)
     int cap = 0;
     int64_t tile_vec = 0;
     if (lean)
-        shape_of<true>(op, sh.threads, cap, tile_vec);
+        shape_of<true>(op, bits, sh.threads, cap, tile_vec);
     else
-        shape_of<false>(op, sh.threads, cap, tile_vec);
+        shape_of<false>(op, bits, sh.threads, cap, tile_vec);
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, sh.threads, sh.smem) != cudaSuccess || nb < 1) nb = 1;
     sh.per_sm = (cap > 0 && nb > cap) ? cap : nb;
@@ -550,9 +573,9 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool l
     int threads = 0, cap = 0;
     int64_t tile_vec = 0;
     if (lean)
-        shape_of<true>(op, threads, cap, tile_vec);
+        shape_of<true>(op, bits, threads, cap, tile_vec);
     else
-        shape_of<false>(op, threads, cap, tile_vec);
+        shape_of<false>(op, bits, threads, cap, tile_vec);
     int64_t tiles = 0;
     for (int k = 0; k < lp.nslots; ++k) {
         lp.slot[k].tile0 = tiles;
@@ -560,7 +583,7 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool l
     }
     lp.ntiles = tiles;
     if (tiles <= 0) return cudaSuccess;
-    const Shape sh = launch_shape(fn, lean, op);
+    const Shape sh = launch_shape(fn, lean, op, bits);
     const int64_t cap_blocks = (int64_t)num_sms() * sh.per_sm;
     const int grid = (int)(tiles < cap_blocks ? tiles : cap_blocks);
     fn<<<grid, sh.threads, sh.smem, stream>>>(lp);
