@@ -107,6 +107,13 @@ template <>
 struct QShape<QuantOp::Compress, false, 1> : QShapeOne<512, 2> {};
 template <>
 struct QShape<QuantOp::Decompress, false, 1> : QShapeOne<256, 8> {};
+// Lean-state sender (bf16 E): 1024 x 2 stays best for k = 2 (91.3%); k = 4 and
+// k = 1 want more vectors per thread: 512 x 4 (88.4 -> 91.4%) and 256 x 16
+// (87.8 -> 91.5%), steps of the CogVideoX-shaped and stress workloads.
+template <>
+struct QShape<QuantOp::Compress, true, 4> : QShapeOne<512, 4> {};
+template <>
+struct QShape<QuantOp::Compress, true, 1> : QShapeOne<256, 16> {};
 template <QuantOp OP, bool LEAN, int K>
 constexpr int64_t qtile_vec()
 {
