@@ -59,10 +59,9 @@ struct QShapeBase<QuantOp::Compress, false> {
 };
 template <>
 struct QShapeBase<QuantOp::Loopback, false> {
-    // fused sender + receiver: 9 streams per tile; best of the sweep (90.6%
-    // of the copy peak), still below the separate pair (94.3%)
+    // fused sender + receiver (9 streams per tile); per-width shapes below
     static constexpr int kThreads = 256;
-    static constexpr int kUnroll = 8;
+    static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 1;
 };
 template <>
@@ -107,6 +106,13 @@ template <>
 struct QShape<QuantOp::Compress, false, 1> : QShapeOne<512, 2> {};
 template <>
 struct QShape<QuantOp::Decompress, false, 1> : QShapeOne<256, 8> {};
+// Loopback (sender and receiver of a step in one kernel): 256 x 4 for k = 2
+// (94.96%, faster than the separate pair), 320 x 4 for k = 4 (91.0%), 256 x 6
+// for k = 1 (92.7%); the shape is sensitive (256 x 3: 79.7% for k = 2).
+template <>
+struct QShape<QuantOp::Loopback, false, 4> : QShapeOne<320, 4> {};
+template <>
+struct QShape<QuantOp::Loopback, false, 1> : QShapeOne<256, 6> {};
 // Lean-state sender (bf16 E): 1024 x 2 stays best for k = 2 (91.3%); k = 4 and
 // k = 1 want more vectors per thread: 512 x 4 (88.4 -> 91.4%) and 256 x 16
 // (87.8 -> 91.5%), steps of the CogVideoX-shaped and stress workloads.
