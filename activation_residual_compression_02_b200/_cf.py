@@ -22,7 +22,7 @@ CF_MODE_QUANT, CF_MODE_LOWRANK = 0, 1
 
 EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
             "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
-            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback"]
+            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback", "cf_resume"]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.cf_last_error.restype = ctypes.c_char_p
         L.cf_destroy.argtypes = [P]
         L.cf_destroy.restype = I
+        L.cf_resume.argtypes = [P, I64]
+        L.cf_resume.restype = I
         L.cf_lowrank_noalloc.argtypes = [ctypes.POINTER(cf_config), I, I64, I64, PP, PP, PP, PP, PP, PP, PP, P]
         L.cf_lowrank_noalloc.restype = I
         _lib = L
@@ -205,6 +207,11 @@ class Context:
                               _parr(C), _stream_handle(stream))
         self._raise(st, "cf_lowrank")
 
+    def resume(self, steps_done: int):
+        """Continue a run whose state buffers the caller restored (steps
+        0..steps_done done); the next call may be step steps_done + 1."""
+        self._raise(lib().cf_resume(self._h, steps_done), "cf_resume")
+
     def check(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         """Synchronise and return the device status (CF_OK, CF_E_NONFINITE, ...)."""
         return int(lib().cf_check(self._h, _stream_handle(stream)))
@@ -248,6 +255,10 @@ def cf_check(ctx: Context, stream=None) -> int:
 
 def cf_payload_bytes(ctx: Context, slot: int) -> int:
     return ctx.payload_bytes(slot)
+
+
+def cf_resume(ctx: Context, steps_done: int):
+    ctx.resume(steps_done)
 
 
 def cf_destroy(ctx: Context):

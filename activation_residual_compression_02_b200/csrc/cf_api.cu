@@ -6,6 +6,7 @@
 // "Dataset Splits" row (an uncompressed warmup step initialises the base
 // tensor) and "Pseudocode" row, Algorithm 3 (rank-r subspace iteration).
 #include <stdarg.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -27,6 +28,26 @@ struct cf_ctx {
     int device = 0;
     std::string err;
 };
+
+namespace cf {
+
+bool log_enabled()
+{
+    static const bool on = [] {
+        const char *v = getenv("CF_LOG");
+        return v && v[0] == '1';
+    }();
+    return on;
+}
+
+void log_launch(const char *kernel, dim3 grid, dim3 block, size_t smem)
+{
+    if (!log_enabled()) return;
+    fprintf(stderr, "cf: launch %s grid (%u, %u, %u) block (%u, %u, %u) smem %zu\n", kernel, grid.x, grid.y, grid.z,
+            block.x, block.y, block.z, smem);
+}
+
+}  // namespace cf
 
 namespace {
 
@@ -455,6 +476,17 @@ const char *cf_last_error(const cf_ctx *ctx)
 {
     if (!ctx) return "null context";
     return ctx->err.c_str();
+}
+
+cf_status cf_resume(cf_ctx *ctx, int64_t steps_done)
+{
+    if (!ctx) return CF_E_ARG;
+    if (steps_done < 0) return fail(ctx, CF_E_ARG, "steps_done must be >= 0");
+    ctx->warm_sender = true;
+    ctx->warm_receiver = true;
+    ctx->lowrank_steps = steps_done;   // compressed steps after the warmup
+    ctx->err.clear();
+    return CF_OK;
 }
 
 cf_status cf_destroy(cf_ctx *ctx)

@@ -86,4 +86,10 @@ cudaError_t launch_residual_f32(const void *const *x, void *const *base, const f
 
 int num_sms();
 
+// Host-side launch log: with CF_LOG=1 in the environment (read once), every
+// kernel launch prints one line to stderr with its name, grid, block and
+// dynamic shared memory.
+void log_launch(const char *kernel, dim3 grid, dim3 block, size_t smem);
+bool log_enabled();
+
 }  // namespace cf

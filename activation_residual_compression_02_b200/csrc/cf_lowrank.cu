@@ -74,6 +74,7 @@ cudaError_t launch_residual_f32(const void *const *x, void *const *base, const f
             const int64_t cap = (int64_t)num_sms() * 8 / (cnt > 0 ? cnt : 1) + 1;
             if (bx > cap) bx = cap;
             dim3 grid((unsigned)bx, (unsigned)cnt);
+            log_launch("k_residual_f32", grid, dim3(kResThreads), 0);
             k_residual_f32<<<grid, kResThreads, 0, stream>>>(*p);
         }
         delete p;

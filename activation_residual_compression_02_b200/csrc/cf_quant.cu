@@ -22,6 +22,7 @@
 // contraction can change a code; the absmax is an integer max over the
 // magnitude bits (exact, and a NaN or infinity is seen as non-finite).
 #include <cuda_bf16.h>
+#include <stdio.h>
 
 #include <mutex>
 #include <unordered_map>
@@ -599,6 +600,12 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool l
     const Shape sh = launch_shape(fn, lean, op, bits);
     const int64_t cap_blocks = (int64_t)num_sms() * sh.per_sm;
     const int grid = (int)(tiles < cap_blocks ? tiles : cap_blocks);
+    if (log_enabled()) {
+        char name[64];
+        snprintf(name, sizeof name, "k_quant<op %d, k %d, G %d, ss %d, %s>", (int)op, bits, group, sign_scale,
+                 lean ? "bf16 state" : "fp32 state");
+        log_launch(name, dim3(grid), dim3(sh.threads), sh.smem);
+    }
     fn<<<grid, sh.threads, sh.smem, stream>>>(lp);
     return cudaGetLastError();
 }

@@ -908,6 +908,7 @@ cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
                                         (int)gemm_smem_bytes<RP>());
     });
     if (attr_err != cudaSuccess) return attr_err;
+    log_launch(RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>", dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP>());
     k_gemm_tf32<RP><<<grid, kGemmThreads, gemm_smem_bytes<RP>(), stream>>>(gp);
     return cudaGetLastError();
 }
@@ -1027,6 +1028,8 @@ cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsL
         dim3 fgrid((unsigned)((rows + kCqrRows - 1) / kCqrRows), (unsigned)cnt);
         dim3 agrid((unsigned)((rows + kCqrThreads - 1) / kCqrThreads), (unsigned)cnt);
         const bool r16 = r <= 16;
+        log_launch(mode == 0 ? "k_cholqr_factor<Q>" : "k_cholqr_factor<U>", fgrid, dim3(kCqrThreads), 0);
+        log_launch(mode == 0 ? "k_cholqr_apply<Q>" : "k_cholqr_apply<U>", agrid, dim3(kCqrThreads), 0);
         if (mode == 0) {
             k_cholqr_factor<0><<<fgrid, kCqrThreads, 0, stream>>>(*cp);
             if (r16)
@@ -1092,6 +1095,7 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
                 smem = async_smem_bytes<false, true>();
             }
             cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            log_launch("k_apply_async", dim3(blocks), dim3(kApplyThreads), smem);
             fn<<<blocks, kApplyThreads, smem, stream>>>(*ap);
             err = cudaGetLastError();
             continue;
@@ -1100,6 +1104,7 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
             fn = has_e ? (has_c ? k_apply<16, true, true> : k_apply<16, true, false>) : k_apply<16, false, true>;
         else
             fn = has_e ? (has_c ? k_apply<32, true, true> : k_apply<32, true, false>) : k_apply<32, false, true>;
+        log_launch("k_apply", dim3(blocks), dim3(kApplyThreads), 0);
         fn<<<blocks, kApplyThreads, 0, stream>>>(*ap);
         err = cudaGetLastError();
     }

@@ -256,6 +256,17 @@ size_t cf_payload_bytes(const cf_ctx *ctx, int slot);
  * The string is owned by the context. */
 const char *cf_last_error(const cf_ctx *ctx);
 
+/* Resume a run from caller-saved state (checkpoint / restart).  All codec
+ * state lives in caller memory -- base, err and cache of every slot, and V
+ * for the low-rank warm start -- so a checkpoint is a copy of those buffers
+ * plus the index of the last step done.  After restoring them, call this on
+ * a fresh context with the same configuration and shapes: it records that
+ * steps 0..steps_done (the warmup included) have run on both the sender and
+ * the receiver side, so the next call may be step steps_done + 1, and a
+ * warm-start low-rank context starts Algorithm 3 from the restored V.
+ * Enqueues nothing.  Errors: CF_E_ARG (NULL context, steps_done < 0). */
+cf_status cf_resume(cf_ctx *ctx, int64_t steps_done);
+
 /* Free the context (waits for nothing; the caller must not destroy a
  * context while its launches are still running on a stream). */
 cf_status cf_destroy(cf_ctx *ctx);

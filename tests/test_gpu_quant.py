@@ -83,6 +83,14 @@ def test_loopback_bit_exact(cf, oracle, bits, group, ss):
     run_case(cf, oracle, shapes, 4, bits, group, ss, w=synth.FLUX, loopback=True)
 
 
+@pytest.mark.parametrize("bits,group", [(2, 128), (1, 128), (4, 64)])
+def test_more_slots_than_one_launch(cf, oracle, bits, group):
+    """A call with more slots than one grouped launch's table holds (128) is
+    split into several launches; every slot still matches the oracle."""
+    shapes = [(3 + i % 5, 256) for i in range(131)]
+    run_case(cf, oracle, shapes, 3, bits, group, w=synth.FLUX, check_every_step=False)
+
+
 def test_grouped_equals_per_slot(cf):
     """Launch-shape invariance: one grouped launch over all slots equals one
     context (and launch) per slot, bit for bit."""
