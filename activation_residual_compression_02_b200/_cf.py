@@ -39,7 +39,8 @@ class cf_shape(ctypes.Structure):
 class cf_slot(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("base", ctypes.c_void_p), ("err", ctypes.c_void_p),
                 ("cache", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("q0", ctypes.c_void_p), ("U", ctypes.c_void_p), ("R", ctypes.c_void_p), ("V", ctypes.c_void_p)]
+                ("q0", ctypes.c_void_p), ("U", ctypes.c_void_p), ("R", ctypes.c_void_p), ("V", ctypes.c_void_p),
+                ("recon", ctypes.c_void_p)]
 
 
 class CfError(RuntimeError):
@@ -120,12 +121,13 @@ def _parr(ts: Optional[Sequence[Optional[torch.Tensor]]]):
 class Slot:
     """Per-slot tensors for one call (any may be None when a call does not use it)."""
 
-    __slots__ = ("x", "base", "err", "cache", "codes", "scales", "q0", "U", "R", "V")
+    __slots__ = ("x", "base", "err", "cache", "codes", "scales", "q0", "U", "R", "V", "recon")
 
     def __init__(self, x=None, base=None, err=None, cache=None, codes=None, scales=None, q0=None, U=None, R=None,
-                 V=None):
+                 V=None, recon=None):
         self.x, self.base, self.err, self.cache = x, base, err, cache
         self.codes, self.scales, self.q0, self.U, self.R, self.V = codes, scales, q0, U, R, V
+        self.recon = recon
 
     def to_c(self) -> cf_slot:
         return cf_slot(*[_ptr(getattr(self, f)) for f in Slot.__slots__])

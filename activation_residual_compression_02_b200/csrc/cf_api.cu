@@ -138,7 +138,8 @@ cf_status check_quant_slot(cf_ctx *ctx, const cf_slot &s, int i, bool sender, in
             if (!aligned16(s.base) || !aligned16(s.err)) return fail(ctx, CF_E_ALIGN, "slot %d: base/err not 16-byte aligned", i);
         } else {
             if (!s.cache) return fail(ctx, CF_E_ARG, "slot %d: cache is NULL", i);
-            if (!aligned16(s.cache)) return fail(ctx, CF_E_ALIGN, "slot %d: cache not 16-byte aligned", i);
+            if (!aligned16(s.cache) || !aligned16(s.recon))
+                return fail(ctx, CF_E_ALIGN, "slot %d: cache/recon not 16-byte aligned", i);
         }
         return CF_OK;
     }
@@ -149,7 +150,7 @@ cf_status check_quant_slot(cf_ctx *ctx, const cf_slot &s, int i, bool sender, in
             return fail(ctx, CF_E_ALIGN, "slot %d: pointers must be 16-byte aligned", i);
     } else {
         if (!s.codes || !s.scales || !s.cache) return fail(ctx, CF_E_ARG, "slot %d: codes/scales/cache must be non-NULL", i);
-        if (!aligned16(s.codes) || !aligned16(s.scales) || !aligned16(s.cache))
+        if (!aligned16(s.codes) || !aligned16(s.scales) || !aligned16(s.cache) || !aligned16(s.recon))
             return fail(ctx, CF_E_ALIGN, "slot %d: pointers must be 16-byte aligned", i);
     }
     return CF_OK;
@@ -176,6 +177,7 @@ cf_status run_quant(cf_ctx *ctx, const cf_slot *slots, cf::QuantOp op, cudaStrea
             d.cache = s.cache;
             d.codes = s.codes;
             d.scales = s.scales;
+            d.recon = op == cf::QuantOp::Compress || op == cf::QuantOp::WarmupSender ? nullptr : s.recon;
             d.nvec = elems / 8;
         }
         cudaError_t e = cf::launch_quant(op, ctx->cfg.bits, ctx->cfg.group, ctx->cfg.sign_scale, ctx->cfg.state_bf16 != 0,
@@ -214,7 +216,8 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
                 return fail(ctx, CF_E_SHAPE, "slot %d: rows and cols must be >= rank", i);
         } else {
             if (!s.cache) return fail(ctx, CF_E_ARG, "slot %d: cache must be non-NULL", i);
-            if (!aligned16(s.cache)) return fail(ctx, CF_E_ALIGN, "slot %d: cache must be 16-byte aligned", i);
+            if (!aligned16(s.cache) || !aligned16(s.recon))
+                return fail(ctx, CF_E_ALIGN, "slot %d: cache/recon must be 16-byte aligned", i);
         }
     }
     // fp32 residual of every slot, base <- x
@@ -256,6 +259,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
             m.V = slots[k].V;
             m.E = sender ? static_cast<float *>(slots[k].err) : nullptr;
             m.C = sender ? nullptr : static_cast<float *>(slots[k].cache);
+            m.recon = sender ? nullptr : slots[k].recon;
         }
         cf::LowrankPlan plan{};
         plan.nmat = (int)(j - i);

@@ -28,6 +28,7 @@ struct QuantSlotDesc {
     void *cache;       // fp32, or bf16 with the lean state
     uint8_t *codes;    // packed codes
     float *scales;     // fp32 group scales
+    void *recon;       // bf16 copy of the receiver's cache after the call, or null
     int64_t nvec;      // elements / 8
     int64_t tile0;     // first tile index of this slot in the launch (set by launch_quant)
 };
@@ -39,6 +40,7 @@ struct QuantLaunch {
     uint32_t *status;
     QuantSlotDesc slot[kMaxSlotsPerLaunch];
 };
+static_assert(sizeof(QuantLaunch) <= 32764, "a kernel takes at most 32764 bytes of parameters");
 
 enum class QuantOp { WarmupSender, WarmupReceiver, Compress, Decompress, Loopback };
 
@@ -59,6 +61,7 @@ struct LowrankMat {
     float *V;          // [n x r]
     float *E;          // [m x n] or null
     float *C;          // [m x n] or null
+    void *recon;       // bf16 [m x n] or null: bf16(C) after C += D
 };
 
 struct LowrankPlan {

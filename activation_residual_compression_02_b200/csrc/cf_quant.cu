@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
                     float f[8];
                     unpack8(xv[u], f);
                     SV::store(S.cache, v, f);   // bf16 -> fp32 is exact; fp32 -> bf16 of a bf16 value too
+                    if (S.recon) __stcs(static_cast<uint4 *>(S.recon) + v, xv[u]);
                 }
             }
         } else if constexpr (OP == QuantOp::Compress || OP == QuantOp::Loopback) {
@@ -377,6 +378,7 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
 #pragma unroll
                         for (int j = 0; j < 8; ++j) c[j] = __fadd_rn(c[j], d[j]);
                         SV::store(S.cache, v, c);
+                        if (S.recon) StateVec<true>::store(S.recon, v, c);
                     }
                 }
             }
@@ -413,10 +415,12 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
                             d[j] = c ? s : -s;
                     }
                     const float4 a = ca[u], b = cb[u];
-                    __stcs(C + 2 * v, make_float4(__fadd_rn(a.x, d[0]), __fadd_rn(a.y, d[1]),
-                                                  __fadd_rn(a.z, d[2]), __fadd_rn(a.w, d[3])));
-                    __stcs(C + 2 * v + 1, make_float4(__fadd_rn(b.x, d[4]), __fadd_rn(b.y, d[5]),
-                                                      __fadd_rn(b.z, d[6]), __fadd_rn(b.w, d[7])));
+                    const float c[8] = {__fadd_rn(a.x, d[0]), __fadd_rn(a.y, d[1]), __fadd_rn(a.z, d[2]),
+                                        __fadd_rn(a.w, d[3]), __fadd_rn(b.x, d[4]), __fadd_rn(b.y, d[5]),
+                                        __fadd_rn(b.z, d[6]), __fadd_rn(b.w, d[7])};
+                    __stcs(C + 2 * v, make_float4(c[0], c[1], c[2], c[3]));
+                    __stcs(C + 2 * v + 1, make_float4(c[4], c[5], c[6], c[7]));
+                    if (S.recon) StateVec<true>::store(S.recon, v, c);
                 }
             }
         } else {  // Decompress, bf16 cache (lean state)
@@ -454,6 +458,7 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
 #pragma unroll
                     for (int j = 0; j < 8; ++j) c[j] = __fadd_rn(c[j], d[j]);
                     SV::store(S.cache, v, c);
+                    if (S.recon) SV::store(S.recon, v, c);
                 }
             }
         }

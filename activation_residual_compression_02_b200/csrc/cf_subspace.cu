@@ -30,6 +30,7 @@
 // CTA raises an abort flag and a status bit, drains its own TMA loads and
 // MMAs, frees TMEM and returns.
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include <stdlib.h>
 
@@ -591,6 +592,7 @@ struct ApplyMat {
     const float *V;   // [n x r]
     float *E;         // [m x n] or null: E = A - D
     float *C;         // [m x n] or null: C += D
+    void *recon;      // bf16 [m x n] or null: bf16(C) after C += D (only with C)
 };
 
 constexpr int kMaxApplyMats = 192;
@@ -601,9 +603,15 @@ struct ApplyParams {
     int m, n, r;
     int row_tiles, col_tiles;
 };
+static_assert(sizeof(ApplyParams) <= 32764, "a kernel takes at most 32764 bytes of parameters");
 
 template <int CPT>
 struct Vec;
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
 template <> struct Vec<4> {
     using T = float4;
     static __device__ __forceinline__ void load(const float *p, float (&v)[4])
@@ -615,6 +623,12 @@ template <> struct Vec<4> {
     {
         __stcs((float4 *)p, make_float4(v[0], v[1], v[2], v[3]));
     }
+    // bf16, rounded to nearest even, at element offset off of a bf16 array
+    static __device__ __forceinline__ void store_bf16(void *base, int64_t off, const float (&v)[4])
+    {
+        __stcs(reinterpret_cast<uint2 *>(static_cast<uint16_t *>(base) + off),
+               make_uint2(bf16x2_rn(v[0], v[1]), bf16x2_rn(v[2], v[3])));
+    }
 };
 template <> struct Vec<2> {
     static __device__ __forceinline__ void load(const float *p, float (&v)[2])
@@ -625,6 +639,10 @@ template <> struct Vec<2> {
     static __device__ __forceinline__ void store(float *p, const float (&v)[2])
     {
         __stcs((float2 *)p, make_float2(v[0], v[1]));
+    }
+    static __device__ __forceinline__ void store_bf16(void *base, int64_t off, const float (&v)[2])
+    {
+        __stcs(reinterpret_cast<unsigned int *>(static_cast<uint16_t *>(base) + off), bf16x2_rn(v[0], v[1]));
     }
 };
 
@@ -710,6 +728,7 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply(const __grid_constan
 #pragma unroll
                 for (int c = 0; c < CPT; ++c) o[c] = cv[u][c] + d[c];
                 Vec<CPT>::store(M.C + off, o);
+                if (M.recon) Vec<CPT>::store_bf16(M.recon, off, o);
             }
         }
     }
@@ -855,7 +874,9 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply_async(const __grid_c
             }
             if (HAS_C && M.C) {
                 const float4 c = ringC[(slot * RF + u) * kApplyThreads + tid];
-                __stcs((float4 *)(M.C + off), make_float4(c.x + d[0], c.y + d[1], c.z + d[2], c.w + d[3]));
+                const float o[CPT] = {c.x + d[0], c.y + d[1], c.z + d[2], c.w + d[3]};
+                Vec<CPT>::store(M.C + off, o);
+                if (M.recon) Vec<CPT>::store_bf16(M.recon, off, o);
             }
         }
         __syncwarp();
@@ -1074,6 +1095,7 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
             a.V = s.V;
             a.E = sender ? s.E : nullptr;
             a.C = s.C;
+            a.recon = s.C ? s.recon : nullptr;
             has_e = has_e || a.E;
             has_c = has_c || a.C;
         }

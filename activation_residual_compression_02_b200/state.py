@@ -34,7 +34,8 @@ class QuantState:
     err and cache in bf16 (the context's state_bf16 option).
     """
 
-    def __init__(self, shapes: Sequence[Sequence[int]], bits: int, group: int, device="cuda", lean: bool = False):
+    def __init__(self, shapes: Sequence[Sequence[int]], bits: int, group: int, device="cuda", lean: bool = False,
+                 recon: bool = False):
         self.shapes = [tuple(s) for s in shapes]
         self.bits, self.group, self.lean = bits, group, lean
         n = [r * c for r, c in self.shapes]
@@ -48,6 +49,9 @@ class QuantState:
         self.base = [v[:k] for v, k in zip(_split(self.base_all, nb), n)]
         self.err = [v[:k] for v, k in zip(_split(self.err_all, nf), n)]
         self.cache = [v[:k] for v, k in zip(_split(self.cache_all, nf), n)]
+        # optional bf16 copy of each cache, written by the receiver calls
+        self.recon_all = torch.empty(sum(nb), dtype=torch.bfloat16, device=device) if recon else None
+        self.recon = [v[:k] for v, k in zip(_split(self.recon_all, nb), n)] if recon else [None] * len(n)
         self.codes_all, self.codes, self.scales_all, self.scales = self.payload_buffers(device)
 
     def payload_buffers(self, device="cuda", pin: bool = False):
@@ -73,8 +77,8 @@ class QuantState:
               scales: Optional[Sequence[torch.Tensor]] = None) -> List[Slot]:
         codes = self.codes if codes is None else codes
         scales = self.scales if scales is None else scales
-        return [Slot(x=x.reshape(-1), base=b, err=e, cache=c, codes=k, scales=s)
-                for x, b, e, c, k, s in zip(xs, self.base, self.err, self.cache, codes, scales)]
+        return [Slot(x=x.reshape(-1), base=b, err=e, cache=c, codes=k, scales=s, recon=rc)
+                for x, b, e, c, k, s, rc in zip(xs, self.base, self.err, self.cache, codes, scales, self.recon)]
 
 
 def alloc_quant_state(shapes, bits, group, device="cuda") -> QuantState:

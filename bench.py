@@ -348,6 +348,52 @@ def run_cf(args, w):
               "note": "cf_loopback: compress and decompress of a step in one launch (both sides on this GPU)"}
     comp_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     deco_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+
+    # ---- receiver with the bf16 reconstruction (recon), same payload ------
+    # The decompress of the last timed step again, K times, with every slot's
+    # recon set; beside it the same decompress followed by torch's fp32 -> bf16
+    # cast of the caches (the separate pass recon replaces).
+    rc = None
+    if not args.no_recon:
+        last = (args.warmup + args.steps - 1) % len(c_slots)
+        recon_all = torch.empty(st.cache_all.numel(), dtype=torch.bfloat16, device=dev)
+        r_list = st.slots(x_at(last + 1))
+        for sl_, c_ in zip(r_list, st.cache):
+            # recon of a slot at its cache's element offset (16-byte aligned: cols % 8 == 0)
+            o = c_.storage_offset() - st.cache_all.storage_offset()
+            sl_.recon = recon_all[o:o + c_.numel()]
+        r_arr = ctx._slots(r_list)
+        i_dec = args.warmup + args.steps
+
+        def deco(arr):
+            if L.cf_decompress(h, arr, i_dec, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+
+        for _ in range(args.warmup):
+            deco(r_arr)
+        barrier(world)
+        torch.cuda.synchronize()
+        r0, r1, r2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        r0.record(stream)
+        for _ in range(args.steps):
+            deco(r_arr)
+        r1.record(stream)
+        for _ in range(args.steps):
+            deco(c_slots[last])
+            recon_all.copy_(st.cache_all)
+        r2.record(stream)
+        torch.cuda.synchronize()
+        if ctx.check() != 0:
+            raise RuntimeError("device status in the recon run")
+        r_ms = max_over_ranks(r0.elapsed_time(r1), world) / args.steps
+        cast_ms = max_over_ranks(r1.elapsed_time(r2), world) / args.steps
+        _, bd_ = alg_bytes_per_elem(w.bits, w.group)
+        r_bytes = (bd_ + 2) * n_elem
+        rc = {"ms_per_launch": r_ms, "alg_bytes_per_launch": r_bytes, "achieved": r_bytes / (r_ms * 1e-3) / 1e9,
+              "frac": r_bytes / (r_ms * 1e-3) / 1e9 / hbm_peak()[0], "decompress_then_cast_ms": cast_ms,
+              "note": "cf_decompress with recon: C += deq and recon = bf16(C) in one pass (bd + 2 B/elt); "
+                      "decompress_then_cast_ms: the same decompress followed by torch's cast of C to bf16"}
+        del recon_all, r_arr, r_list
     ms_per_step = ms / args.steps
     value = world * x_bytes / (ms_per_step * 1e-3) / 1e9
 
@@ -471,7 +517,7 @@ def run_cf(args, w):
                                 "alg_bytes_per_launch": bd * n_elem, "ms_per_launch": deco_ms},
         "roofline_step": {"achieved": ach_pair, "frac": ach_pair / peak, "frac_of_8tbs": ach_pair / 8000.0,
                           "alg_bytes_per_step": (bc + bd) * n_elem},
-        "loopback": lb, "lean_state": lean,
+        "loopback": lb, "lean_state": lean, "recon": rc,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
@@ -594,6 +640,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-loopback", action="store_true")
     ap.add_argument("--no-lean", action="store_true")
+    ap.add_argument("--no-recon", action="store_true")
     ap.add_argument("--warm-start", action="store_true", help="low-rank: T = 1 from the previous call's V")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -124,6 +124,8 @@ typedef struct cf_slot {
     float *U;        /* low-rank payload [rows x r] */
     float *R;        /* low-rank payload [r x r] */
     float *V;        /* low-rank payload [cols x r] */
+    void *recon;     /* bf16 [rows*cols] or NULL: receiver output, bf16(cache) after the call
+                        (see cf_decompress) */
 } cf_slot;
 
 /* Create a context for `nslots` slots of the given shapes (host array).
@@ -162,7 +164,13 @@ cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
  *   step >= 1, quantised: cache += deq(codes, scales).  Uses codes, scales,
  *           cache.
  *   step >= 1, low-rank: cache += U R V^T.  Uses U, R, V, cache.
- * Errors as cf_compress (CF_E_STATE: step >= 1 before a receiver warmup). */
+ * A slot whose recon is non-NULL also gets recon = bf16(cache) after the
+ * update, rounded to nearest even (at step 0 that is x itself), from the same
+ * pass: 2 more bytes per element, where a separate cast would read the fp32
+ * cache back (4) and write bf16 (2).  It is meant for the consumer of a
+ * received K or V, which reads bf16.  The same holds for cf_loopback.
+ * Errors as cf_compress (CF_E_STATE: step >= 1 before a receiver warmup;
+ * CF_E_ALIGN: recon not 16-byte aligned). */
 cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
 
 /* Sender and receiver of step `step` in one pass, for when both sides of a

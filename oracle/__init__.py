@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         _lib.cfo_warmup_receiver_lean.argtypes = [I64, P, P]
         _lib.cfo_compress_lean.argtypes = [I64, I, I, I, P, P, P, P, P, U32P]
         _lib.cfo_decompress_lean.argtypes = [I64, I, I, P, P, P]
+        _lib.cfo_to_bf16.argtypes = [I64, P, P]
     return _lib
 
 
@@ -148,6 +149,14 @@ def decompress(codes: np.ndarray, scales: np.ndarray, cache: np.ndarray, bits: i
                                 _ptr(np.ascontiguousarray(scales)), _ptr(cache)), "decompress")
 
 
+def to_bf16(f: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 (raw 16-bit patterns), round to nearest even."""
+    f = np.ascontiguousarray(f, dtype=np.float32).ravel()
+    out = np.empty(f.size, np.uint16)
+    _check(lib().cfo_to_bf16(f.size, _ptr(f), _ptr(out)), "to_bf16")
+    return out
+
+
 def put_code(stream: np.ndarray, i: int, bits: int, code: int) -> None:
     _check(lib().cfo_put_code(_ptr(stream), i, bits, code), "put_code")
 
@@ -190,6 +199,11 @@ class QuantSlot:
         self.base = self.err = self.cache = None
         self.codes = self.scales = None
         self.flags = 0
+
+    @property
+    def recon(self) -> np.ndarray:
+        """The receiver's reconstruction in bf16 (raw bits): bf16(C) after the last step."""
+        return self.cache.copy() if self.lean else to_bf16(self.cache)
 
     def step(self, t: int, x_bits: np.ndarray) -> None:
         if self.lean:

@@ -69,6 +69,15 @@ static uint16_t float_to_bf16(float f)
     return (uint16_t)((u + 0x7fffu + lsb) >> 16);
 }
 
+/* bf16 copy of the receiver's reconstruction, for a consumer that reads K or
+ * V in bf16: out[i] = float_to_bf16(in[i]). */
+int cfo_to_bf16(int64_t n, const float *in, uint16_t *out)
+{
+    if (n < 0 || (n > 0 && (!in || !out))) return CFO_E_ARG;
+    for (int64_t i = 0; i < n; ++i) out[i] = float_to_bf16(in[i]);
+    return CFO_OK;
+}
+
 /* ------------------------------------------------------- bit stream ----- */
 
 /* The payload is one bit stream per slot, bytes in increasing address order,

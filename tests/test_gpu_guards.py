@@ -56,7 +56,8 @@ def test_quantised_kernels_write_only_their_buffers(cf, bits, group, lean, loopb
     for r, c in shapes:
         n = r * c
         bufs.append(dict(base=Guarded(n, torch.bfloat16), err=Guarded(n, sdt), cache=Guarded(n, sdt),
-                         codes=Guarded(n * bits // 8, torch.uint8), scales=Guarded(n // group, torch.float32)))
+                         codes=Guarded(n * bits // 8, torch.uint8), scales=Guarded(n // group, torch.float32),
+                         recon=Guarded(n, torch.bfloat16)))
     streams = [synth.SlotStream(synth.FLUX.scaled(rows=r, cols=c), slot=i) for i, (r, c) in enumerate(shapes)]
     for t in range(3):
         xs = [s.next().cuda().reshape(-1) for s in streams]

@@ -174,7 +174,12 @@ def test_lowrank_full_size_sampled(cf, oracle):
 
 def test_lowrank_mode_through_slots(cf, oracle):
     """cf_compress / cf_decompress in low-rank mode: residual + error feedback
-    into Algorithm 3, E and the receiver cache updated, base advanced."""
+    into Algorithm 3, E and the receiver cache updated, base advanced.  The
+    oracle runs its own chain (its own fp32 E carried between steps); the two
+    chains agree within the low-rank tolerance at every step.  The receiver
+    also writes the bf16 reconstruction: torch's round-to-nearest-even cast of
+    the cache it wrote, and within the tolerance plus one bf16 rounding
+    (2^-8 relative) of the oracle's cache."""
     rows, cols, r, T = 192, 256, 16, 2
     shapes = [(rows, cols), (rows, cols)]
     ctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
@@ -197,13 +202,14 @@ def test_lowrank_mode_through_slots(cf, oracle):
     U = [torch.empty(rows, r, device="cuda") for _ in shapes]
     R = [torch.empty(r, r, device="cuda") for _ in shapes]
     V = [torch.empty(cols, r, device="cuda") for _ in shapes]
+    recon = [torch.empty(rows * cols, dtype=torch.bfloat16, device="cuda") for _ in shapes]
     ob = [None, None]
     oe = [None, None]
     oc = [None, None]
     for t in range(3):
         q0 = [synth.q0(cols, r, seed=0, mat=i, call=t) for i in range(2)]
         slots = [cf.Slot(x=xs[i][t].reshape(-1).cuda(), base=base[i], err=err[i], cache=cache[i], q0=q0[i].cuda(),
-                         U=U[i], R=R[i], V=V[i]) for i in range(2)]
+                         U=U[i], R=R[i], V=V[i], recon=recon[i]) for i in range(2)]
         ctx.compress(slots, t)
         ctx.decompress(slots, t)
         for i in range(2):
@@ -221,8 +227,10 @@ def test_lowrank_mode_through_slots(cf, oracle):
             oc[i] = oc[i] + Do.ravel()
             assert rel(cache[i].cpu().double().numpy(), oc[i], Do) <= TOL, (t, i)
             assert np.array_equal(base[i].view(torch.int16).cpu().numpy().view(np.uint16), xb)
-            # continue the oracle from the GPU's error buffer (E is unique only to 1e-3)
-            oe[i] = err[i].cpu().numpy().copy()
+            cg = cache[i].cpu()
+            assert torch.equal(recon[i].cpu(), cg.to(torch.bfloat16)), (t, i)
+            assert rel(recon[i].cpu().double().numpy(), oc[i], oc[i]) <= TOL + 2.0 ** -8, (t, i)
+            oe[i] = Eo.ravel().astype(np.float32)     # the oracle's E buffer is fp32, as the codec's
     assert ctx.check() == cf.CF_OK
     for i in range(2):
         x = xs[i][2].float().reshape(-1).cuda()
@@ -231,8 +239,10 @@ def test_lowrank_mode_through_slots(cf, oracle):
 
 def test_lowrank_warm_start_through_slots(cf, oracle):
     """warm_start: from the second compressed step on, Algorithm 3 starts from
-    the previous step's V (T = 1 here).  Each step matches the oracle run from
-    the same start block, and the error feedback keeps C + E = X."""
+    the previous step's V (T = 1 here).  The oracle runs the same warm-started
+    chain from its own V and E (both kept in fp32, as the codec keeps them);
+    every step agrees within the tolerance, and the error feedback keeps
+    C + E = X."""
     rows, cols, r, T = 192, 256, 16, 1
     shapes = [(rows, cols)]
     ctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T, warm_start=1)
@@ -253,9 +263,9 @@ def test_lowrank_warm_start_through_slots(cf, oracle):
     cache = torch.empty(rows * cols, device="cuda")
     U, R, V = torch.empty(rows, r, device="cuda"), torch.empty(r, r, device="cuda"), torch.empty(cols, r, device="cuda")
     q0 = synth.q0(cols, r, seed=0, mat=7).cuda()
-    ob = oe = None
+    ob = oe = ov = None
     for t, xt in enumerate(seq):
-        start = q0 if t <= 1 else V.clone()
+        start = q0.cpu().numpy() if t <= 1 else ov
         slot = cf.Slot(x=xt.reshape(-1).cuda(), base=base, err=err, cache=cache, q0=q0 if t <= 1 else None,
                        U=U, R=R, V=V)
         ctx.compress([slot], t)
@@ -265,12 +275,13 @@ def test_lowrank_warm_start_through_slots(cf, oracle):
             ob, oe = oracle.warmup_sender(xb)
             continue
         a = oracle.residual(xb, ob, oe).reshape(rows, cols)
-        Uo, Ro, Vo = oracle.subspace_iteration(a, start.cpu().numpy(), T)
+        Uo, Ro, Vo = oracle.subspace_iteration(a, start, T)
         Do, Eo, _ = oracle.lowrank_apply(a, Uo, Ro, Vo)
         torch.cuda.synchronize()
         eg = err.cpu().double().numpy().reshape(rows, cols)
         assert rel(eg, Eo, Do) <= TOL, t
-        oe = err.cpu().numpy().copy()
+        oe = Eo.ravel().astype(np.float32)
+        ov = Vo.astype(np.float32)
     assert ctx.check() == cf.CF_OK
     xl = seq[-1].float().reshape(-1).cuda()
     assert (torch.linalg.vector_norm(cache + err - xl) / torch.linalg.vector_norm(xl)).item() < 1e-5

@@ -28,10 +28,10 @@ def u16(t):
 
 
 def run_case(cf, oracle, shapes, steps, bits, group, ss=0, seed=0, w=synth.TINY, check_every_step=True,
-             loopback=False):
+             loopback=False, recon=False):
     """Run the codec on the GPU and the oracle on the CPU for `steps` steps."""
     ctx = cf.Context(shapes, bits=bits, group=group, sign_scale=ss)
-    st = cf.QuantState(shapes, bits, group)
+    st = cf.QuantState(shapes, bits, group, recon=recon)
     streams = [synth.SlotStream(w.scaled(rows=r, cols=c), slot=i, seed=seed) for i, (r, c) in enumerate(shapes)]
     ors = [oracle.QuantSlot(bits, group, ss) for _ in shapes]
     for t in range(steps):
@@ -52,6 +52,8 @@ def run_case(cf, oracle, shapes, steps, bits, group, ss=0, seed=0, w=synth.TINY,
                 assert np.array_equal(u16(st.base[i]), o.base), (t, i, "base")
                 assert np.array_equal(st.err[i].cpu().numpy(), o.err), (t, i, "err")
                 assert np.array_equal(st.cache[i].cpu().numpy(), o.cache), (t, i, "cache")
+                if recon:
+                    assert np.array_equal(u16(st.recon[i]), o.recon), (t, i, "recon")
                 if t > 0:
                     assert np.array_equal(st.codes[i].cpu().numpy(), o.codes), (t, i, "codes")
                     assert np.array_equal(st.scales[i].cpu().numpy(), o.scales), (t, i, "scales")
@@ -262,9 +264,9 @@ def test_host_stream_codec_matches_oracle(cf, oracle):
         assert np.array_equal(hc.st.err[i].cpu().numpy(), ors[i].err)
 
 
-def run_lean(cf, oracle, shapes, steps, bits, group, ss=0, loopback=False, w=synth.FLUX):
+def run_lean(cf, oracle, shapes, steps, bits, group, ss=0, loopback=False, w=synth.FLUX, recon=False):
     ctx = cf.Context(shapes, bits=bits, group=group, sign_scale=ss, state_bf16=1)
-    st = cf.QuantState(shapes, bits, group, lean=True)
+    st = cf.QuantState(shapes, bits, group, lean=True, recon=recon)
     streams = [synth.SlotStream(w.scaled(rows=r, cols=c), slot=i) for i, (r, c) in enumerate(shapes)]
     ors = [oracle.QuantSlot(bits, group, ss, lean=True) for _ in shapes]
     for t in range(steps):
@@ -283,6 +285,8 @@ def run_lean(cf, oracle, shapes, steps, bits, group, ss=0, loopback=False, w=syn
             assert np.array_equal(u16(st.err[i]), o.err), (t, i, "err")
             assert np.array_equal(u16(st.cache[i]), o.cache), (t, i, "cache")
             assert np.array_equal(u16(st.base[i]), o.base), (t, i, "base")
+            if recon:
+                assert np.array_equal(u16(st.recon[i]), o.recon), (t, i, "recon")
             if t > 0:
                 assert np.array_equal(st.codes[i].cpu().numpy(), o.codes), (t, i, "codes")
                 assert np.array_equal(st.scales[i].cpu().numpy(), o.scales), (t, i, "scales")
@@ -303,3 +307,52 @@ def test_lean_state_rejected_in_lowrank_mode(cf):
     with pytest.raises(cf.CfError) as e:
         cf.Context([(64, 64)], mode=cf.CF_MODE_LOWRANK, rank=4, iters=1, state_bf16=1)
     assert e.value.status == cf.CF_E_ARG
+
+
+@pytest.mark.parametrize("bits,group", [(2, 128), (4, 64), (1, 128), (2, 8)])
+@pytest.mark.parametrize("lean,loopback", [(False, False), (False, True), (True, False), (True, True)])
+def test_bf16_reconstruction_bit_exact(cf, oracle, bits, group, lean, loopback):
+    """With a recon buffer the receiver also writes bf16(C) (RNE) from the same
+    pass: equal to the oracle's rounding of its own C at every step (X_0 at the
+    warmup), and C, E, codes and scales unchanged by it."""
+    shapes = [(37, 512), (1, 256), (0, 256), (129, 768)]
+    shapes = [(r, c) for r, c in shapes if c % group == 0]
+    if lean:
+        run_lean(cf, oracle, shapes, 4, bits, group, loopback=loopback, recon=True)
+    else:
+        run_case(cf, oracle, shapes, 4, bits, group, w=synth.FLUX, loopback=loopback, recon=True)
+
+
+def test_bf16_reconstruction_only_where_asked(cf, oracle):
+    """recon is per slot and per call: slot 1 gets a recon buffer at steps 0
+    and 1 only, so afterwards it holds the step-1 reconstruction while slot 0's
+    follows every step; a misaligned recon is refused before any launch."""
+    shapes = [(64, 512), (32, 256)]
+    ctx = cf.Context(shapes, bits=2, group=128)
+    st = cf.QuantState(shapes, 2, 128, recon=True)
+    streams = [synth.SlotStream(synth.FLUX.scaled(rows=r, cols=c), slot=i) for i, (r, c) in enumerate(shapes)]
+    ors = [oracle.QuantSlot(2, 128) for _ in shapes]
+    side = torch.empty(32 * 256, dtype=torch.bfloat16, device="cuda")
+    expect_side = None
+    for t in range(3):
+        xs = [s.next() for s in streams]
+        slots = st.slots([x.cuda() for x in xs])
+        slots[1].recon = side if t < 2 else None
+        ctx.compress(slots, t)
+        if t == 2:
+            bad = torch.empty(64 * 512 + 8, dtype=torch.bfloat16, device="cuda")
+            slots[0].recon = bad[1:1 + 64 * 512]
+            with pytest.raises(cf.CfError) as e:
+                ctx.decompress(slots, t)
+            assert e.value.status == cf.CF_E_ALIGN
+            slots[0].recon = st.recon[0]
+        ctx.decompress(slots, t)
+        for i, x in enumerate(xs):
+            ors[i].step(t, u16(x))
+        if t == 1:
+            expect_side = ors[1].recon
+    torch.cuda.synchronize()
+    assert ctx.check() == cf.CF_OK
+    assert np.array_equal(u16(st.recon[0]), ors[0].recon)
+    assert np.array_equal(st.cache[1].cpu().numpy(), ors[1].cache)
+    assert np.array_equal(u16(side), expect_side)

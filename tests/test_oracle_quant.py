@@ -324,3 +324,56 @@ def test_lean_state_error_feedback_identity(oracle):
         rec = _bits_to_f32(st.cache).astype(np.float64) + _bits_to_f32(st.err).astype(np.float64)
         rel = np.linalg.norm(rec - x64) / np.linalg.norm(x64)
         assert rel <= (t + 1) * 2.0 ** -9, (t, rel)
+
+
+@pytest.mark.parametrize("bits_in,bits_out", [
+    (0x3F800000, 0x3F80),   # 1.0
+    (0x3F808000, 0x3F80),   # 1 + 2^-8: halfway, the even neighbour is 1.0
+    (0x3F818000, 0x3F82),   # 1 + 3*2^-8: halfway, the even neighbour is above
+    (0x3F808001, 0x3F81),   # just above halfway rounds up
+    (0x3F80FFFF, 0x3F81),
+    (0xC0200000, 0xC020),   # -2.5, exact
+    (0x80000000, 0x8000),   # -0 keeps its sign
+    (0x7F7FFFFF, 0x7F80),   # the largest float rounds to +inf
+    (0x7F800000, 0x7F80),   # +inf
+    (0xFF800000, 0xFF80),   # -inf
+    (0x00008000, 0x0000),   # subnormal halfway, even neighbour 0
+    (0x00018000, 0x0002),   # subnormal halfway, even neighbour above
+    (0x7FC00000, 0x7FC0),   # quiet NaN
+    (0x7F800001, 0x7FC0),   # signalling NaN comes out quiet
+])
+def test_bf16_rounding_hand_values(oracle, bits_in, bits_out):
+    """The receiver's bf16 reconstruction rounds to nearest even: hand-checked
+    bit patterns, ties both ways, overflow, signed zero, subnormals, NaN."""
+    f = np.array([bits_in], np.uint32).view(np.float32)
+    assert int(oracle.to_bf16(f)[0]) == bits_out
+
+
+def test_bf16_rounding_matches_torch(oracle):
+    """Against torch's own float -> bfloat16 conversion (round to nearest even)
+    on 2^20 finite floats spread over every exponent."""
+    rng = np.random.default_rng(5)
+    u = rng.integers(0, 2 ** 32, size=1 << 20, dtype=np.uint64).astype(np.uint32)
+    f = u.view(np.float32)
+    f = f[np.isfinite(f)]
+    want = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.to_bf16(f), want)
+
+
+def test_bf16_reconstruction_of_a_slot(oracle):
+    """QuantSlot.recon is the warmup activation itself at step 0 and the
+    rounding of the fp32 cache afterwards; with the lean state it is the
+    cache."""
+    w = synth.FLUX.scaled(rows=8, cols=256)
+    xs = synth.activations(w, 0, 3)
+    s32 = oracle.QuantSlot(2, 128)
+    s16 = oracle.QuantSlot(2, 128, lean=True)
+    for t, x in enumerate(xs):
+        xb = synth.bf16_bits(x).numpy().view(np.uint16).ravel().copy()
+        s32.step(t, xb)
+        s16.step(t, xb)
+        if t == 0:
+            assert np.array_equal(s32.recon, xb)
+            assert np.array_equal(s16.recon, xb)
+        assert np.array_equal(s32.recon, oracle.to_bf16(s32.cache))
+        assert np.array_equal(s16.recon, s16.cache)
