@@ -36,14 +36,17 @@ namespace {
 // per code width k): threads per CTA, vectors (of 8 elements) each thread
 // keeps in flight (a tile is threads * unroll vectors), and a cap on resident
 // CTAs per SM (0: as many as fit).  Chosen by sweeps on the B200 over
-// 128..1024 threads, 1..16 vectors and 1..4 CTAs per SM on the 57-slot
-// FLUX-shaped (k = 2), 30-slot CogVideoX-shaped (k = 4) and 60-slot stress
-// (k = 1) steps, as a fraction of the measured copy bandwidth:
-//   compress   k = 2: 256 x 8 at 1 CTA/SM, 95.3% (1024 x 1: 93.4%)
-//              k = 4: 512 x 2, 94.0% (1024 x 1: 89.5%; 256 x 8: 91.4%)
-//              k = 1: 512 x 2, 93.3% (1024 x 1: 89.3%)
-//   decompress k = 2, 4: 512 x 4 at 1 CTA/SM, 94.5% / 93.1% (256 x 8: 90.1% / 92.1%)
-//              k = 1: 256 x 8, 98.9% (512 x 4: 89.1%)
+// 128..1024 threads (in steps of one or two warps near the optimum), 1..16
+// vectors and 1..4 CTAs per SM on the 57-slot FLUX-shaped (k = 2), 30-slot
+// CogVideoX-shaped (k = 4) and 60-slot stress (k = 1) steps, as a fraction
+// of the measured copy bandwidth:
+//   compress   k = 2: 256 x 8 at 1 CTA/SM, 95.2% (1024 x 1: 93.4%; 224 x 8: 90.1%;
+//                     288 x 8: 86.6%; 256 x 7: 94.3%)
+//              k = 4: 512 x 2, 94.0% (1024 x 1: 89.5%; 256 x 8: 91.4%; 256 x 6: 94.1%)
+//              k = 1: 512 x 2, 93.3% (1024 x 1: 89.3%; 256 x 7: 91.3%)
+//   decompress k = 2, 4: 448 x 4 at 1 CTA/SM, 98.9% / 97.5% (512 x 4: 94.9% / 93.5%;
+//                     416 x 4: 97.2% / 97.2%; 480 x 4: 98.4% / 95.2%; 448 x 5: 94.1% / 92.4%)
+//              k = 1: 256 x 8, 98.9% (512 x 4: 89.1%; 448 x 4: 95.6%)
 // More resident CTAs per SM, i.e. more concurrent streams into HBM, were
 // slower in every case.
 template <QuantOp OP, bool LEAN = false>
@@ -61,13 +64,13 @@ struct QShapeBase<QuantOp::Compress, false> {
 template <>
 struct QShapeBase<QuantOp::Loopback, false> {
     // fused sender + receiver (9 streams per tile); per-width shapes below
-    static constexpr int kThreads = 256;
-    static constexpr int kUnroll = 4;
+    static constexpr int kThreads = 384;
+    static constexpr int kUnroll = 3;
     static constexpr int kMaxPerSm = 1;
 };
 template <>
 struct QShapeBase<QuantOp::Decompress, false> {
-    static constexpr int kThreads = 512;
+    static constexpr int kThreads = 448;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 1;
 };
@@ -85,9 +88,11 @@ struct QShapeBase<QuantOp::Loopback, true> {
     static constexpr int kUnroll = 8;
     static constexpr int kMaxPerSm = 1;
 };
+// (896 x 4: 95.1% / 95.1% / 97.3% on the k = 2 / 4 / 1 steps; 1024 x 4: 95.1% /
+// 90.7% / 91.4%; 640 x 6: 91.5% / 94.8% / 96.7%)
 template <>
 struct QShapeBase<QuantOp::Decompress, true> {
-    static constexpr int kThreads = 1024;
+    static constexpr int kThreads = 896;
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 1;
 };
@@ -107,24 +112,34 @@ template <>
 struct QShape<QuantOp::Compress, false, 1> : QShapeOne<512, 2> {};
 template <>
 struct QShape<QuantOp::Decompress, false, 1> : QShapeOne<256, 8> {};
-// Loopback (sender and receiver of a step in one kernel): 256 x 4 for k = 2
-// (94.96%, faster than the separate pair), 320 x 4 for k = 4 (91.0%), 256 x 6
-// for k = 1 (92.7%); the shape is sensitive (256 x 3: 79.7% for k = 2).
-template <>
-struct QShape<QuantOp::Loopback, false, 4> : QShapeOne<320, 4> {};
+// Loopback (sender and receiver of a step in one kernel): 384 x 3 for k = 2
+// and k = 4 (95.4% / 93.4%; 256 x 4: 94.9% / 89.8%; 320 x 4: 93.7% / 91.1%;
+// 448 x 3: 91.1% / 88.7%), 256 x 6 for k = 1 (92.7%; 384 x 3: 92.1%); the
+// shape is sensitive (256 x 3: 79.7% for k = 2).
 template <>
 struct QShape<QuantOp::Loopback, false, 1> : QShapeOne<256, 6> {};
-// Lean-state sender (bf16 E): 1024 x 2 stays best for k = 2 (91.3%); k = 4 and
-// k = 1 want more vectors per thread: 512 x 4 (88.4 -> 91.4%) and 256 x 16
-// (87.8 -> 91.5%), steps of the CogVideoX-shaped and stress workloads.
+// Lean-state sender (bf16 E): 1024 x 2 stays best for k = 2 (88.1%; 448 x 4:
+// 87.7%; 512 x 4: 85.9%); k = 4 and k = 1 want more vectors per thread:
+// 384 x 6 (1024 x 2: 86.6%; 512 x 4: 90.4%; 384 x 6: 91.6%) and 256 x 16
+// (1024 x 2: 86.2%; 256 x 16: 91.5%; 384 x 6: 90.8%), steps of the
+// CogVideoX-shaped and stress workloads.
 template <>
-struct QShape<QuantOp::Compress, true, 4> : QShapeOne<512, 4> {};
+struct QShape<QuantOp::Compress, true, 4> : QShapeOne<384, 6> {};
 template <>
 struct QShape<QuantOp::Compress, true, 1> : QShapeOne<256, 16> {};
-template <QuantOp OP, bool LEAN, int K>
+// Receivers that also write the bf16 reconstruction (RC): one more output
+// stream per vector.  The fp32-state receiver with recon runs 384 x 4 (sweep
+// on the FLUX- and CogVideoX-shaped steps: 99.0% / 97.8% of the copy
+// bandwidth for its 10.28 / 10.56 bytes per element; 512 x 4: 85.1% / 84.2%,
+// 256 x 8: 98.6% / 96.5%).
+template <QuantOp OP, bool LEAN, int K, bool RC>
+struct QShapeR : QShape<OP, LEAN, K> {};
+template <int K>
+struct QShapeR<QuantOp::Decompress, false, K, true> : QShapeOne<384, 4> {};
+template <QuantOp OP, bool LEAN, int K, bool RC>
 constexpr int64_t qtile_vec()
 {
-    return (int64_t)QShape<OP, LEAN, K>::kThreads * QShape<OP, LEAN, K>::kUnroll;
+    return (int64_t)QShapeR<OP, LEAN, K, RC>::kThreads * QShapeR<OP, LEAN, K, RC>::kUnroll;
 }
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kAbsMask = 0x7fffffffu;
@@ -240,12 +255,15 @@ __device__ __forceinline__ float group_scale(const float (&a)[8], bool &nonfinit
     }
 }
 
-template <QuantOp OP, int K, int G, int SS, bool LEAN>
-__global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
+// RC: the receiver part also writes recon = bf16(C) for every slot whose
+// recon pointer is set (instances without RC never touch recon, apart from
+// the warmup receiver, which checks the pointer).
+template <QuantOp OP, int K, int G, int SS, bool LEAN, bool RC>
+__global__ void __launch_bounds__(QShapeR<OP, LEAN, K, RC>::kThreads) k_quant(const __grid_constant__ QuantLaunch p)
 {
     using SV = StateVec<LEAN>;
-    constexpr int kThreads = QShape<OP, LEAN, K>::kThreads;
-    constexpr int kUnroll = QShape<OP, LEAN, K>::kUnroll;
+    constexpr int kThreads = QShapeR<OP, LEAN, K, RC>::kThreads;
+    constexpr int kUnroll = QShapeR<OP, LEAN, K, RC>::kUnroll;
     constexpr int kTileVec = kThreads * kUnroll;
     constexpr int LPG = G / 8;
     constexpr int L = (K >= 2) ? (1 << (K - 1)) - 1 : 1;
@@ -378,7 +396,7 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
 #pragma unroll
                         for (int j = 0; j < 8; ++j) c[j] = __fadd_rn(c[j], d[j]);
                         SV::store(S.cache, v, c);
-                        if (S.recon) StateVec<true>::store(S.recon, v, c);
+                        if (RC && S.recon) StateVec<true>::store(S.recon, v, c);
                     }
                 }
             }
@@ -420,7 +438,7 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
                                         __fadd_rn(b.z, d[6]), __fadd_rn(b.w, d[7])};
                     __stcs(C + 2 * v, make_float4(c[0], c[1], c[2], c[3]));
                     __stcs(C + 2 * v + 1, make_float4(c[4], c[5], c[6], c[7]));
-                    if (S.recon) StateVec<true>::store(S.recon, v, c);
+                    if (RC && S.recon) StateVec<true>::store(S.recon, v, c);
                 }
             }
         } else {  // Decompress, bf16 cache (lean state)
@@ -458,7 +476,7 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
 #pragma unroll
                     for (int j = 0; j < 8; ++j) c[j] = __fadd_rn(c[j], d[j]);
                     SV::store(S.cache, v, c);
-                    if (S.recon) SV::store(S.recon, v, c);
+                    if (RC && S.recon) SV::store(S.recon, v, c);
                 }
             }
         }
@@ -467,42 +485,46 @@ __global__ void __launch_bounds__(QShape<OP, LEAN, K>::kThreads) k_quant(const _
 
 using KernelFn = void (*)(QuantLaunch);
 
-template <QuantOp OP, int K, int SS, bool LEAN>
+template <QuantOp OP, int K, int SS, bool LEAN, bool RC>
 KernelFn pick_group(int group)
 {
     switch (group) {
-    case 8: return k_quant<OP, K, 8, SS, LEAN>;
-    case 16: return k_quant<OP, K, 16, SS, LEAN>;
-    case 32: return k_quant<OP, K, 32, SS, LEAN>;
-    case 64: return k_quant<OP, K, 64, SS, LEAN>;
-    case 128: return k_quant<OP, K, 128, SS, LEAN>;
-    case 256: return k_quant<OP, K, 256, SS, LEAN>;
+    case 8: return k_quant<OP, K, 8, SS, LEAN, RC>;
+    case 16: return k_quant<OP, K, 16, SS, LEAN, RC>;
+    case 32: return k_quant<OP, K, 32, SS, LEAN, RC>;
+    case 64: return k_quant<OP, K, 64, SS, LEAN, RC>;
+    case 128: return k_quant<OP, K, 128, SS, LEAN, RC>;
+    case 256: return k_quant<OP, K, 256, SS, LEAN, RC>;
     default: return nullptr;
     }
 }
 
-template <QuantOp OP, bool LEAN>
+template <QuantOp OP, bool LEAN, bool RC>
 KernelFn pick_bits(int bits, int group, int ss)
 {
     if (bits == 1) {
         if constexpr (OP == QuantOp::Compress || OP == QuantOp::Loopback)
-            if (ss) return pick_group<OP, 1, 1, LEAN>(group);
-        return pick_group<OP, 1, 0, LEAN>(group);
+            if (ss) return pick_group<OP, 1, 1, LEAN, RC>(group);
+        return pick_group<OP, 1, 0, LEAN, RC>(group);
     }
-    if (bits == 2) return pick_group<OP, 2, 0, LEAN>(group);
-    if (bits == 4) return pick_group<OP, 4, 0, LEAN>(group);
+    if (bits == 2) return pick_group<OP, 2, 0, LEAN, RC>(group);
+    if (bits == 4) return pick_group<OP, 4, 0, LEAN, RC>(group);
     return nullptr;
 }
 
 template <bool LEAN>
-KernelFn pick(QuantOp op, int bits, int group, int ss)
+KernelFn pick(QuantOp op, int bits, int group, int ss, bool rc)
 {
     switch (op) {
-    case QuantOp::WarmupSender: return k_quant<QuantOp::WarmupSender, 2, 8, 0, LEAN>;
-    case QuantOp::WarmupReceiver: return k_quant<QuantOp::WarmupReceiver, 2, 8, 0, LEAN>;
-    case QuantOp::Compress: return pick_bits<QuantOp::Compress, LEAN>(bits, group, ss);
-    case QuantOp::Decompress: return pick_bits<QuantOp::Decompress, LEAN>(bits, group, ss);
-    case QuantOp::Loopback: return pick_bits<QuantOp::Loopback, LEAN>(bits, group, ss);
+    case QuantOp::WarmupSender: return k_quant<QuantOp::WarmupSender, 2, 8, 0, LEAN, false>;
+    case QuantOp::WarmupReceiver: return k_quant<QuantOp::WarmupReceiver, 2, 8, 0, LEAN, false>;
+    case QuantOp::Compress: return pick_bits<QuantOp::Compress, LEAN, false>(bits, group, ss);
+    case QuantOp::Decompress:
+        return rc ? pick_bits<QuantOp::Decompress, LEAN, true>(bits, group, ss)
+                  : pick_bits<QuantOp::Decompress, LEAN, false>(bits, group, ss);
+    case QuantOp::Loopback:
+        return rc ? pick_bits<QuantOp::Loopback, LEAN, true>(bits, group, ss)
+                  : pick_bits<QuantOp::Loopback, LEAN, false>(bits, group, ss);
     }
     return nullptr;
 }
@@ -515,40 +537,50 @@ struct Shape {
     int per_sm;
 };
 
-template <QuantOp OP, bool LEAN, int K>
+template <QuantOp OP, bool LEAN, int K, bool RC>
 void shape_is(int &threads, int &cap, int64_t &tile_vec)
 {
-    threads = QShape<OP, LEAN, K>::kThreads;
-    cap = QShape<OP, LEAN, K>::kMaxPerSm;
-    tile_vec = qtile_vec<OP, LEAN, K>();
+    threads = QShapeR<OP, LEAN, K, RC>::kThreads;
+    cap = QShapeR<OP, LEAN, K, RC>::kMaxPerSm;
+    tile_vec = qtile_vec<OP, LEAN, K, RC>();
 }
 
-template <QuantOp OP, bool LEAN>
+template <QuantOp OP, bool LEAN, bool RC>
 void shape_bits(int bits, int &threads, int &cap, int64_t &tile_vec)
 {
     if (bits == 1)
-        shape_is<OP, LEAN, 1>(threads, cap, tile_vec);
+        shape_is<OP, LEAN, 1, RC>(threads, cap, tile_vec);
     else if (bits == 4)
-        shape_is<OP, LEAN, 4>(threads, cap, tile_vec);
+        shape_is<OP, LEAN, 4, RC>(threads, cap, tile_vec);
     else
-        shape_is<OP, LEAN, 2>(threads, cap, tile_vec);
+        shape_is<OP, LEAN, 2, RC>(threads, cap, tile_vec);
 }
 
 // The shape of the instance pick() returns: the warmup kernels are the k = 2
 // instances.
 template <bool LEAN>
-void shape_of(QuantOp op, int bits, int &threads, int &cap, int64_t &tile_vec)
+void shape_of(QuantOp op, int bits, bool rc, int &threads, int &cap, int64_t &tile_vec)
 {
     switch (op) {
-    case QuantOp::WarmupSender: shape_is<QuantOp::WarmupSender, LEAN, 2>(threads, cap, tile_vec); break;
-    case QuantOp::WarmupReceiver: shape_is<QuantOp::WarmupReceiver, LEAN, 2>(threads, cap, tile_vec); break;
-    case QuantOp::Compress: shape_bits<QuantOp::Compress, LEAN>(bits, threads, cap, tile_vec); break;
-    case QuantOp::Decompress: shape_bits<QuantOp::Decompress, LEAN>(bits, threads, cap, tile_vec); break;
-    case QuantOp::Loopback: shape_bits<QuantOp::Loopback, LEAN>(bits, threads, cap, tile_vec); break;
+    case QuantOp::WarmupSender: shape_is<QuantOp::WarmupSender, LEAN, 2, false>(threads, cap, tile_vec); break;
+    case QuantOp::WarmupReceiver: shape_is<QuantOp::WarmupReceiver, LEAN, 2, false>(threads, cap, tile_vec); break;
+    case QuantOp::Compress: shape_bits<QuantOp::Compress, LEAN, false>(bits, threads, cap, tile_vec); break;
+    case QuantOp::Decompress:
+        if (rc)
+            shape_bits<QuantOp::Decompress, LEAN, true>(bits, threads, cap, tile_vec);
+        else
+            shape_bits<QuantOp::Decompress, LEAN, false>(bits, threads, cap, tile_vec);
+        break;
+    case QuantOp::Loopback:
+        if (rc)
+            shape_bits<QuantOp::Loopback, LEAN, true>(bits, threads, cap, tile_vec);
+        else
+            shape_bits<QuantOp::Loopback, LEAN, false>(bits, threads, cap, tile_vec);
+        break;
     }
 }
 
-Shape launch_shape(KernelFn fn, bool lean, QuantOp op, int bits)
+Shape launch_shape(KernelFn fn, bool lean, QuantOp op, int bits, bool rc)
 {
     static std::mutex mu;
     static std::unordered_map<const void *, Shape> cache;
@@ -559,9 +591,9 @@ Shape launch_shape(KernelFn fn, bool lean, QuantOp op, int bits)
     int cap = 0;
     int64_t tile_vec = 0;
     if (lean)
-        shape_of<true>(op, bits, sh.threads, cap, tile_vec);
+        shape_of<true>(op, bits, rc, sh.threads, cap, tile_vec);
     else
-        shape_of<false>(op, bits, sh.threads, cap, tile_vec);
+        shape_of<false>(op, bits, rc, sh.threads, cap, tile_vec);
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, sh.threads, sh.smem) != cudaSuccess || nb < 1) nb = 1;
     sh.per_sm = (cap > 0 && nb > cap) ? cap : nb;
@@ -586,15 +618,19 @@ int num_sms()
 cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool lean, QuantLaunch &lp,
                          cudaStream_t stream)
 {
-    KernelFn fn = lean ? pick<true>(op, bits, group, sign_scale) : pick<false>(op, bits, group, sign_scale);
+    // the receiver instances that write recon are used when a slot asks for it
+    bool rc = false;
+    if (op == QuantOp::Decompress || op == QuantOp::Loopback)
+        for (int k = 0; k < lp.nslots; ++k) rc = rc || lp.slot[k].recon != nullptr;
+    KernelFn fn = lean ? pick<true>(op, bits, group, sign_scale, rc) : pick<false>(op, bits, group, sign_scale, rc);
     if (!fn) return cudaErrorInvalidValue;
     // tile prefix of every slot, in this kernel's tile size
     int threads = 0, cap = 0;
     int64_t tile_vec = 0;
     if (lean)
-        shape_of<true>(op, bits, threads, cap, tile_vec);
+        shape_of<true>(op, bits, rc, threads, cap, tile_vec);
     else
-        shape_of<false>(op, bits, threads, cap, tile_vec);
+        shape_of<false>(op, bits, rc, threads, cap, tile_vec);
     int64_t tiles = 0;
     for (int k = 0; k < lp.nslots; ++k) {
         lp.slot[k].tile0 = tiles;
@@ -602,13 +638,13 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool l
     }
     lp.ntiles = tiles;
     if (tiles <= 0) return cudaSuccess;
-    const Shape sh = launch_shape(fn, lean, op, bits);
+    const Shape sh = launch_shape(fn, lean, op, bits, rc);
     const int64_t cap_blocks = (int64_t)num_sms() * sh.per_sm;
     const int grid = (int)(tiles < cap_blocks ? tiles : cap_blocks);
     if (log_enabled()) {
         char name[64];
-        snprintf(name, sizeof name, "k_quant<op %d, k %d, G %d, ss %d, %s>", (int)op, bits, group, sign_scale,
-                 lean ? "bf16 state" : "fp32 state");
+        snprintf(name, sizeof name, "k_quant<op %d, k %d, G %d, ss %d, %s%s>", (int)op, bits, group, sign_scale,
+                 lean ? "bf16 state" : "fp32 state", rc ? ", recon" : "");
         log_launch(name, dim3(grid), dim3(sh.threads), sh.smem);
     }
     fn<<<grid, sh.threads, sh.smem, stream>>>(lp);

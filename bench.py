@@ -422,20 +422,33 @@ def run_cf(args, w):
         barrier(world)
         torch.cuda.synchronize()
         q0e, q1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        lev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
         q0e.record(stream)
         for k in range(args.steps):
             i = args.warmup + 1 + k
-            lean_step(i, l_arrays[(i - 1) % len(l_arrays)])
+            arr = l_arrays[(i - 1) % len(l_arrays)]
+            lev[k][0].record(stream)
+            if L.cf_compress(lh, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(lh).decode())
+            lev[k][1].record(stream)
+            if L.cf_decompress(lh, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(lh).decode())
+            lev[k][2].record(stream)
         q1e.record(stream)
         torch.cuda.synchronize()
         if lctx.check() != 0:
             raise RuntimeError("device status in the lean run")
         lean_ms = max_over_ranks(q0e.elapsed_time(q1e), world) / args.steps
+        lc_ms = sum(e[0].elapsed_time(e[1]) for e in lev) / args.steps
+        ld_ms = sum(e[1].elapsed_time(e[2]) for e in lev) / args.steps
         pay = w.bits / 8 + 4 / w.group
-        lean_bytes = (2 + 2 + 2 + 2 + 2 + pay + pay + 2 + 2) * n_elem
+        lc_b, ld_b = (2 + 2 + 2 + 2 + 2 + pay) * n_elem, (pay + 2 + 2) * n_elem
+        lean_bytes = lc_b + ld_b
         lean = {"ms_per_step": lean_ms, "value": world * x_bytes / (lean_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "alg_bytes_per_step": lean_bytes, "achieved": lean_bytes / (lean_ms * 1e-3) / 1e9,
                 "frac": lean_bytes / (lean_ms * 1e-3) / 1e9 / peak,
+                "compress": {"ms_per_launch": lc_ms, "frac": lc_b / (lc_ms * 1e-3) / 1e9 / peak},
+                "decompress": {"ms_per_launch": ld_ms, "frac": ld_b / (ld_ms * 1e-3) / 1e9 / peak},
                 "note": "state_bf16=1: E and C kept in bf16 (14.56 B/elt for compress + decompress)"}
         del lctx, lst, l_arrays
 
