@@ -69,7 +69,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if _stale(LIB, objs):
         tmp = LIB + ".tmp.%d" % os.getpid()
         cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
-               "-lcudart_static" if False else "-lcudart"]
+               "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

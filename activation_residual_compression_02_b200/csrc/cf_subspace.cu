@@ -58,10 +58,20 @@ constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parame
 // one box per stage with 8 stages ran at 5.2-5.6 TB/s; three boxes with four
 // stages at 6.6 TB/s, bit-identical.  RP = 32 needs twice the B space and
 // keeps two boxes with five stages to stay within 227 KB of shared memory.
+//
+// Accumulation in chunks of K.  The tensor core's fp32 accumulator loses a
+// fraction of an ulp towards zero at each accumulating MMA, so one long
+// accumulation chain shrinks the product by a factor that grows with K
+// (measured on exactly rank-16 matrices: P = A Q was 2.8e-5 small at
+// K = 4096 and 1.6e-4 at K = 32768, and E = A - U R V^T inherits it).  The
+// MMA therefore restarts its accumulator every CH stages (about 1000 of K),
+// and the epilogue adds the chunk sums on the CUDA cores with round to
+// nearest, in chunk order, so the loss stays at its K = 1000 level.
 template <int RP>
 struct GemmCfg {
     static constexpr int NB = RP == 16 ? 3 : 2;         // boxes of A per stage
     static constexpr int ST = RP == 16 ? 4 : 5;         // pipeline stages
+    static constexpr int CH = RP == 16 ? 10 : 16;       // stages per accumulation chunk (960 / 1024 of K)
     static constexpr int BK = NB * kBoxK;               // K per stage
     static constexpr int ATile = NB * kBoxBytes;        // A bytes per stage
     static constexpr int BBox = RP * kBoxK * 4;         // one RP x 32 box of Q^T / P^T
@@ -197,41 +207,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
         const uint32_t idesc = instr_desc_tf32(RP, p.mn_major);
-        uint32_t it = 0, lt = 0;
+        uint32_t it = 0, lc = 0;   // stage counter; accumulation-chunk counter (selects the TMEM buffer)
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++lt) {
-            const int b = lt & 1;
-            const uint32_t aph = (lt >> 1) & 1u;
-            if (!wait_bounded(&S->acce[b], aph ^ 1u, abort_flag, p.status, wait_ns)) break;
-            tc_fence_after();
-            const uint32_t dtm = tmem + (uint32_t)(b * 32);
-            for (int kt = 0; kt < p.ktiles; ++kt, ++it) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1u;
-                if (!wait_bounded(&S->conv[s], ph, abort_flag, p.status, wait_ns)) {
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            for (int k0 = 0; k0 < p.ktiles && ok; k0 += C::CH, ++lc) {
+                const int k1 = min(p.ktiles, k0 + C::CH);
+                const int b = lc & 1;
+                const uint32_t aph = (lc >> 1) & 1u;
+                if (!wait_bounded(&S->acce[b], aph ^ 1u, abort_flag, p.status, wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t a0 = smem_u32(sA + s * C::ATile);
-                    const uint32_t b0 = smem_u32(sB + s * C::BTile);
-#pragma unroll
-                    for (int k = 0; k < C::BK / 8; ++k) {
-                        // K step k: box k / 4, 8-element slice k % 4 of it
-                        const uint32_t ah = a0 + (k / 4) * kBoxBytes, bh = b0 + (k / 4) * C::BBox;
-                        const uint32_t kk = (uint32_t)(k % 4);
-                        const uint64_t ad = p.mn_major ? smem_desc(ah + kk * 1024, 4096, 512, kLayoutSw128Atom32)
-                                                       : smem_desc(ah + kk * 32, 16, 1024, kLayoutSw128);
-                        const uint64_t bd = smem_desc(bh + kk * 32, 16, 1024, kLayoutSw128);
-                        tc_mma_tf32(dtm, ad, bd, idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                const uint32_t dtm = tmem + (uint32_t)(b * 32);
+                for (int kt = k0; kt < k1; ++kt, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!wait_bounded(&S->conv[s], ph, abort_flag, p.status, wait_ns)) {
+                        ok = false;
+                        break;
                     }
-                    tc_commit(&S->empty[s]);
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a0 = smem_u32(sA + s * C::ATile);
+                        const uint32_t b0 = smem_u32(sB + s * C::BTile);
+#pragma unroll
+                        for (int k = 0; k < C::BK / 8; ++k) {
+                            // K step k: box k / 4, 8-element slice k % 4 of it
+                            const uint32_t ah = a0 + (k / 4) * kBoxBytes, bh = b0 + (k / 4) * C::BBox;
+                            const uint32_t kk = (uint32_t)(k % 4);
+                            const uint64_t ad = p.mn_major ? smem_desc(ah + kk * 1024, 4096, 512, kLayoutSw128Atom32)
+                                                           : smem_desc(ah + kk * 32, 16, 1024, kLayoutSw128);
+                            const uint64_t bd = smem_desc(bh + kk * 32, 16, 1024, kLayoutSw128);
+                            tc_mma_tf32(dtm, ad, bd, idesc, (kt > k0 || k > 0) ? 1u : 0u);
+                        }
+                        tc_commit(&S->empty[s]);
+                    }
+                    __syncwarp();
                 }
+                if (ok && lane == 0) tc_commit(&S->accf[b]);
                 __syncwarp();
             }
-            if (ok && lane == 0) tc_commit(&S->accf[b]);
-            __syncwarp();
         }
         // Drain: all MMAs this thread issued have completed before TMEM is freed.
         if (lane == 0) {
@@ -270,29 +286,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
     } else {
         // ----------------------------------------------------- epilogue --
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
-            const int b = lt & 1;
-            const uint32_t aph = (lt >> 1) & 1u;
-            if (!wait_bounded(&S->accf[b], aph, abort_flag, p.status, wait_ns)) break;
-            tc_fence_after();
-            uint32_t v[32];
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * 32);
-            {
-                uint32_t lo[16];
-                tc_ld16(taddr, lo);
+        uint32_t lc = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            // sum of the tile's accumulation chunks, in chunk order, rounded to nearest
+            float acc[RP];
+            for (int k0 = 0; k0 < p.ktiles; k0 += C::CH, ++lc) {
+                const int b = lc & 1;
+                const uint32_t aph = (lc >> 1) & 1u;
+                if (!wait_bounded(&S->accf[b], aph, abort_flag, p.status, wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t v[32];
+                const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * 32);
+                {
+                    uint32_t lo[16];
+                    tc_ld16(taddr, lo);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) v[c] = lo[c];
-            }
-            if (RP > 16) {
-                uint32_t hi[16];
-                tc_ld16(taddr + 16, hi);
+                    for (int c = 0; c < 16; ++c) v[c] = lo[c];
+                }
+                if (RP > 16) {
+                    uint32_t hi[16];
+                    tc_ld16(taddr + 16, hi);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) v[16 + c] = hi[c];
+                    for (int c = 0; c < 16; ++c) v[16 + c] = hi[c];
+                }
+                tc_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&S->acce[b]);
+#pragma unroll
+                for (int c = 0; c < RP; ++c)
+                    acc[c] = k0 == 0 ? __uint_as_float(v[c]) : __fadd_rn(acc[c], __uint_as_float(v[c]));
             }
-            tc_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&S->acce[b]);
+            if (!ok) break;
 
             const int mi = tile / p.tiles_per_mat;
             const int mt = tile - mi * p.tiles_per_mat;
@@ -302,13 +330,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_cons
                 if (p.out_mode == 0) {
 #pragma unroll
                     for (int c = 0; c < RP; ++c)
-                        out[(int64_t)c * p.out_ld + row] = round_tf32(__uint_as_float(v[c]));
+                        out[(int64_t)c * p.out_ld + row] = round_tf32(acc[c]);
                 } else {
                     float4 *o = (float4 *)(out + (int64_t)row * RP);
 #pragma unroll
                     for (int c = 0; c < RP; c += 4)
-                        o[c / 4] = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                               __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                        o[c / 4] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
                 }
             }
         }
