@@ -57,20 +57,21 @@ def alg_bytes_per_elem(bits, group):
     return 2 + 2 + 4 + 2 + 4 + payload, payload + 4 + 4
 
 
-def source_hash():
-    p = os.path.join(ROOT, "activation_residual_compression_02_b200", "csrc", "cf_quant.cu")
+def source_hash(src="cf_quant.cu"):
+    p = os.path.join(ROOT, "activation_residual_compression_02_b200", "csrc", src)
     with open(p, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(kernel):
-    """DRAM bytes per launch from a committed ncu summary of the same source."""
+def recorded_traffic(kernel, src="cf_quant.cu"):
+    """DRAM bytes per launch (per call for the low-rank call) from a committed
+    ncu summary of the same source file."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         e = d.get(kernel)
-        if e and e.get("source_sha") == source_hash():
+        if e and e.get("source_sha") == source_hash(src):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -624,7 +625,9 @@ def run_lowrank_bench(args, w):
                    "l2": "inputs larger than L2 (3.2 GB of A per step)"},
         "roofline": {"bound": "hbm", "kernel": "whole cf_lowrank call", "achieved": alg_bytes / (ms * 1e-3) / 1e9,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": alg_bytes / (ms * 1e-3) / 1e9 / peak, "traffic": None,
+                     "frac": alg_bytes / (ms * 1e-3) / 1e9 / peak,
+                     "traffic": (recorded_traffic("lowrank_call", "cf_subspace.cu")
+                                 if k == w.slots and not args.warm_start else None),
                      "alg_bytes_per_step": alg_bytes, "tflops": flops / (ms * 1e-3) / 1e12,
                      "schedule_bytes_per_step": sched_bytes,
                      "schedule_frac": sched_bytes / (ms * 1e-3) / 1e9 / peak,
