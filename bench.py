@@ -642,6 +642,85 @@ def run_lowrank_bench(args, w):
     return 0
 
 
+def run_exchange_bench(args, w):
+    """Algorithm 1's K/V all-gather with compressed payloads (PatchAllGather)
+    against the same all-gather of the bf16 activations, on N GPUs.  Each rank
+    owns the workload's slots as its shard.  At N = 1 the rank decodes its own
+    payload (include_self) so that every stage of the step runs."""
+    import datetime
+
+    import torch.distributed as dist
+
+    world, rank, local = dist_init()
+    if world == 1:
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{29400 + os.getpid() % 500}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120))
+    from activation_residual_compression_02_b200.exchange import PatchAllGather, gather_payloads
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shapes = [(w.rows, w.cols)] * w.slots
+    ex = PatchAllGather(shapes, bits=w.bits, group=w.group, buckets=args.buckets, include_self=world == 1)
+    nsteps = min(w.steps, 1 + args.warmup + args.steps)
+    streams = [synth.SlotStream(w, s, seed=rank, device=dev) for s in range(w.slots)]
+    X = [[streams[s].next().reshape(-1) for s in range(w.slots)] for _ in range(nsteps)]
+    del streams
+    x_bytes = w.elems * 2
+    stream = torch.cuda.current_stream()
+
+    def x_at(i):
+        return X[1 + (i - 1) % (nsteps - 1)] if nsteps > 1 else X[0]
+
+    ex.step(0, X[0])
+    for i in range(1, args.warmup + 1):
+        ex.step(i, x_at(i))
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for k in range(args.steps):
+            i = args.warmup + 1 + k
+            ex.step(i, x_at(i))
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if ex.check() != 0:
+        raise RuntimeError("device status in the exchange run")
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    # the same all-gather of the bf16 activations themselves
+    flat = torch.cat([x.view(torch.uint8) for x in X[0]])
+    for _ in range(args.warmup):
+        gather_payloads(flat, world)
+    torch.cuda.synchronize()
+    barrier(world)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for _ in range(args.steps):
+        gather_payloads(flat, world)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    raw_ms = max_over_ranks(r0.elapsed_time(r1), world) / args.steps
+    pay = sum(b.nbytes for b in ex.send_buf)
+    line = {
+        "metric": "compressed K/V all-gather step (compress + all-gather + decompress), GB/s of bf16 activations",
+        "value": world * x_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.slots} slots x {w.rows} x {w.cols} bf16 per rank, k={w.bits}, "
+                               f"G={w.group}, patch-parallel all-gather (Algorithm 1), {len(ex.buckets)} buckets",
+                   "decoded_peers": len(ex.peers)},
+        "payload_bytes_per_rank": pay, "raw_bytes_per_rank": x_bytes,
+        "raw_bf16_allgather_ms": raw_ms,
+        "note": "raw_bf16_allgather_ms: NCCL all-gather of the same activations uncompressed; at N = 1 both "
+                "collectives are local copies",
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del ex
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -658,6 +737,9 @@ def main():
     ap.add_argument("--no-lean", action="store_true")
     ap.add_argument("--no-recon", action="store_true")
     ap.add_argument("--warm-start", action="store_true", help="low-rank: T = 1 from the previous call's V")
+    ap.add_argument("--exchange", action="store_true",
+                    help="time the compressed K/V all-gather of patch parallelism instead of the codec alone")
+    ap.add_argument("--buckets", type=int, default=4, help="--exchange: slot buckets overlapped with the collective")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -668,6 +750,8 @@ def main():
         return run_reference(args, w)
     if w.mode == 1:
         return run_lowrank_bench(args, w)
+    if args.exchange:
+        return run_exchange_bench(args, w)
     return run_cf(args, w)
 
 
