@@ -55,6 +55,21 @@ struct QShapeBase {
     static constexpr int kUnroll = 4;
     static constexpr int kMaxPerSm = 0;
 };
+// Warmup step (fp32 state), once per run: sender 384 x 4 (94.2% / 94.5% of the
+// copy bandwidth on the FLUX- / CogVideoX-shaped steps; 256 x 4 uncapped:
+// 82.3% / 82.6%), receiver 512 x 4 (90.9% / 92.8%; 256 x 4: 72.9% / 73.1%).
+template <>
+struct QShapeBase<QuantOp::WarmupSender, false> {
+    static constexpr int kThreads = 384;
+    static constexpr int kUnroll = 4;
+    static constexpr int kMaxPerSm = 1;
+};
+template <>
+struct QShapeBase<QuantOp::WarmupReceiver, false> {
+    static constexpr int kThreads = 512;
+    static constexpr int kUnroll = 4;
+    static constexpr int kMaxPerSm = 1;
+};
 template <>
 struct QShapeBase<QuantOp::Compress, false> {
     static constexpr int kThreads = 1024;
