@@ -615,6 +615,62 @@ def run_lowrank_bench(args, w):
     sched_bytes = elems * (4 * (2 * T + 2) + 4)   # A read by each of the 2T+1 products and the apply, E written
     flops = 2.0 * (2 * T + 1) * m * n * r * k + 2.0 * m * n * r * k
 
+    # ---- low-rank mode through cf_compress / cf_decompress ---------------
+    # The same shapes as bf16 activation slots: each compressed step first
+    # materialises A = (X - base) + E in fp32 (k_residual_f32), then runs the
+    # call above on it; the receiver adds U R V^T to its cache.
+    lr_mode = None
+    if args.through_slots:
+        shapes = [(m, n)] * k
+        mctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+        mws = torch.empty(mctx.workspace_bytes(), dtype=torch.uint8, device=dev)
+        mctx.set_workspace(mws)
+        wq = synth.FLUX.scaled(slots=k, rows=m, cols=n)
+        sst = [synth.SlotStream(wq, i, seed=rank, device=dev) for i in range(k)]
+        Xs = [[st_.next().reshape(-1) for st_ in sst] for _ in range(6)]
+        del sst
+        mb = [torch.empty(m * n, dtype=torch.bfloat16, device=dev) for _ in range(k)]
+        me = [torch.empty(m * n, device=dev) for _ in range(k)]
+        mc = [torch.empty(m * n, device=dev) for _ in range(k)]
+        arrs = [mctx._slots([cf.Slot(x=Xs[j][i], base=mb[i], err=me[i], cache=mc[i], q0=Q0[i], U=U[i], R=R[i],
+                                     V=V[i]) for i in range(k)]) for j in range(6)]
+        L, h, sh = cf.lib(), mctx.handle, stream.cuda_stream
+
+        def mstep(i, ev=None):
+            arr = arrs[0] if i == 0 else arrs[1 + (i - 1) % 5]
+            if ev:
+                ev[0].record(stream)
+            if L.cf_compress(h, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+            if ev:
+                ev[1].record(stream)
+            if L.cf_decompress(h, arr, i, sh) != 0:
+                raise RuntimeError(L.cf_last_error(h).decode())
+            if ev:
+                ev[2].record(stream)
+
+        for i in range(args.warmup + 1):
+            mstep(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        mev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for j in range(args.steps):
+            mstep(args.warmup + 1 + j, mev[j])
+        torch.cuda.synchronize()
+        if mctx.check() != 0:
+            raise RuntimeError("device status in the low-rank mode run")
+        c_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in mev) / args.steps, world)
+        d_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in mev) / args.steps, world)
+        lr_mode = {"compress_ms": c_ms, "decompress_ms": d_ms, "ms_per_step": c_ms + d_ms,
+                   "value": world * elems * 2 / ((c_ms + d_ms) * 1e-3) / 1e9, "unit": "GB/s of bf16 activations",
+                   "residual_ms_est": c_ms - ms,
+                   "residual_frac_est": 14 * elems / ((c_ms - ms) * 1e-3) / 1e9 / peak if c_ms > ms else None,
+                   "decompress_frac": 8 * elems / (d_ms * 1e-3) / 1e9 / peak,
+                   "note": "cf_compress = residual (14 B/elt: x, base, E read, A and base written) + the cf_lowrank "
+                           "call timed above; residual_ms_est = compress_ms - that call; decompress: C += U R V^T "
+                           "(8 B/elt)"}
+        del mctx, mws, Xs, mb, me, mc, arrs
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         import concurrent.futures
@@ -658,6 +714,7 @@ def run_lowrank_bench(args, w):
                      "note": "alg bytes count A once and E once; the schedule reads A from HBM in each of the "
                              "2T+1 products and in the apply"},
         "gpu_launches": args.steps * (2 * (T + 2) + (2 * T + 1) + 1), "e2e": None, "cpu_baseline": cpu,
+        "lowrank_mode": lr_mode,
         "clocks": clk.summary(),
     }
     if rank == 0:
@@ -761,6 +818,8 @@ def main():
     ap.add_argument("--no-lean", action="store_true")
     ap.add_argument("--no-recon", action="store_true")
     ap.add_argument("--warm-start", action="store_true", help="low-rank: T = 1 from the previous call's V")
+    ap.add_argument("--through-slots", action="store_true",
+                    help="low-rank: also time cf_compress / cf_decompress in low-rank mode on bf16 slots")
     ap.add_argument("--exchange", action="store_true",
                     help="time the compressed K/V all-gather of patch parallelism instead of the codec alone")
     ap.add_argument("--buckets", type=int, default=4, help="--exchange: slot buckets overlapped with the collective")
