@@ -331,7 +331,7 @@ cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes,
     if (cudaGetDevice(&dev) != cudaSuccess) return CF_E_CUDA;
     cudaDeviceProp prop;
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return CF_E_CUDA;
-    if (prop.major != 10) return CF_E_CUDA;  // the kernels are built for sm_100a only
+    if (prop.major != 10 || prop.minor != 0) return CF_E_CUDA;  // sm_100a code runs on compute capability 10.0 only
 
     cf_ctx *ctx = new (std::nothrow) cf_ctx;
     if (!ctx) return CF_E_NOMEM;

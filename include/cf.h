@@ -130,7 +130,7 @@ typedef struct cf_slot {
 
 /* Create a context for `nslots` slots of the given shapes (host array).
  * Validates the configuration and the shapes, checks that device 0 of the
- * current CUDA context is sm_100, and allocates the device status word.
+ * current CUDA context has compute capability 10.0 (sm_100a), and allocates the device status word.
  * nslots may be 0 for a context used only with cf_lowrank.
  * Errors: CF_E_ARG, CF_E_SHAPE, CF_E_NOMEM, CF_E_CUDA; *out is NULL then. */
 cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes, cf_ctx **out);
