@@ -129,8 +129,9 @@ typedef struct cf_slot {
 } cf_slot;
 
 /* Create a context for `nslots` slots of the given shapes (host array).
- * Validates the configuration and the shapes, checks that device 0 of the
- * current CUDA context has compute capability 10.0 (sm_100a), and allocates the device status word.
+ * Validates the configuration and the shapes, checks that the current CUDA
+ * device has compute capability 10.0 (the only target of sm_100a code), and
+ * allocates the device status word on it.
  * nslots may be 0 for a context used only with cf_lowrank.
  * Errors: CF_E_ARG, CF_E_SHAPE, CF_E_NOMEM, CF_E_CUDA; *out is NULL then. */
 cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes, cf_ctx **out);
