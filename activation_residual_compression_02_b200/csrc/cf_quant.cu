@@ -133,11 +133,13 @@ struct QShape<QuantOp::Decompress, false, 1> : QShapeOne<256, 8> {};
 // shape is sensitive (256 x 3: 79.7% for k = 2).
 template <>
 struct QShape<QuantOp::Loopback, false, 1> : QShapeOne<256, 6> {};
-// Lean-state sender (bf16 E): 1024 x 2 stays best for k = 2 (88.1%; 448 x 4:
-// 87.7%; 512 x 4: 85.9%); k = 4 and k = 1 want more vectors per thread:
-// 384 x 6 (1024 x 2: 86.6%; 512 x 4: 90.4%; 384 x 6: 91.6%) and 256 x 16
-// (1024 x 2: 86.2%; 256 x 16: 91.5%; 384 x 6: 90.8%), steps of the
-// CogVideoX-shaped and stress workloads.
+// Lean-state sender (bf16 E), steps of the FLUX-, CogVideoX-shaped and stress
+// workloads: k = 2 640 x 3 (94.0%; 1024 x 2: 88.3%; 896 x 2: 93.0%; 768 x 3:
+// 88.3%; 512 x 3: 89.9%); k = 4 384 x 6 (1024 x 2: 86.6%; 512 x 4: 90.4%;
+// 384 x 6: 91.6%); k = 1 256 x 16 (1024 x 2: 86.2%; 256 x 16: 91.2%;
+// 256 x 12: 90.6%; 384 x 6: 90.8%).
+template <>
+struct QShape<QuantOp::Compress, true, 2> : QShapeOne<640, 3> {};
 template <>
 struct QShape<QuantOp::Compress, true, 4> : QShapeOne<384, 6> {};
 template <>

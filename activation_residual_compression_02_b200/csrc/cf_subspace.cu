@@ -785,7 +785,9 @@ __device__ __forceinline__ void cp_async_wait()
 template <bool HAS_E, bool HAS_C>
 __host__ __device__ constexpr int async_stages()
 {
-    return (HAS_E && HAS_C) ? 3 : 4;
+    // E and C: 3 stages (smem); C only: 5 (85.4% of measured on the receiver of
+    // the 57 x 4608 x 3072 step, 4 stages: 84.6%); E only: 4
+    return (HAS_E && HAS_C) ? 3 : (HAS_C ? 5 : 4);
 }
 
 template <bool HAS_E, bool HAS_C>
