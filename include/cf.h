@@ -59,9 +59,12 @@
  * and state errors return before anything is launched and leave all buffers
  * untouched.  Device-side conditions (non-finite scale, a bounded wait that
  * gave up) set bits in the context's status word and are reported by the
- * next cf_check.  A context is not thread-safe; separate contexts are
- * independent.  There is no CPU fallback: without a usable sm_100 device
- * cf_create returns CF_E_CUDA.
+ * next cf_check.  The stream-ordered calls allocate no device memory and
+ * do not synchronise, so they can be captured into a CUDA graph and replayed
+ * (the kernels read the slot pointers given at capture; a quantised step
+ * >= 1 is the same launch for every later step).  A context is not
+ * thread-safe; separate contexts are independent.  There is no CPU fallback:
+ * without a usable sm_100 device cf_create returns CF_E_CUDA.
  */
 #ifndef CF_H
 #define CF_H
