@@ -797,6 +797,29 @@ constexpr size_t async_smem_bytes()
            ((HAS_E ? kApplyThreads * 16 : 0) + (HAS_C ? kApplyThreads * 16 : 0) + 8 * 64);
 }
 
+// Paired fp32 arithmetic of sm_100 (PTX .f32x2): two independent
+// round-to-nearest FMAs in one instruction, on 64-bit register pairs whose
+// low half is the first element.
+__device__ __forceinline__ unsigned long long f32x2_pack(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f32x2_fma(unsigned long long a, unsigned long long b,
+                                                        unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ float f32x2_sum(unsigned long long a)
+{
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a));
+    return lo + hi;
+}
+
 template <bool HAS_E, bool HAS_C>
 __global__ void __launch_bounds__(kApplyThreads, 2) k_apply_async(const __grid_constant__ ApplyParams p)
 {
@@ -833,16 +856,21 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply_async(const __grid_c
     // U slots past column r are never copied: they must read as zero
     for (int i = tid; i < S * RF * 8 * 16; i += kApplyThreads) ringU[i] = 0.0f;
     __syncthreads();
-    float w[RMAX][CPT];
+    // W[k][c] for k = 2h (low half) and 2h + 1 (high half) of wp[h][c]: the
+    // row products below accumulate even and odd k in the two halves of a pair
+    // (half the FMA instructions; the kernel is otherwise issue-bound).
+    unsigned long long wp[RMAX / 2][CPT];
 #pragma unroll
-    for (int k = 0; k < RMAX; ++k)
+    for (int h = 0; h < RMAX / 2; ++h)
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
-            float acc = 0.0f;
+            float acc[2] = {0.0f, 0.0f};
             const int j = lane * CPT + c;
 #pragma unroll
-            for (int q = 0; q < RMAX; ++q) acc = fmaf(Rs[k * 33 + q], Vs[j * (RMAX + 1) + q], acc);
-            w[k][c] = acc;
+            for (int e = 0; e < 2; ++e)
+#pragma unroll
+                for (int q = 0; q < RMAX; ++q) acc[e] = fmaf(Rs[(2 * h + e) * 33 + q], Vs[j * (RMAX + 1) + q], acc[e]);
+            wp[h][c] = f32x2_pack(acc[0], acc[1]);
         }
 
     const int nrows = row_end - row0;
@@ -883,19 +911,21 @@ __global__ void __launch_bounds__(kApplyThreads, 2) k_apply_async(const __grid_c
         for (int u = 0; u < RF; ++u) {
             const int row = row0 + g * 8 * RF + warp + 8 * u;
             if (row >= row_end || !col_ok) continue;
-            const float4 *urow4 = reinterpret_cast<const float4 *>(&ringU[((slot * RF + u) * 8 + warp) * 16]);
-            float d[CPT] = {0.f, 0.f, 0.f, 0.f};
+            // U row as (u_2h, u_2h+1) pairs, straight from shared memory
+            const ulonglong2 *urow = reinterpret_cast<const ulonglong2 *>(&ringU[((slot * RF + u) * 8 + warp) * 16]);
+            unsigned long long dp[CPT] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int k4 = 0; k4 < RMAX / 4; ++k4) {
-                const float4 uk = urow4[k4];
+                const ulonglong2 uk = urow[k4];
 #pragma unroll
                 for (int c = 0; c < CPT; ++c) {
-                    d[c] = fmaf(uk.x, w[4 * k4][c], d[c]);
-                    d[c] = fmaf(uk.y, w[4 * k4 + 1][c], d[c]);
-                    d[c] = fmaf(uk.z, w[4 * k4 + 2][c], d[c]);
-                    d[c] = fmaf(uk.w, w[4 * k4 + 3][c], d[c]);
+                    dp[c] = f32x2_fma(uk.x, wp[2 * k4][c], dp[c]);
+                    dp[c] = f32x2_fma(uk.y, wp[2 * k4 + 1][c], dp[c]);
                 }
             }
+            float d[CPT];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) d[c] = f32x2_sum(dp[c]);
             const int64_t off = (int64_t)row * n + col;
             if (HAS_E && M.E) {
                 const float4 a = ringA[(slot * RF + u) * kApplyThreads + tid];

@@ -707,7 +707,7 @@ def run_lowrank_bench(args, w):
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": alg_bytes / (ms * 1e-3) / 1e9 / peak,
                      "traffic": (recorded_traffic("lowrank_call", "cf_subspace.cu")
-                                 if k == w.slots and not args.warm_start else None),
+                                 if not args.slots and not args.warm_start else None),
                      "alg_bytes_per_step": alg_bytes, "tflops": flops / (ms * 1e-3) / 1e12,
                      "schedule_bytes_per_step": sched_bytes,
                      "schedule_frac": sched_bytes / (ms * 1e-3) / 1e9 / peak,
