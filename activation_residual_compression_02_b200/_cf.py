@@ -22,7 +22,7 @@ CF_MODE_QUANT, CF_MODE_LOWRANK = 0, 1
 
 EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
             "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
-            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback", "cf_resume"]
+            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback", "cf_resume", "cf_trace_enable", "cf_trace_read"]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -34,6 +34,10 @@ class cf_config(ctypes.Structure):
 
 class cf_shape(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+class cf_trace_entry(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char * 80), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
 
 
 class cf_slot(ctypes.Structure):
@@ -88,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.cf_destroy.restype = I
         L.cf_resume.argtypes = [P, I64]
         L.cf_resume.restype = I
+        L.cf_trace_enable.argtypes = [P, I]
+        L.cf_trace_enable.restype = I
+        L.cf_trace_read.argtypes = [P, ctypes.POINTER(cf_trace_entry), I]
+        L.cf_trace_read.restype = I
         L.cf_lowrank_noalloc.argtypes = [ctypes.POINTER(cf_config), I, I64, I64, PP, PP, PP, PP, PP, PP, PP, P]
         L.cf_lowrank_noalloc.restype = I
         _lib = L
@@ -208,6 +216,20 @@ class Context:
         st = lib().cf_lowrank(self._h, nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R), _parr(V), _parr(E),
                               _parr(C), _stream_handle(stream))
         self._raise(st, "cf_lowrank")
+
+    def trace(self, on: bool = True):
+        """Time every kernel launch of this context with CUDA events (cf_trace_enable)."""
+        self._raise(lib().cf_trace_enable(self._h, int(bool(on))), "cf_trace_enable")
+
+    def trace_read(self) -> List[dict]:
+        """Per-kernel launches and summed milliseconds since the last read (cf_trace_read)."""
+        cap = 64
+        buf = (cf_trace_entry * cap)()
+        n = lib().cf_trace_read(self._h, buf, cap)
+        if n < 0:
+            raise CfError(-n, f"cf_trace_read: {lib().cf_last_error(self._h).decode()}")
+        return [{"kernel": buf[i].kernel.decode(), "launches": buf[i].launches, "total_ms": buf[i].total_ms}
+                for i in range(min(n, cap))]
 
     def resume(self, steps_done: int):
         """Continue a run whose state buffers the caller restored (steps

@@ -16,8 +16,33 @@
 
 #include "cf_internal.h"
 
+namespace cf {
+
+// Event pairs of traced launches, summed per kernel name by cf_trace_read.
+struct Tracer {
+    struct Rec {
+        std::string kernel;
+        cudaEvent_t e0, e1;
+    };
+    std::vector<Rec> recs;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pool;   // events free for reuse
+    bool failed = false;                                     // an event could not be created or recorded
+    ~Tracer()
+    {
+        for (auto &r : recs) pool.emplace_back(r.e0, r.e1);
+        for (auto &e : pool) {
+            cudaEventDestroy(e.first);
+            cudaEventDestroy(e.second);
+        }
+    }
+};
+
+}  // namespace cf
+
 struct cf_ctx {
     cf_config cfg{};
+    bool tracing = false;
+    cf::Tracer tracer;
     std::vector<cf_shape> shapes;
     uint32_t *d_status = nullptr;
     void *ws = nullptr;
@@ -47,9 +72,51 @@ void log_launch(const char *kernel, dim3 grid, dim3 block, size_t smem)
             block.x, block.y, block.z, smem);
 }
 
+namespace {
+thread_local Tracer *t_tracer = nullptr;   // the tracer of the API call running on this thread
+}
+
+bool trace_on() { return t_tracer != nullptr; }
+
+void trace_begin(const char *kernel, cudaStream_t stream)
+{
+    Tracer *t = t_tracer;
+    if (!t) return;
+    std::pair<cudaEvent_t, cudaEvent_t> ev;
+    if (!t->pool.empty()) {
+        ev = t->pool.back();
+        t->pool.pop_back();
+    } else if (cudaEventCreate(&ev.first) != cudaSuccess) {
+        t->failed = true;
+        return;
+    } else if (cudaEventCreate(&ev.second) != cudaSuccess) {
+        cudaEventDestroy(ev.first);
+        t->failed = true;
+        return;
+    }
+    if (cudaEventRecord(ev.first, stream) != cudaSuccess) t->failed = true;
+    t->recs.push_back(Tracer::Rec{kernel, ev.first, ev.second});
+}
+
+void trace_end(cudaStream_t stream)
+{
+    Tracer *t = t_tracer;
+    if (!t || t->recs.empty()) return;
+    if (cudaEventRecord(t->recs.back().e1, stream) != cudaSuccess) t->failed = true;
+}
+
 }  // namespace cf
 
 namespace {
+
+// Sets this thread's tracer for the duration of one API call of a tracing context.
+struct TraceGuard {
+    explicit TraceGuard(cf_ctx *ctx)
+    {
+        if (ctx && ctx->tracing) cf::t_tracer = &ctx->tracer;
+    }
+    ~TraceGuard() { cf::t_tracer = nullptr; }
+};
 
 cf_status fail(cf_ctx *ctx, cf_status st, const char *fmt, ...)
 {
@@ -281,6 +348,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
 cf_status codec_call(cf_ctx *ctx, const cf_slot *slots, int step, void *stream_, bool sender)
 {
     if (!ctx) return CF_E_ARG;
+    TraceGuard trace(ctx);
     if (step < 0) return fail(ctx, CF_E_ARG, "step must be >= 0");
     const int n = (int)ctx->shapes.size();
     if (n > 0 && !slots) return fail(ctx, CF_E_ARG, "slots is NULL");
@@ -387,6 +455,7 @@ cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
     }
     if (!(ctx->warm_sender && ctx->warm_receiver))
         return fail(ctx, CF_E_STATE, "step %d before the warmup step (step 0) on this context", step);
+    TraceGuard trace(ctx);
     const int n = (int)ctx->shapes.size();
     if (n > 0 && !slots) return fail(ctx, CF_E_ARG, "slots is NULL");
     for (int i = 0; i < n; ++i) {
@@ -411,6 +480,7 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
                      void *cuda_stream)
 {
     if (!ctx) return CF_E_ARG;
+    TraceGuard trace(ctx);
     if (ctx->cfg.mode != CF_MODE_LOWRANK) return fail(ctx, CF_E_ARG, "context is not in low-rank mode");
     if (nmat < 0) return fail(ctx, CF_E_ARG, "nmat must be >= 0");
     if (nmat == 0) return CF_OK;
@@ -491,6 +561,53 @@ cf_status cf_resume(cf_ctx *ctx, int64_t steps_done)
     ctx->lowrank_steps = steps_done;   // compressed steps after the warmup
     ctx->err.clear();
     return CF_OK;
+}
+
+cf_status cf_trace_enable(cf_ctx *ctx, int on)
+{
+    if (!ctx) return CF_E_ARG;
+    if (on != 0 && on != 1) return fail(ctx, CF_E_ARG, "on must be 0 or 1");
+    ctx->tracing = on != 0;
+    return CF_OK;
+}
+
+int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries)
+{
+    if (!ctx || max_entries < 0 || (max_entries > 0 && !out)) return -CF_E_ARG;
+    cf::Tracer &t = ctx->tracer;
+    struct Sum {
+        std::string kernel;
+        int launches;
+        double ms;
+    };
+    std::vector<Sum> sums;   // in order of first launch
+    bool bad = t.failed;
+    for (auto &r : t.recs) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(r.e1) != cudaSuccess || cudaEventElapsedTime(&ms, r.e0, r.e1) != cudaSuccess) {
+            bad = true;
+            ms = 0.0f;
+        }
+        size_t k = 0;
+        while (k < sums.size() && sums[k].kernel != r.kernel) ++k;
+        if (k == sums.size()) sums.push_back(Sum{r.kernel, 0, 0.0});
+        sums[k].launches += 1;
+        sums[k].ms += ms;
+        t.pool.emplace_back(r.e0, r.e1);
+    }
+    t.recs.clear();
+    t.failed = false;
+    for (size_t k = 0; k < sums.size() && (int)k < max_entries; ++k) {
+        memset(&out[k], 0, sizeof out[k]);
+        snprintf(out[k].kernel, sizeof out[k].kernel, "%s", sums[k].kernel.c_str());
+        out[k].launches = sums[k].launches;
+        out[k].total_ms = sums[k].ms;
+    }
+    if (bad) {
+        fail(ctx, CF_E_CUDA, "a trace event could not be created, recorded or read");
+        return -CF_E_CUDA;
+    }
+    return (int)sums.size();
 }
 
 cf_status cf_destroy(cf_ctx *ctx)

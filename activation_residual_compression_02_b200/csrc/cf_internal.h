@@ -95,4 +95,12 @@ int num_sms();
 void log_launch(const char *kernel, dim3 grid, dim3 block, size_t smem);
 bool log_enabled();
 
+// Per-launch device timing (cf_trace_enable / cf_trace_read): while an API
+// call of a tracing context runs, trace_on() is true on the calling thread and
+// each launch site brackets its kernel with trace_begin / trace_end, which
+// record a pair of CUDA events on the launch stream.
+bool trace_on();
+void trace_begin(const char *kernel, cudaStream_t stream);
+void trace_end(cudaStream_t stream);
+
 }  // namespace cf

@@ -109,7 +109,9 @@ cudaError_t launch_residual_f32(const void *const *x, void *const *base, const f
         if (tiles > 0) {
             const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
             log_launch("k_residual_f32", dim3(grid), dim3(kResThreads), 0);
+            trace_begin("k_residual_f32", stream);
             k_residual_f32<<<grid, kResThreads, 0, stream>>>(*p);
+            trace_end(stream);
             e = cudaGetLastError();
         }
     }

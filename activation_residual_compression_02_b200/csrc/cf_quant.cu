@@ -658,13 +658,16 @@ cudaError_t launch_quant(QuantOp op, int bits, int group, int sign_scale, bool l
     const Shape sh = launch_shape(fn, lean, op, bits, rc);
     const int64_t cap_blocks = (int64_t)num_sms() * sh.per_sm;
     const int grid = (int)(tiles < cap_blocks ? tiles : cap_blocks);
-    if (log_enabled()) {
-        char name[64];
+    const bool traced = trace_on();
+    if (log_enabled() || traced) {
+        char name[80];
         snprintf(name, sizeof name, "k_quant<op %d, k %d, G %d, ss %d, %s%s>", (int)op, bits, group, sign_scale,
                  lean ? "bf16 state" : "fp32 state", rc ? ", recon" : "");
         log_launch(name, dim3(grid), dim3(sh.threads), sh.smem);
+        if (traced) trace_begin(name, stream);
     }
     fn<<<grid, sh.threads, sh.smem, stream>>>(lp);
+    if (traced) trace_end(stream);
     return cudaGetLastError();
 }
 

@@ -988,8 +988,11 @@ cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
                                         (int)gemm_smem_bytes<RP>());
     });
     if (attr_err != cudaSuccess) return attr_err;
-    log_launch(RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>", dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP>());
+    const char *name = RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>";
+    log_launch(name, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP>());
+    trace_begin(name, stream);
     k_gemm_tf32<RP><<<grid, kGemmThreads, gemm_smem_bytes<RP>(), stream>>>(gp);
+    trace_end(stream);
     return cudaGetLastError();
 }
 
@@ -1108,21 +1111,29 @@ cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsL
         dim3 fgrid((unsigned)((rows + kCqrRows - 1) / kCqrRows), (unsigned)cnt);
         dim3 agrid((unsigned)((rows + kCqrThreads - 1) / kCqrThreads), (unsigned)cnt);
         const bool r16 = r <= 16;
-        log_launch(mode == 0 ? "k_cholqr_factor<Q>" : "k_cholqr_factor<U>", fgrid, dim3(kCqrThreads), 0);
-        log_launch(mode == 0 ? "k_cholqr_apply<Q>" : "k_cholqr_apply<U>", agrid, dim3(kCqrThreads), 0);
-        if (mode == 0) {
+        const char *fname = mode == 0 ? "k_cholqr_factor<Q>" : "k_cholqr_factor<U>";
+        const char *aname = mode == 0 ? "k_cholqr_apply<Q>" : "k_cholqr_apply<U>";
+        log_launch(fname, fgrid, dim3(kCqrThreads), 0);
+        log_launch(aname, agrid, dim3(kCqrThreads), 0);
+        trace_begin(fname, stream);
+        if (mode == 0)
             k_cholqr_factor<0><<<fgrid, kCqrThreads, 0, stream>>>(*cp);
+        else
+            k_cholqr_factor<1><<<fgrid, kCqrThreads, 0, stream>>>(*cp);
+        trace_end(stream);
+        trace_begin(aname, stream);
+        if (mode == 0) {
             if (r16)
                 k_cholqr_apply<0, 16><<<agrid, kCqrThreads, 0, stream>>>(*cp);
             else
                 k_cholqr_apply<0, 32><<<agrid, kCqrThreads, 0, stream>>>(*cp);
         } else {
-            k_cholqr_factor<1><<<fgrid, kCqrThreads, 0, stream>>>(*cp);
             if (r16)
                 k_cholqr_apply<1, 16><<<agrid, kCqrThreads, 0, stream>>>(*cp);
             else
                 k_cholqr_apply<1, 32><<<agrid, kCqrThreads, 0, stream>>>(*cp);
         }
+        trace_end(stream);
         err = cudaGetLastError();
     }
     delete cp;
@@ -1177,7 +1188,9 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
             }
             cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             log_launch("k_apply_async", dim3(blocks), dim3(kApplyThreads), smem);
+            trace_begin("k_apply_async", stream);
             fn<<<blocks, kApplyThreads, smem, stream>>>(*ap);
+            trace_end(stream);
             err = cudaGetLastError();
             continue;
         }
@@ -1186,7 +1199,9 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
         else
             fn = has_e ? (has_c ? k_apply<32, true, true> : k_apply<32, true, false>) : k_apply<32, false, true>;
         log_launch("k_apply", dim3(blocks), dim3(kApplyThreads), 0);
+        trace_begin("k_apply", stream);
         fn<<<blocks, kApplyThreads, 0, stream>>>(*ap);
+        trace_end(stream);
         err = cudaGetLastError();
     }
     delete ap;

@@ -254,6 +254,25 @@ cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64_t m, int64
                              const float *const *Q0, float *const *U, float *const *R, float *const *V,
                              float *const *E_opt, float *const *C_opt, void *cuda_stream);
 
+/* Per-launch device timing.  While tracing is on (cf_trace_enable(ctx, 1)),
+ * every kernel this context launches (in cf_compress, cf_decompress,
+ * cf_loopback and cf_lowrank) is bracketed by a pair of CUDA events recorded
+ * on its stream; the events come from a pool the context keeps.  Not for use
+ * while a stream is being captured into a CUDA graph.  Errors: CF_E_ARG. */
+cf_status cf_trace_enable(cf_ctx *ctx, int on);
+
+typedef struct cf_trace_entry {
+    char kernel[80];   /* kernel name and template arguments, NUL-terminated */
+    int launches;      /* traced launches of it since the last cf_trace_read */
+    double total_ms;   /* summed event-timed duration of those launches */
+} cf_trace_entry;
+
+/* Waits for the traced launches, writes per-kernel totals (in order of first
+ * launch) to out[0 .. min(count, max_entries)), clears them and returns the
+ * number of distinct kernels (which may exceed max_entries), or -CF_E_ARG /
+ * -CF_E_CUDA (an event could not be created, recorded or read). */
+int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries);
+
 /* Synchronise `cuda_stream`, read and clear the device status word.
  * Returns CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or CF_E_CUDA (an asynchronous
  * CUDA error, e.g. from an earlier launch). */
