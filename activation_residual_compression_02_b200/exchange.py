@@ -208,3 +208,103 @@ class PatchAllGather:
             if st != CF_OK:
                 worst = st
         return worst
+
+
+def ring_pass(local: torch.Tensor, world: int, rank: int, on_receive, pg=None, spare: Optional[torch.Tensor] = None):
+    """Algorithm 2's ring schedule for one flat buffer per rank.
+
+    In round s (s = 1 .. world - 1) every rank sends the buffer it holds to
+    rank + 1 and receives rank - 1's, so that after round s it holds the buffer
+    that started on rank - s; ``on_receive(src, buf)`` is called with it before
+    the next round forwards it.  ``spare`` (same size as ``local``) is the
+    second buffer of the double buffer; ``local`` itself is sent in round 1
+    and not modified.
+    """
+    if world <= 1:
+        return
+    nxt, prv = (rank + 1) % world, (rank - 1) % world
+    bufs = [local, torch.empty_like(local) if spare is None else spare, torch.empty_like(local)]
+    cur = 0
+    for s in range(1, world):
+        dst = 1 if cur != 1 else 2
+        ops = [dist.P2POp(dist.isend, bufs[cur], nxt, group=pg), dist.P2POp(dist.irecv, bufs[dst], prv, group=pg)]
+        for w in dist.batch_isend_irecv(ops):
+            w.wait()
+        on_receive((rank - s) % world, bufs[dst])
+        cur = dst
+
+
+class RingExchange:
+    """Compressed K/V ring of ring attention (Algorithm 2) for one rank.
+
+    Each step the rank compresses its own slots into one packed payload
+    buffer, which then travels the ring: in round s the rank receives the
+    payload that started on rank - s, decompresses it into the cache it keeps
+    for that rank's shards (the attention over that K/V block would follow
+    here), and forwards it.  Step 0 sends the bf16 activations themselves.
+    With ``include_self`` the rank also decodes its own payload before round 1.
+    """
+
+    def __init__(self, shapes: Sequence[Sequence[int]], bits: int = 2, group: int = 128, sign_scale: int = 0,
+                 pg=None, include_self: bool = False, recon: bool = False, device=None):
+        self.pg = pg
+        self.world = dist.get_world_size(pg)
+        self.rank = dist.get_rank(pg)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.shapes = [tuple(int(v) for v in s) for s in shapes]
+        self.bits, self.group = bits, group
+        self.include_self = include_self
+        self.send_ctx = Context(self.shapes, bits=bits, group=group, sign_scale=sign_scale)
+        self.send_state = QuantState(self.shapes, bits, group, device=self.device)
+        self.send_buf = PayloadBuffer(self.shapes, bits, group, device=self.device)
+        self.spare = torch.empty_like(self.send_buf.data)
+        self.peers = [p for p in range(self.world) if include_self or p != self.rank]
+        self.recv_ctx = {p: Context(self.shapes, bits=bits, group=group, sign_scale=sign_scale) for p in self.peers}
+        self.recv_state = {p: QuantState(self.shapes, bits, group, device=self.device, recon=recon)
+                           for p in self.peers}
+        ns = len(self.shapes)
+        send = self.send_state.slots([torch.empty(0, dtype=torch.bfloat16, device=self.device)] * ns,
+                                     codes=[self.send_buf.codes(s) for s in range(ns)],
+                                     scales=[self.send_buf.scales(s) for s in range(ns)])
+        self._send_arr = self.send_ctx._slots(send)
+
+    def cache(self, peer: int, slot: int, bf16: bool = False) -> torch.Tensor:
+        st = self.recv_state[peer]
+        return st.recon[slot] if bf16 else st.cache[slot]
+
+    def _decode(self, t: int, src: int, buf: torch.Tensor) -> None:
+        st = self.recv_state[src]
+        if t == 0:
+            slots, off = [], 0
+            for i, (r, c) in enumerate(self.shapes):
+                n = r * c
+                slots.append(Slot(x=buf[off:off + 2 * n].view(torch.bfloat16), cache=st.cache[i], recon=st.recon[i]))
+                off += 2 * n
+        else:
+            pb = PayloadBuffer(self.shapes, self.bits, self.group, data=buf)
+            slots = [Slot(codes=pb.codes(i), scales=pb.scales(i), cache=st.cache[i], recon=st.recon[i])
+                     for i in range(len(self.shapes))]
+        PatchAllGather._call(lib().cf_decompress, self.recv_ctx[src], slots, t)
+
+    def step(self, t: int, xs: Sequence[torch.Tensor]) -> None:
+        """Ring step t for this rank's activations ``xs`` (bf16, one per slot)."""
+        xs = [x.reshape(-1) for x in xs]
+        for x, (r, c) in zip(xs, self.shapes):
+            if x.dtype != torch.bfloat16 or x.device != self.device or not x.is_contiguous() or x.numel() != r * c:
+                raise ValueError("activations must be contiguous bf16 tensors of the slot shapes on this device")
+        for s, x in enumerate(xs):
+            self._send_arr[s].x = x.data_ptr() if x.numel() else None
+        PatchAllGather._call(lib().cf_compress, self.send_ctx, self._send_arr, t)
+        local = torch.cat([x.view(torch.uint8) for x in xs]) if t == 0 else self.send_buf.data
+        if self.include_self:
+            self._decode(t, self.rank, local)
+        ring_pass(local, self.world, self.rank, lambda src, buf: self._decode(t, src, buf), self.pg,
+                  spare=None if t == 0 else self.spare)
+
+    def check(self) -> int:
+        worst = CF_OK
+        for ctx in [self.send_ctx, *self.recv_ctx.values()]:
+            st = ctx.check()
+            if st != CF_OK:
+                worst = st
+        return worst

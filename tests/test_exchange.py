@@ -1,4 +1,5 @@
-"""The payload all-gather of patch parallelism (Algorithm 1), host side, on CPU.
+"""The payload all-gather of patch parallelism (Algorithm 1) and the payload
+ring of ring attention (Algorithm 2), host side, on CPU.
 
 Two gloo ranks each own the K/V shards of their own patch.  Each packs the
 oracle's payload of its shards into the exchange layout, the ranks all-gather
@@ -97,3 +98,55 @@ def test_payload_all_gather_gloo():
         out = man.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
         assert dict(out) == {0: True, 1: True}
+
+
+def _ring_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import torch.distributed as dist
+
+    import oracle
+    from activation_residual_compression_02_b200.exchange import PayloadBuffer, ring_pass
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ok = True
+        t = 2
+        mine = _oracle_slots(oracle, rank, t)
+        buf = PayloadBuffer(SHAPES, BITS, GROUP, device="cpu")
+        for s, o in enumerate(mine):
+            buf.codes(s).copy_(torch.from_numpy(o.codes))
+            buf.scales(s).copy_(torch.from_numpy(o.scales))
+        before = buf.data.clone()
+        order = []
+
+        def on_receive(src, data):
+            nonlocal ok
+            order.append(src)
+            got = PayloadBuffer(SHAPES, BITS, GROUP, data=data)
+            want, prev = _oracle_slots(oracle, src, t), _oracle_slots(oracle, src, t - 1)
+            for s, o in enumerate(want):
+                ok &= np.array_equal(got.codes(s).numpy(), o.codes)
+                ok &= np.array_equal(got.scales(s).numpy(), o.scales)
+                cache = prev[s].cache.copy()
+                if cache.size:
+                    oracle.decompress(got.codes(s).numpy(), got.scales(s).numpy(), cache, BITS, GROUP)
+                ok &= np.array_equal(cache, o.cache)
+
+        ring_pass(buf.data, world, rank, on_receive)
+        ok &= order == [(rank - s) % world for s in range(1, world)]
+        ok &= torch.equal(buf.data, before)       # the rank's own payload is not overwritten
+        out[rank] = bool(ok)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_payload_ring_gloo():
+    """Algorithm 2's ring over three gloo ranks: each rank receives every other
+    rank's payload once, in ring order, bit-exact and decodable by the oracle."""
+    port = 29800 + os.getpid() % 1000
+    with mp.Manager() as man:
+        out = man.dict()
+        mp.spawn(_ring_worker, args=(3, port, out), nprocs=3, join=True)
+        assert dict(out) == {0: True, 1: True, 2: True}

@@ -64,3 +64,26 @@ def test_patch_all_gather_matches_oracle(cf, oracle, pg, bits, group, buckets):
                 s = ex.buckets[b].index(i)
                 assert np.array_equal(ex.send_buf[b].codes(s).cpu().numpy(), ors[i].codes), (t, i)
     assert ex.check() == cf.CF_OK
+
+
+@pytest.mark.parametrize("bits,group", [(2, 128), (4, 64)])
+def test_ring_exchange_matches_oracle(cf, oracle, pg, bits, group):
+    """Algorithm 2's ring on a one-rank group: the rank decodes its own payload
+    (include_self) through libcf; the ring itself has no rounds here."""
+    from activation_residual_compression_02_b200.exchange import RingExchange
+
+    shapes = [(37, 512), (129, 768), (64, 256)]
+    shapes = [(r, c) for r, c in shapes if c % group == 0]
+    ex = RingExchange(shapes, bits=bits, group=group, include_self=True, recon=True)
+    streams = [synth.SlotStream(synth.FLUX.scaled(rows=r, cols=c), slot=i) for i, (r, c) in enumerate(shapes)]
+    ors = [oracle.QuantSlot(bits, group) for _ in shapes]
+    for t in range(4):
+        xs = [s.next() for s in streams]
+        ex.step(t, [x.cuda() for x in xs])
+        for i, x in enumerate(xs):
+            ors[i].step(t, u16(x))
+        torch.cuda.synchronize()
+        for i in range(len(shapes)):
+            assert np.array_equal(ex.cache(0, i).cpu().numpy(), ors[i].cache), (t, i)
+            assert np.array_equal(u16(ex.cache(0, i, bf16=True)), ors[i].recon), (t, i)
+    assert ex.check() == cf.CF_OK
