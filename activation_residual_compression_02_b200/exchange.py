@@ -217,7 +217,7 @@ def ring_pass(local: torch.Tensor, world: int, rank: int, on_receive, pg=None, s
     rank + 1 and receives rank - 1's, so that after round s it holds the buffer
     that started on rank - s; ``on_receive(src, buf)`` is called with it before
     the next round forwards it.  ``spare`` (same size as ``local``) is the
-    second buffer of the double buffer; ``local`` itself is sent in round 1
+    second buffer of the double buffer; ``local`` itself is sent in the first ring round
     and not modified.
     """
     if world <= 1:
@@ -242,7 +242,7 @@ class RingExchange:
     payload that started on rank - s, decompresses it into the cache it keeps
     for that rank's shards (the attention over that K/V block would follow
     here), and forwards it.  Step 0 sends the bf16 activations themselves.
-    With ``include_self`` the rank also decodes its own payload before round 1.
+    With ``include_self`` the rank also decodes its own payload before the first ring round.
     """
 
     def __init__(self, shapes: Sequence[Sequence[int]], bits: int = 2, group: int = 128, sign_scale: int = 0,
