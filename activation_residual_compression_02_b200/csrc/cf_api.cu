@@ -109,6 +109,23 @@ void trace_end(cudaStream_t stream)
 
 namespace {
 
+// Makes the context's device current for the duration of one API call (a
+// process may drive several GPUs, each with its own contexts) and restores
+// the caller's device afterwards.
+struct DeviceGuard {
+    int prev = -1;
+    explicit DeviceGuard(const cf_ctx *ctx)
+    {
+        int cur = 0;
+        if (ctx && cudaGetDevice(&cur) == cudaSuccess && cur != ctx->device && cudaSetDevice(ctx->device) == cudaSuccess)
+            prev = cur;
+    }
+    ~DeviceGuard()
+    {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
 // Sets this thread's tracer for the duration of one API call of a tracing context.
 struct TraceGuard {
     explicit TraceGuard(cf_ctx *ctx)
@@ -348,6 +365,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
 cf_status codec_call(cf_ctx *ctx, const cf_slot *slots, int step, void *stream_, bool sender)
 {
     if (!ctx) return CF_E_ARG;
+    DeviceGuard device(ctx);
     TraceGuard trace(ctx);
     if (step < 0) return fail(ctx, CF_E_ARG, "step must be >= 0");
     const int n = (int)ctx->shapes.size();
@@ -455,6 +473,7 @@ cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
     }
     if (!(ctx->warm_sender && ctx->warm_receiver))
         return fail(ctx, CF_E_STATE, "step %d before the warmup step (step 0) on this context", step);
+    DeviceGuard device(ctx);
     TraceGuard trace(ctx);
     const int n = (int)ctx->shapes.size();
     if (n > 0 && !slots) return fail(ctx, CF_E_ARG, "slots is NULL");
@@ -480,6 +499,7 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
                      void *cuda_stream)
 {
     if (!ctx) return CF_E_ARG;
+    DeviceGuard device(ctx);
     TraceGuard trace(ctx);
     if (ctx->cfg.mode != CF_MODE_LOWRANK) return fail(ctx, CF_E_ARG, "context is not in low-rank mode");
     if (nmat < 0) return fail(ctx, CF_E_ARG, "nmat must be >= 0");
@@ -520,6 +540,7 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
 cf_status cf_check(cf_ctx *ctx, void *cuda_stream)
 {
     if (!ctx) return CF_E_ARG;
+    DeviceGuard device(ctx);
     cudaStream_t stream = (cudaStream_t)cuda_stream;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "stream synchronize");
@@ -574,6 +595,7 @@ cf_status cf_trace_enable(cf_ctx *ctx, int on)
 int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries)
 {
     if (!ctx || max_entries < 0 || (max_entries > 0 && !out)) return -CF_E_ARG;
+    DeviceGuard device(ctx);
     cf::Tracer &t = ctx->tracer;
     struct Sum {
         std::string kernel;
@@ -613,6 +635,7 @@ int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries)
 cf_status cf_destroy(cf_ctx *ctx)
 {
     if (!ctx) return CF_E_ARG;
+    DeviceGuard device(ctx);
     if (ctx->d_status) cudaFree(ctx->d_status);
     delete ctx;
     return CF_OK;

@@ -981,13 +981,21 @@ WsLayout layout(int nmat, int64_t m, int64_t n, int r)
 template <int RP>
 cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
 {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(k_gemm_tf32<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)gemm_smem_bytes<RP>());
-    });
-    if (attr_err != cudaSuccess) return attr_err;
+    // the shared-memory opt-in is a per-device function attribute: set it once per device
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 0 || dev >= 64 || !done[dev]) {
+            e = cudaFuncSetAttribute(k_gemm_tf32<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gemm_smem_bytes<RP>());
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) done[dev] = true;
+        }
+    }
     const char *name = RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>";
     log_launch(name, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP>());
     trace_begin(name, stream);

@@ -62,7 +62,9 @@
  * next cf_check.  The stream-ordered calls allocate no device memory and
  * do not synchronise, so they can be captured into a CUDA graph and replayed
  * (the kernels read the slot pointers given at capture; a quantised step
- * >= 1 is the same launch for every later step).  A context is not
+ * >= 1 is the same launch for every later step).  A context belongs to the
+ * device that was current at cf_create; each call makes that device current
+ * for its duration and restores the caller's.  A context is not
  * thread-safe; separate contexts are independent.  There is no CPU fallback:
  * without a usable sm_100 device cf_create returns CF_E_CUDA.
  */
