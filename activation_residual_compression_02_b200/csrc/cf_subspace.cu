@@ -54,10 +54,10 @@ constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parame
 // Pipeline shape per padded rank RP (the MMA's N).  A stage holds NB boxes of
 // A side by side in K, so each row of A is read NB x 128 contiguous bytes at
 // a time and the per-stage handshakes (barrier, TF32 rounding, fence, MMA
-// batch) are paid once per NB boxes.  Measured on the 57 x 4608 x 3072 pass:
-// one box per stage with 8 stages ran at 5.2-5.6 TB/s; three boxes with four
-// stages at 6.6 TB/s, bit-identical.  RP = 32 needs twice the B space and
-// keeps two boxes with five stages to stay within 227 KB of shared memory.
+// batch) are paid once per NB boxes.  Measured on the 57 x 4608 x 3072 pass
+// with one CTA per SM: one box per stage with 8 stages ran at 5.2-5.6 TB/s;
+// three boxes with four stages at 6.6 TB/s, bit-identical.  RP = 32 needs
+// twice the B space and keeps two boxes with five stages (one CTA per SM).
 //
 // Accumulation in chunks of K.  The tensor core's fp32 accumulator loses a
 // fraction of an ulp towards zero at each accumulating MMA, so one long
@@ -67,11 +67,16 @@ constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parame
 // MMA therefore restarts its accumulator every CH stages (about 1000 of K),
 // and the epilogue adds the chunk sums on the CUDA cores with round to
 // nearest, in chunk order, so the loss stays at its K = 1000 level.
+//
+// At RP = 16 two CTAs share an SM (two boxes x three stages each): more
+// independent TMA streams per SM than one CTA with three boxes x four stages,
+// 0.475 against 0.482 ms per pass over the 57 x 4608 x 3072 batch.
 template <int RP>
 struct GemmCfg {
-    static constexpr int NB = RP == 16 ? 3 : 2;         // boxes of A per stage
-    static constexpr int ST = RP == 16 ? 4 : 5;         // pipeline stages
-    static constexpr int CH = RP == 16 ? 10 : 16;       // stages per accumulation chunk (960 / 1024 of K)
+    static constexpr int NB = 2;                        // boxes of A per stage
+    static constexpr int ST = RP == 16 ? 3 : 5;         // pipeline stages
+    static constexpr int CPS = RP == 16 ? 2 : 1;        // resident CTAs per SM
+    static constexpr int CH = 16;                       // stages per accumulation chunk (1024 of K)
     static constexpr int BK = NB * kBoxK;               // K per stage
     static constexpr int ATile = NB * kBoxBytes;        // A bytes per stage
     static constexpr int BBox = RP * kBoxK * 4;         // one RP x 32 box of Q^T / P^T
@@ -120,7 +125,7 @@ struct GemmSmem {
 
 // ------------------------------------------------------------ the GEMM ----
 template <int RP>
-__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_tf32(const __grid_constant__ GemmParams p)
+__global__ void __launch_bounds__(kGemmThreads, GemmCfg<RP>::CPS) k_gemm_tf32(const __grid_constant__ GemmParams p)
 {
     using C = GemmCfg<RP>;
     constexpr int kStages = C::ST;
@@ -356,6 +361,8 @@ constexpr size_t gemm_smem_bytes()
     return 1024 + (size_t)C::ST * (C::ATile + C::BTile) + sizeof(GemmSmem<C::ST>);
 }
 static_assert(gemm_smem_bytes<16>() <= 227 * 1024, "GEMM shared memory (RP = 16) exceeds 227 KB");
+static_assert(GemmCfg<16>::CPS * (gemm_smem_bytes<16>() + 1024) <= 228 * 1024,
+              "the resident GEMM CTAs (RP = 16) do not fit in one SM's shared memory");
 static_assert(gemm_smem_bytes<32>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
 
 // ------------------------------------------------------ CholeskyQR -------
@@ -1006,7 +1013,8 @@ cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
 
 cudaError_t gemm_launch(GemmParams &gp, int total_tiles, cudaStream_t stream)
 {
-    const int grid = total_tiles < num_sms() ? total_tiles : num_sms();
+    const int cps = gp.rp == 16 ? GemmCfg<16>::CPS : GemmCfg<32>::CPS;
+    const int grid = total_tiles < cps * num_sms() ? total_tiles : cps * num_sms();
     if (grid <= 0) return cudaSuccess;
     return gp.rp == 16 ? gemm_launch_rp<16>(gp, grid, stream) : gemm_launch_rp<32>(gp, grid, stream);
 }
