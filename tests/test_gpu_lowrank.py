@@ -99,6 +99,19 @@ def test_lowrank_matches_oracle(cf, oracle, m, n, r, T):
     check(oracle, As, Q0s, out, T)
 
 
+# Shapes smaller than one tile or one TMA box in one or both dimensions, and
+# the degenerate ranks: r == n (Q spans every column: D = A) and r == m (U is
+# square).
+@pytest.mark.parametrize("m,n,r,T", [(17, 20, 4, 2), (33, 36, 16, 1), (1000, 16, 16, 1), (16, 1000, 16, 2),
+                                     (129, 8, 8, 1)])
+def test_lowrank_small_and_degenerate_shapes(cf, oracle, m, n, r, T):
+    k = 3
+    As = [synth.lowrank_matrix(m, n, r, mat=i, noise=0.01) for i in range(k)]
+    Q0s = [synth.q0(n, r, seed=0, mat=i) for i in range(k)]
+    out = run_gpu(cf, As, Q0s, r, T)
+    check(oracle, As, Q0s, out, T)
+
+
 @pytest.mark.parametrize("k,m,n,r,T", [(8, 1024, 3072, 16, 2), (80, 1000, 128, 8, 1)])
 def test_lowrank_many_tiles_and_matrices(cf, oracle, k, m, n, r, T):
     """Many matrices of many 128-row tiles in one call: the persistent GEMM

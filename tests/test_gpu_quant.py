@@ -356,3 +356,11 @@ def test_bf16_reconstruction_only_where_asked(cf, oracle):
     assert np.array_equal(u16(st.recon[0]), ors[0].recon)
     assert np.array_equal(st.cache[1].cpu().numpy(), ors[1].cache)
     assert np.array_equal(u16(side), expect_side)
+
+
+@pytest.mark.parametrize("bits,ss", [(2, 0), (4, 0), (1, 0), (1, 1)])
+def test_narrowest_rows(cf, oracle, bits, ss):
+    """Rows of a single vector (cols = G = 8) and of two or three groups, with
+    one-row slots: every group is a whole row and lanes of a warp cover
+    several rows."""
+    run_case(cf, oracle, [(3, 8), (1, 16), (7, 24), (1, 8), (65, 8)], 4, bits, 8, ss, w=synth.FLUX)
