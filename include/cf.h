@@ -54,8 +54,8 @@
  * the workspace are caller memory (device pointers).  The library performs
  * no transmission between devices.
  *
- * Concurrency and errors: every call except cf_create, cf_destroy and
- * cf_check is stream-ordered and asynchronous.  Argument, shape, alignment
+ * Concurrency and errors: every call except cf_create, cf_destroy, cf_check
+ * and cf_trace_read is stream-ordered and asynchronous.  Argument, shape, alignment
  * and state errors return before anything is launched and leave all buffers
  * untouched.  Device-side conditions (non-finite scale, a bounded wait that
  * gave up) set bits in the context's status word and are reported by the
