@@ -68,15 +68,17 @@ constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parame
 // and the epilogue adds the chunk sums on the CUDA cores with round to
 // nearest, in chunk order, so the loss stays at its K = 1000 level.
 //
-// At RP = 16 two CTAs share an SM (two boxes x three stages each): more
-// independent TMA streams per SM than one CTA with three boxes x four stages,
-// 0.475 against 0.482 ms per pass over the 57 x 4608 x 3072 batch.
-template <int RP>
+// At RP = 16 and with at least two tiles per SM, two CTAs share an SM (two
+// boxes x three stages each): more independent TMA streams per SM than one
+// CTA with three boxes x four stages, 0.475 against 0.482 ms per pass over the
+// 57 x 4608 x 3072 batch.  With fewer tiles (a few matrices) the one-CTA form
+// is faster (4 matrices: 43.5 / 51.0 against 48.8 / 67.0 us for A Q / A^T P),
+// so the host picks the form by tile count.
+template <int RP, int CPS>
 struct GemmCfg {
-    static constexpr int NB = 2;                        // boxes of A per stage
-    static constexpr int ST = RP == 16 ? 3 : 5;         // pipeline stages
-    static constexpr int CPS = RP == 16 ? 2 : 1;        // resident CTAs per SM
-    static constexpr int CH = 16;                       // stages per accumulation chunk (1024 of K)
+    static constexpr int NB = (RP == 16 && CPS == 1) ? 3 : 2;        // boxes of A per stage
+    static constexpr int ST = RP == 16 ? (CPS == 2 ? 3 : 4) : 5;     // pipeline stages
+    static constexpr int CH = NB == 3 ? 10 : 16;                      // stages per accumulation chunk (960 / 1024 of K)
     static constexpr int BK = NB * kBoxK;               // K per stage
     static constexpr int ATile = NB * kBoxBytes;        // A bytes per stage
     static constexpr int BBox = RP * kBoxK * 4;         // one RP x 32 box of Q^T / P^T
@@ -124,10 +126,10 @@ struct GemmSmem {
 };
 
 // ------------------------------------------------------------ the GEMM ----
-template <int RP>
-__global__ void __launch_bounds__(kGemmThreads, GemmCfg<RP>::CPS) k_gemm_tf32(const __grid_constant__ GemmParams p)
+template <int RP, int CPS>
+__global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_constant__ GemmParams p)
 {
-    using C = GemmCfg<RP>;
+    using C = GemmCfg<RP, CPS>;
     constexpr int kStages = C::ST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -354,16 +356,16 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<RP>::CPS) k_gemm_tf32(co
     }
 }
 
-template <int RP>
+template <int RP, int CPS>
 constexpr size_t gemm_smem_bytes()
 {
-    using C = GemmCfg<RP>;
+    using C = GemmCfg<RP, CPS>;
     return 1024 + (size_t)C::ST * (C::ATile + C::BTile) + sizeof(GemmSmem<C::ST>);
 }
-static_assert(gemm_smem_bytes<16>() <= 227 * 1024, "GEMM shared memory (RP = 16) exceeds 227 KB");
-static_assert(GemmCfg<16>::CPS * (gemm_smem_bytes<16>() + 1024) <= 228 * 1024,
-              "the resident GEMM CTAs (RP = 16) do not fit in one SM's shared memory");
-static_assert(gemm_smem_bytes<32>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
+static_assert(gemm_smem_bytes<16, 1>() <= 227 * 1024, "GEMM shared memory (RP = 16) exceeds 227 KB");
+static_assert(2 * (gemm_smem_bytes<16, 2>() + 1024) <= 228 * 1024,
+              "two GEMM CTAs (RP = 16) do not fit in one SM's shared memory");
+static_assert(gemm_smem_bytes<32, 1>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
 
 // ------------------------------------------------------ CholeskyQR -------
 // Two launches per orthonormalisation.  k_cholqr_factor: CTA (chunk, matrix)
@@ -985,7 +987,7 @@ WsLayout layout(int nmat, int64_t m, int64_t n, int r)
     return L;
 }
 
-template <int RP>
+template <int RP, int CPS>
 cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
 {
     // the shared-memory opt-in is a per-device function attribute: set it once per device
@@ -997,29 +999,35 @@ cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || !done[dev]) {
-            e = cudaFuncSetAttribute(k_gemm_tf32<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)gemm_smem_bytes<RP>());
+            e = cudaFuncSetAttribute(k_gemm_tf32<RP, CPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gemm_smem_bytes<RP, CPS>());
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) done[dev] = true;
         }
     }
     const char *name = RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>";
-    log_launch(name, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP>());
+    log_launch(name, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP, CPS>());
     trace_begin(name, stream);
-    k_gemm_tf32<RP><<<grid, kGemmThreads, gemm_smem_bytes<RP>(), stream>>>(gp);
+    k_gemm_tf32<RP, CPS><<<grid, kGemmThreads, gemm_smem_bytes<RP, CPS>(), stream>>>(gp);
     trace_end(stream);
     return cudaGetLastError();
 }
 
-cudaError_t gemm_launch(GemmParams &gp, int total_tiles, cudaStream_t stream)
+// Resident CTAs per SM for a launch of `total_tiles` tiles (see GemmCfg).
+int gemm_cps(int rp, int64_t total_tiles) { return rp == 16 && total_tiles >= 2 * (int64_t)num_sms() ? 2 : 1; }
+
+cudaError_t gemm_launch(GemmParams &gp, int total_tiles, int cps, cudaStream_t stream)
 {
-    const int cps = gp.rp == 16 ? GemmCfg<16>::CPS : GemmCfg<32>::CPS;
     const int grid = total_tiles < cps * num_sms() ? total_tiles : cps * num_sms();
     if (grid <= 0) return cudaSuccess;
-    return gp.rp == 16 ? gemm_launch_rp<16>(gp, grid, stream) : gemm_launch_rp<32>(gp, grid, stream);
+    if (gp.rp != 16) return gemm_launch_rp<32, 1>(gp, grid, stream);
+    return cps == 2 ? gemm_launch_rp<16, 2>(gp, grid, stream) : gemm_launch_rp<16, 1>(gp, grid, stream);
 }
 
-int gemm_bk(int rp) { return rp == 16 ? GemmCfg<16>::BK : GemmCfg<32>::BK; }
+int gemm_bk(int rp, int cps)
+{
+    return rp != 16 ? GemmCfg<32, 1>::BK : (cps == 2 ? GemmCfg<16, 2>::BK : GemmCfg<16, 1>::BK);
+}
 
 // out_i = A_i Q_i (mn_major = 0) or A_i^T P_i (mn_major = 1) for every matrix.
 cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLayout &L, int mn_major, int out_mode,
@@ -1048,9 +1056,11 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             gp->wait_ns = 20000000ull;
         }
         bool ok;
+        const int cps = gemm_cps(L.rp, (int64_t)cnt * (((!mn_major ? m : n) + kBM - 1) / kBM));
+        const int bk = gemm_bk(L.rp, cps);
         if (!mn_major) {
             gp->tiles_per_mat = (int)((m + kBM - 1) / kBM);
-            gp->ktiles = (int)((n + gemm_bk(L.rp) - 1) / gemm_bk(L.rp));
+            gp->ktiles = (int)((n + bk - 1) / bk);
             gp->out_rows = (int)m;
             gp->out_ld = (int)L.mp;
             ok = make_map3(&gp->tb, ws + L.qt + (size_t)first * L.rp * L.np * 4, n, L.rp, cnt, L.np, L.rp * L.np,
@@ -1064,7 +1074,7 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             }
         } else {
             gp->tiles_per_mat = (int)((n + kBM - 1) / kBM);
-            gp->ktiles = (int)((m + gemm_bk(L.rp) - 1) / gemm_bk(L.rp));
+            gp->ktiles = (int)((m + bk - 1) / bk);
             gp->out_rows = (int)n;
             gp->out_ld = 0;
             ok = make_map3(&gp->tb, ws + L.pt + (size_t)first * L.rp * L.mp * 4, m, L.rp, cnt, L.mp, L.rp * L.mp,
@@ -1081,7 +1091,7 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             err = cudaErrorInvalidValue;
             break;
         }
-        err = gemm_launch(*gp, cnt * gp->tiles_per_mat, stream);
+        err = gemm_launch(*gp, cnt * gp->tiles_per_mat, cps, stream);
     }
     delete gp;
     return err;
