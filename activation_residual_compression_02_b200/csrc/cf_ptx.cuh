@@ -1,5 +1,5 @@
 // cf_ptx.cuh -- thin wrappers over the sm_100a PTX the codec kernels use:
-// mbarriers (with a bounded wait), bulk-async copies, tensor-memory fences.
+// mbarriers (with a bounded wait) and the async-proxy fence.
 #pragma once
 
 #include <stdint.h>
@@ -68,26 +68,6 @@ static __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
             }
         }
     }
-}
-
-// One-dimensional bulk copy global -> shared, completing on `bar` (bytes and
-// both addresses must be multiples of 16).
-static __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                                uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
-            "r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
-// L2 policy for data read once: evict first.
-static __device__ __forceinline__ uint64_t policy_evict_first()
-{
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
 }
 
 static __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
