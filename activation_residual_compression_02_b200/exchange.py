@@ -210,20 +210,23 @@ class PatchAllGather:
         return worst
 
 
-def ring_pass(local: torch.Tensor, world: int, rank: int, on_receive, pg=None, spare: Optional[torch.Tensor] = None):
+def ring_pass(local: torch.Tensor, world: int, rank: int, on_receive, pg=None,
+              spares: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
     """Algorithm 2's ring schedule for one flat buffer per rank.
 
     In round s (s = 1 .. world - 1) every rank sends the buffer it holds to
     rank + 1 and receives rank - 1's, so that after round s it holds the buffer
     that started on rank - s; ``on_receive(src, buf)`` is called with it before
-    the next round forwards it.  ``spare`` (same size as ``local``) is the
-    second buffer of the double buffer; ``local`` itself is sent in the first ring round
-    and not modified.
+    the next round forwards it.  The received buffers alternate between the
+    two ``spares`` (each the size of ``local``; allocated when not given), so
+    ``local`` itself is only sent, in the first ring round, and not modified.
     """
     if world <= 1:
         return
     nxt, prv = (rank + 1) % world, (rank - 1) % world
-    bufs = [local, torch.empty_like(local) if spare is None else spare, torch.empty_like(local)]
+    if spares is None:
+        spares = (torch.empty_like(local), torch.empty_like(local))
+    bufs = [local, spares[0], spares[1]]
     cur = 0
     for s in range(1, world):
         dst = 1 if cur != 1 else 2
@@ -257,7 +260,7 @@ class RingExchange:
         self.send_ctx = Context(self.shapes, bits=bits, group=group, sign_scale=sign_scale)
         self.send_state = QuantState(self.shapes, bits, group, device=self.device)
         self.send_buf = PayloadBuffer(self.shapes, bits, group, device=self.device)
-        self.spare = torch.empty_like(self.send_buf.data)
+        self.spares = (torch.empty_like(self.send_buf.data), torch.empty_like(self.send_buf.data))
         self.peers = [p for p in range(self.world) if include_self or p != self.rank]
         self.recv_ctx = {p: Context(self.shapes, bits=bits, group=group, sign_scale=sign_scale) for p in self.peers}
         self.recv_state = {p: QuantState(self.shapes, bits, group, device=self.device, recon=recon)
@@ -299,7 +302,7 @@ class RingExchange:
         if self.include_self:
             self._decode(t, self.rank, local)
         ring_pass(local, self.world, self.rank, lambda src, buf: self._decode(t, src, buf), self.pg,
-                  spare=None if t == 0 else self.spare)
+                  spares=None if t == 0 else self.spares)
 
     def check(self) -> int:
         worst = CF_OK
