@@ -47,7 +47,9 @@ _lib: Optional[ctypes.CDLL] = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        # CF_ORACLE_LIB names another build of this source (the mutation test
+        # runs the pins against deliberately broken copies of the oracle)
+        _lib = ctypes.CDLL(os.environ.get("CF_ORACLE_LIB") or build())
         P, I64, I, U32P = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)
         _lib.cfo_warmup_sender.argtypes = [I64, P, P, P]
         _lib.cfo_warmup_receiver.argtypes = [I64, P, P]
