@@ -19,6 +19,7 @@ CF_OK, CF_E_ARG, CF_E_SHAPE, CF_E_ALIGN, CF_E_STATE, CF_E_NOMEM, CF_E_CUDA, CF_E
 STATUS_NAMES = {0: "CF_OK", 1: "CF_E_ARG", 2: "CF_E_SHAPE", 3: "CF_E_ALIGN", 4: "CF_E_STATE", 5: "CF_E_NOMEM",
                 6: "CF_E_CUDA", 7: "CF_E_NONFINITE", 8: "CF_E_TIMEOUT"}
 CF_MODE_QUANT, CF_MODE_LOWRANK = 0, 1
+CF_PRECISION_AUTO, CF_PRECISION_TF32, CF_PRECISION_SPLIT = 0, 1, 2
 
 EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
             "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
@@ -29,7 +30,7 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 class cf_config(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int), ("bits", ctypes.c_int), ("group", ctypes.c_int),
                 ("sign_scale", ctypes.c_int), ("rank", ctypes.c_int), ("iters", ctypes.c_int),
-                ("state_bf16", ctypes.c_int), ("warm_start", ctypes.c_int)]
+                ("state_bf16", ctypes.c_int), ("warm_start", ctypes.c_int), ("precision", ctypes.c_int)]
 
 
 class cf_shape(ctypes.Structure):
@@ -145,9 +146,10 @@ class Context:
     """A libcf context (``cf_create`` ... ``cf_destroy``)."""
 
     def __init__(self, shapes: Sequence[Sequence[int]], mode: int = CF_MODE_QUANT, bits: int = 2, group: int = 128,
-                 sign_scale: int = 0, rank: int = 16, iters: int = 2, state_bf16: int = 0, warm_start: int = 0):
+                 sign_scale: int = 0, rank: int = 16, iters: int = 2, state_bf16: int = 0, warm_start: int = 0,
+                 precision: int = CF_PRECISION_AUTO):
         L = lib()
-        self.cfg = cf_config(mode, bits, group, sign_scale, rank, iters, state_bf16, warm_start)
+        self.cfg = cf_config(mode, bits, group, sign_scale, rank, iters, state_bf16, warm_start, precision)
         self.shapes = [tuple(int(v) for v in s) for s in shapes]
         arr = (cf_shape * max(1, len(self.shapes)))(*[cf_shape(r, c) for r, c in self.shapes])
         h = ctypes.c_void_p()
@@ -212,7 +214,7 @@ class Context:
                 V: List[torch.Tensor], E: Optional[List[torch.Tensor]] = None, C: Optional[List[torch.Tensor]] = None,
                 stream: Optional[torch.cuda.Stream] = None):
         nmat = len(A)
-        m, n = (A[0].shape[0], A[0].shape[1]) if nmat else (0, 0)
+        _, m, n = _check_lowrank_tensors(A, Q0, U, R, V, E, C, self.cfg.rank)
         st = lib().cf_lowrank(self._h, nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R), _parr(V), _parr(E),
                               _parr(C), _stream_handle(stream))
         self._raise(st, "cf_lowrank")
@@ -261,15 +263,50 @@ def cf_lowrank(ctx: Context, A, Q0, U, R, V, E=None, C=None, stream=None):
     ctx.lowrank(A, Q0, U, R, V, E, C, stream)
 
 
-def cf_lowrank_noalloc(A, Q0, U, R, V, E=None, C=None, rank: int = 16, iters: int = 2, stream=None) -> int:
+def _check_lowrank_tensors(A, Q0, U, R, V, E, C, r: int):
+    """Device, dtype and shape of every tensor of a low-rank call (the C ABI
+    takes raw pointers, so a wrong dtype or shape would read or write out of
+    bounds).  Returns (device, m, n)."""
+    nmat = len(A)
+    if nmat == 0:
+        return None, 0, 0
+    if A[0].dim() != 2:
+        raise ValueError("A[i] must be [m, n]")
+    dev = A[0].device
+    m, n = int(A[0].shape[0]), int(A[0].shape[1])
+    want = {"A": (m, n), "Q0": (n, r), "U": (m, r), "R": (r, r), "V": (n, r), "E": (m, n), "C": (m, n)}
+    for name, ts in (("A", A), ("Q0", Q0), ("U", U), ("R", R), ("V", V), ("E", E), ("C", C)):
+        if ts is None:
+            continue
+        if len(ts) != nmat:
+            raise ValueError(f"{name} must hold {nmat} tensors")
+        for i, t in enumerate(ts):
+            if t.device != dev:
+                raise ValueError(f"{name}[{i}] is on {t.device}, A[0] on {dev}")
+            if t.dtype != torch.float32:
+                raise ValueError(f"{name}[{i}] must be float32, not {t.dtype}")
+            if tuple(t.shape) != want[name]:
+                raise ValueError(f"{name}[{i}] must have shape {list(want[name])}, not {list(t.shape)}")
+    return dev, m, n
+
+
+def cf_lowrank_noalloc(A, Q0, U, R, V, E=None, C=None, rank: int = 16, iters: int = 2, stream=None,
+                       precision: int = CF_PRECISION_AUTO) -> int:
     """cf_lowrank without a context or workspace, for callers that cannot
     allocate device memory: the scratch is a fixed 8 MiB device array inside
-    libcf.  Synchronous; returns the C status (CF_OK, CF_E_NOMEM when the call
-    does not fit the scratch, ...)."""
-    cfg = cf_config(CF_MODE_LOWRANK, 0, 0, 0, rank, iters, 0, 0)
+    libcf.  Runs on the device of A[0] (made current for the call); every
+    tensor must be a float32 tensor of that device with its call shape.
+    Synchronous; returns the C status (CF_OK, CF_E_NOMEM when the call does
+    not fit the scratch, ...)."""
+    cfg = cf_config(CF_MODE_LOWRANK, 0, 0, 0, rank, iters, 0, 0, precision)
     nmat = len(A)
-    m, n = (A[0].shape[0], A[0].shape[1]) if nmat else (0, 0)
-    return int(lib().cf_lowrank_noalloc(ctypes.byref(cfg), nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R),
+    dev, m, n = _check_lowrank_tensors(A, Q0, U, R, V, E, C, rank)
+    L = lib()
+    if dev is None:
+        return int(L.cf_lowrank_noalloc(ctypes.byref(cfg), 0, 0, 0, None, None, None, None, None, None, None,
+                                        _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        return int(L.cf_lowrank_noalloc(ctypes.byref(cfg), nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R),
                                         _parr(V), _parr(E), _parr(C), _stream_handle(stream)))
 
 

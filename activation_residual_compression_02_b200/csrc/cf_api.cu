@@ -165,6 +165,7 @@ cf_status validate_config(const cf_config *c, std::string &why)
         if (c->sign_scale != 0 && c->sign_scale != 1) { why = "sign_scale must be 0 or 1"; return CF_E_ARG; }
         if (c->state_bf16 != 0 && c->state_bf16 != 1) { why = "state_bf16 must be 0 or 1"; return CF_E_ARG; }
         if (c->warm_start != 0) { why = "warm_start is a low-rank-mode option"; return CF_E_ARG; }
+        if (c->precision != 0) { why = "precision is a low-rank-mode option"; return CF_E_ARG; }
         return CF_OK;
     }
     if (c->mode == CF_MODE_LOWRANK) {
@@ -172,6 +173,10 @@ cf_status validate_config(const cf_config *c, std::string &why)
         if (c->warm_start != 0 && c->warm_start != 1) { why = "warm_start must be 0 or 1"; return CF_E_ARG; }
         if (c->rank < 1 || c->rank > 32) { why = "rank must be in [1, 32]"; return CF_E_ARG; }
         if (c->iters < 0 || c->iters > 1000) { why = "iters must be in [0, 1000]"; return CF_E_ARG; }
+        if (c->precision < CF_PRECISION_AUTO || c->precision > CF_PRECISION_SPLIT) {
+            why = "precision must be CF_PRECISION_AUTO, _TF32 or _SPLIT";
+            return CF_E_ARG;
+        }
         return CF_OK;
     }
     why = "mode must be CF_MODE_QUANT or CF_MODE_LOWRANK";
@@ -205,8 +210,10 @@ size_t lowrank_mode_bytes(const cf_ctx *ctx)
 {
     size_t algo = 0;
     for_each_run(ctx->shapes, [&](size_t i, size_t j) {
-        const size_t b = cf::lowrank_workspace_bytes((int)(j - i), ctx->shapes[i].rows, ctx->shapes[i].cols,
-                                                     ctx->cfg.rank);
+        const cf_shape &sh = ctx->shapes[i];
+        const size_t b = cf::lowrank_workspace_bytes((int)(j - i), sh.rows, sh.cols, ctx->cfg.rank,
+                                                     cf::lowrank_split(ctx->cfg.precision, sh.rows, sh.cols,
+                                                                       ctx->cfg.rank));
         if (b > algo) algo = b;
     });
     return lowrank_residual_bytes(ctx) + algo;
@@ -351,6 +358,7 @@ cf_status run_lowrank_mode(cf_ctx *ctx, const cf_slot *slots, bool sender, cudaS
         plan.n = sh.cols;
         plan.r = ctx->cfg.rank;
         plan.T = ctx->cfg.iters;
+        plan.split = cf::lowrank_split(ctx->cfg.precision, sh.rows, sh.cols, ctx->cfg.rank);
         plan.ws = algo_ws;
         plan.ws_bytes = ctx->ws_bytes - (size_t)(algo_ws - (char *)ctx->ws);
         plan.status = ctx->d_status;
@@ -398,7 +406,7 @@ cf_status codec_call(cf_ctx *ctx, const cf_slot *slots, int step, void *stream_,
 extern "C" {
 
 cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes, cf_ctx **out)
-{
+try {
     if (!out) return CF_E_ARG;
     *out = nullptr;
     if (!config || nslots < 0 || (nslots > 0 && !shapes)) return CF_E_ARG;
@@ -423,7 +431,12 @@ cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes,
     if (!ctx) return CF_E_NOMEM;
     ctx->cfg = *config;
     ctx->device = dev;
-    ctx->shapes.assign(shapes, shapes + nslots);
+    try {
+        ctx->shapes.assign(shapes, shapes + nslots);
+    } catch (const std::bad_alloc &) {
+        delete ctx;
+        return CF_E_NOMEM;
+    }
     if (cudaMalloc(&ctx->d_status, 256) != cudaSuccess) {
         delete ctx;
         return CF_E_NOMEM;
@@ -435,6 +448,10 @@ cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes,
     }
     *out = ctx;
     return CF_OK;
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;   // a host allocation failed: no C++ exception crosses the C ABI
+} catch (...) {
+    return CF_E_ARG;
 }
 
 size_t cf_workspace_bytes(const cf_ctx *ctx)
@@ -454,17 +471,25 @@ cf_status cf_set_workspace(cf_ctx *ctx, void *dev_ptr, size_t bytes)
 }
 
 cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream)
-{
+try {
     return codec_call(ctx, slots, step, cuda_stream, true);
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;
+} catch (...) {
+    return CF_E_ARG;
 }
 
 cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream)
-{
+try {
     return codec_call(ctx, slots, step, cuda_stream, false);
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;
+} catch (...) {
+    return CF_E_ARG;
 }
 
 cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream)
-{
+try {
     if (!ctx) return CF_E_ARG;
     if (step == 0 || ctx->cfg.mode != CF_MODE_QUANT) {
         cf_status st = codec_call(ctx, slots, step, cuda_stream, true);
@@ -486,18 +511,23 @@ cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
     cf_status st = run_quant(ctx, slots, cf::QuantOp::Loopback, (cudaStream_t)cuda_stream);
     if (st == CF_OK) ctx->err.clear();
     return st;
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;
+} catch (...) {
+    return CF_E_ARG;
 }
 
 size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_t n)
 {
     if (!ctx || ctx->cfg.mode != CF_MODE_LOWRANK || nmat < 0 || m < ctx->cfg.rank || n < ctx->cfg.rank) return 0;
-    return cf::lowrank_workspace_bytes(nmat, m, n, ctx->cfg.rank);
+    return cf::lowrank_workspace_bytes(nmat, m, n, ctx->cfg.rank,
+                                       cf::lowrank_split(ctx->cfg.precision, m, n, ctx->cfg.rank));
 }
 
 cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *const *A, const float *const *Q0,
                      float *const *U, float *const *R, float *const *V, float *const *E_opt, float *const *C_opt,
                      void *cuda_stream)
-{
+try {
     if (!ctx) return CF_E_ARG;
     DeviceGuard device(ctx);
     TraceGuard trace(ctx);
@@ -509,7 +539,8 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
     if (m < r || n < r) return fail(ctx, CF_E_SHAPE, "m and n must be >= rank");
     if (n % 4 != 0) return fail(ctx, CF_E_SHAPE, "n must be a multiple of 4 (16-byte rows)");
     if (m > ((int64_t)1 << 40) / n) return fail(ctx, CF_E_SHAPE, "matrix too large");
-    const size_t need = cf::lowrank_workspace_bytes(nmat, m, n, r);
+    const bool split = cf::lowrank_split(ctx->cfg.precision, m, n, r);
+    const size_t need = cf::lowrank_workspace_bytes(nmat, m, n, r, split);
     if (!ctx->ws || ctx->ws_bytes < need)
         return fail(ctx, CF_E_NOMEM, "cf_lowrank needs %zu bytes of workspace (cf_set_workspace)", need);
     std::vector<cf::LowrankMat> mats(nmat);
@@ -528,6 +559,7 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
     plan.n = n;
     plan.r = r;
     plan.T = ctx->cfg.iters;
+    plan.split = split;
     plan.ws = ctx->ws;
     plan.ws_bytes = ctx->ws_bytes;
     plan.status = ctx->d_status;
@@ -535,6 +567,10 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
     if (e != cudaSuccess) return cuda_fail(ctx, e, "cf_lowrank");
     ctx->err.clear();
     return CF_OK;
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;
+} catch (...) {
+    return CF_E_ARG;
 }
 
 cf_status cf_check(cf_ctx *ctx, void *cuda_stream)
@@ -574,7 +610,7 @@ const char *cf_last_error(const cf_ctx *ctx)
 }
 
 cf_status cf_resume(cf_ctx *ctx, int64_t steps_done)
-{
+try {
     if (!ctx) return CF_E_ARG;
     if (steps_done < 0) return fail(ctx, CF_E_ARG, "steps_done must be >= 0");
     ctx->warm_sender = true;
@@ -582,6 +618,10 @@ cf_status cf_resume(cf_ctx *ctx, int64_t steps_done)
     ctx->lowrank_steps = steps_done;   // compressed steps after the warmup
     ctx->err.clear();
     return CF_OK;
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;
+} catch (...) {
+    return CF_E_ARG;
 }
 
 cf_status cf_trace_enable(cf_ctx *ctx, int on)
@@ -593,7 +633,7 @@ cf_status cf_trace_enable(cf_ctx *ctx, int on)
 }
 
 int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries)
-{
+try {
     if (!ctx || max_entries < 0 || (max_entries > 0 && !out)) return -CF_E_ARG;
     DeviceGuard device(ctx);
     cf::Tracer &t = ctx->tracer;
@@ -630,6 +670,10 @@ int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries)
         return -CF_E_CUDA;
     }
     return (int)sums.size();
+} catch (const std::bad_alloc &) {
+    return -CF_E_NOMEM;
+} catch (...) {
+    return -CF_E_ARG;
 }
 
 cf_status cf_destroy(cf_ctx *ctx)

@@ -68,12 +68,17 @@ struct LowrankPlan {
     int nmat;
     int64_t m, n;
     int r, T;
+    bool split;        // split (3xTF32) products, see lowrank_split
     void *ws;          // device workspace
     size_t ws_bytes;
     uint32_t *status;
 };
 
-size_t lowrank_workspace_bytes(int nmat, int64_t m, int64_t n, int r);
+// Whether the products with A run split (3xTF32) for a config precision
+// (CF_PRECISION_*) and an m x n problem of rank r.
+bool lowrank_split(int precision, int64_t m, int64_t n, int r);
+
+size_t lowrank_workspace_bytes(int nmat, int64_t m, int64_t n, int r, bool split);
 
 // Runs Algorithm 3 (and the apply step) for plan.nmat matrices.  `mats` is a
 // host array.  Returns a cudaError_t from the launches.

@@ -12,6 +12,7 @@
 // keeps for the life of the process.  The caller still owns A, Q0 and the
 // outputs.
 #include <mutex>
+#include <new>
 
 #include "cf_internal.h"
 
@@ -52,6 +53,19 @@ cudaError_t scratch_address(void **out)
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// True when p is device (or managed) memory of device `dev`.  The kernels run
+// on the current device, so a pointer into another GPU's memory, or a host
+// pointer, is refused before anything is launched.
+bool on_device(const void *p, int dev)
+{
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();   // the query's error is the answer, not a sticky state
+        return false;
+    }
+    return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+}
+
 }  // namespace
 }  // namespace cf
 
@@ -59,18 +73,20 @@ extern "C" cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64
                                         const float *const *A, const float *const *Q0, float *const *U,
                                         float *const *R, float *const *V, float *const *E_opt,
                                         float *const *C_opt, void *cuda_stream)
-{
+try {
     using namespace cf;
     if (!config || config->mode != CF_MODE_LOWRANK) return CF_E_ARG;
     const int r = config->rank, T = config->iters;
     if (r < 1 || r > 32 || T < 0 || T > 1000 || nmat < 0) return CF_E_ARG;
+    if (config->precision < CF_PRECISION_AUTO || config->precision > CF_PRECISION_SPLIT) return CF_E_ARG;
     if (nmat == 0) return CF_OK;
     if (nmat > kMaxNoallocMats) return CF_E_NOMEM;
     if (!A || !Q0 || !U || !R || !V) return CF_E_ARG;
     if (m < r || n < r || m > INT32_MAX || n > INT32_MAX) return CF_E_SHAPE;
     if (n % 4 != 0) return CF_E_SHAPE;
     // Reject calls whose Algorithm 3 buffers do not fit the fixed scratch.
-    const size_t need = lowrank_workspace_bytes(nmat, m, n, r);
+    const bool split = lowrank_split(config->precision, m, n, r);
+    const size_t need = lowrank_workspace_bytes(nmat, m, n, r, split);
     if (need > CF_NOALLOC_SCRATCH_BYTES - kStatusBytes) return CF_E_NOMEM;
     LowrankMat mats[kMaxNoallocMats];
     for (int i = 0; i < nmat; ++i) {
@@ -81,6 +97,14 @@ extern "C" cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64
             !aligned16(E) || !aligned16(C))
             return CF_E_ALIGN;
         mats[i] = LowrankMat{A[i], Q0[i], U[i], R[i], V[i], E, C};
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CF_E_CUDA;
+    for (int i = 0; i < nmat; ++i) {
+        const LowrankMat &t = mats[i];
+        if (!on_device(t.A, dev) || !on_device(t.Q0, dev) || !on_device(t.U, dev) || !on_device(t.R, dev) ||
+            !on_device(t.V, dev) || (t.E && !on_device(t.E, dev)) || (t.C && !on_device(t.C, dev)))
+            return CF_E_ARG;
     }
     void *scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return CF_E_CUDA;
@@ -95,6 +119,7 @@ extern "C" cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64
     plan.n = n;
     plan.r = r;
     plan.T = T;
+    plan.split = split;
     plan.ws = (char *)scratch + kStatusBytes;
     plan.ws_bytes = CF_NOALLOC_SCRATCH_BYTES - kStatusBytes;
     plan.status = status;
@@ -106,4 +131,9 @@ extern "C" cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64
     if (word & kStatusTimeout) return CF_E_TIMEOUT;
     if (word & (kStatusNonfinite | kStatusNotSpd)) return CF_E_NONFINITE;
     return CF_OK;
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;   // a host allocation failed: no C++ exception crosses the C ABI
+} catch (...) {
+    return CF_E_ARG;
 }
+

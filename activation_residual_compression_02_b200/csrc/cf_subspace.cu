@@ -74,17 +74,28 @@ constexpr int kMaxGemmMats = 160;   // 128-byte tensor maps in the kernel parame
 // 57 x 4608 x 3072 batch.  With fewer tiles (a few matrices) the one-CTA form
 // is faster (4 matrices: 43.5 / 51.0 against 48.8 / 67.0 us for A Q / A^T P),
 // so the host picks the form by tile count.
-template <int RP, int CPS>
+//
+// Split products (SPLIT, "3xTF32"): each operand is carried as two TF32
+// parts, x = hi + lo with hi = tf32(x) and lo = tf32(x - hi), and each
+// product is hi_A hi_B + (lo_A hi_B + hi_A lo_B), dropping lo_A lo_B (about
+// 2^-22 of the product): close to fp32 accuracy, for iterations that are
+// ill-conditioned with respect to operand rounding.  The converter warps
+// write lo_A beside hi_A; the producer loads hi_B and lo_B blocks.  The two
+// correction products accumulate into their own TMEM accumulator, so the
+// main accumulation chain is as long as in the plain form; the epilogue adds
+// the two.  The stages are smaller (A takes twice the shared memory).
+template <int RP, int CPS, bool SPLIT = false>
 struct GemmCfg {
-    static constexpr int NB = (RP == 16 && CPS == 1) ? 3 : 2;        // boxes of A per stage
-    static constexpr int ST = RP == 16 ? (CPS == 2 ? 3 : 4) : 5;     // pipeline stages
-    static constexpr int CH = NB == 3 ? 10 : 16;                      // stages per accumulation chunk (960 / 1024 of K)
+    static constexpr int NB = SPLIT ? (RP == 16 ? 2 : 1) : ((RP == 16 && CPS == 1) ? 3 : 2);   // boxes of A per stage
+    static constexpr int ST = SPLIT ? (RP == 16 ? 3 : 5) : (RP == 16 ? (CPS == 2 ? 3 : 4) : 5); // pipeline stages
     static constexpr int BK = NB * kBoxK;               // K per stage
-    static constexpr int ATile = NB * kBoxBytes;        // A bytes per stage
+    static constexpr int CH = 1024 / BK;                // stages per accumulation chunk (960 or 1024 of K)
+    static constexpr int NP = SPLIT ? 2 : 1;            // TF32 parts per operand
+    static constexpr int ATile = NB * kBoxBytes;        // A bytes per stage and part
     static constexpr int BBox = RP * kBoxK * 4;         // one RP x 32 box of Q^T / P^T
-    static constexpr int BTile = NB * BBox;
+    static constexpr int BTile = NB * BBox;             // B bytes per stage and part
+    static constexpr int TmemCols = SPLIT ? 128 : 64;   // two accumulators of up to 32 columns (+ two for corrections)
 };
-constexpr int kTmemCols = 64;       // two accumulators of up to 32 columns
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 struct __align__(64) GemmMat {
@@ -94,7 +105,9 @@ struct __align__(64) GemmMat {
 struct GemmParams {
     GemmMat mat[kMaxGemmMats];
     CUtensorMap tb;    // B^T blocks of every matrix, 3-D {K, rp, matrix}: Q^T or P^T (K-major)
+    CUtensorMap tb_lo; // split products: the lo parts of the same blocks
     float *out;        // output of matrix 0; matrix i at out + i * out_stride
+    float *out_lo;     // split products, out_mode 0: lo parts of the transposed output (same strides)
     int64_t out_stride;
     int nmat;
     int tiles_per_mat;
@@ -126,16 +139,17 @@ struct GemmSmem {
 };
 
 // ------------------------------------------------------------ the GEMM ----
-template <int RP, int CPS>
+template <int RP, int CPS, bool SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_constant__ GemmParams p)
 {
-    using C = GemmCfg<RP, CPS>;
+    using C = GemmCfg<RP, CPS, SPLIT>;
     constexpr int kStages = C::ST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sA = base;                                   // kStages x NB boxes of A
-    uint8_t *sB = base + kStages * C::ATile;              // kStages x NB boxes of Q^T / P^T
-    GemmSmem<kStages> *S = (GemmSmem<kStages> *)(sB + kStages * C::BTile);
+    uint8_t *sA = base;                                   // kStages x NB boxes of A (hi part)
+    uint8_t *sAlo = sA + kStages * C::ATile;              // SPLIT: the lo parts, same layout
+    uint8_t *sB = sA + C::NP * kStages * C::ATile;        // kStages x NP x NB boxes of Q^T / P^T
+    GemmSmem<kStages> *S = (GemmSmem<kStages> *)(sB + C::NP * kStages * C::BTile);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -157,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S->tmem_base)),
-                     "r"(kTmemCols)
+                     "r"(C::TmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -167,7 +181,7 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
     const uint32_t tmem = S->tmem_base;
     volatile int *abort_flag = &S->abort_flag;
     const unsigned long long wait_ns = p.wait_ns;
-    const uint32_t stage_bytes = (uint32_t)(C::ATile + C::BTile);
+    const uint32_t stage_bytes = (uint32_t)(C::ATile + C::NP * C::BTile);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -200,7 +214,9 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
                             for (int j = 0; j < 4; ++j)
                                 tma_load_2d(a + j * 4096, &M.ta, mt * kBM + 32 * j, k0, &S->full[s]);
                         }
-                        tma_load_3d(sB + s * C::BTile + h * C::BBox, &p.tb, k0, 0, mi, &S->full[s]);
+                        uint8_t *b = sB + s * C::NP * C::BTile + h * C::BBox;
+                        tma_load_3d(b, &p.tb, k0, 0, mi, &S->full[s]);
+                        if (SPLIT) tma_load_3d(b + C::BTile, &p.tb_lo, k0, 0, mi, &S->full[s]);
                     }
                 }
             }
@@ -227,6 +243,7 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
                 }
                 tc_fence_after();
                 const uint32_t dtm = tmem + (uint32_t)(b * 32);
+                const uint32_t dcor = dtm + 64;   // SPLIT: accumulator of the correction products
                 for (int kt = k0; kt < k1; ++kt, ++it) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -237,7 +254,7 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
                     tc_fence_after();
                     if (lane == 0) {
                         const uint32_t a0 = smem_u32(sA + s * C::ATile);
-                        const uint32_t b0 = smem_u32(sB + s * C::BTile);
+                        const uint32_t b0 = smem_u32(sB + s * C::NP * C::BTile);
 #pragma unroll
                         for (int k = 0; k < C::BK / 8; ++k) {
                             // K step k: box k / 4, 8-element slice k % 4 of it
@@ -246,7 +263,17 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
                             const uint64_t ad = p.mn_major ? smem_desc(ah + kk * 1024, 4096, 512, kLayoutSw128Atom32)
                                                            : smem_desc(ah + kk * 32, 16, 1024, kLayoutSw128);
                             const uint64_t bd = smem_desc(bh + kk * 32, 16, 1024, kLayoutSw128);
-                            tc_mma_tf32(dtm, ad, bd, idesc, (kt > k0 || k > 0) ? 1u : 0u);
+                            const uint32_t acc = (kt > k0 || k > 0) ? 1u : 0u;
+                            if (SPLIT) {
+                                // the lo parts sit kStages * ATile (A) and BTile (B) bytes further on
+                                const uint32_t alo = ah + (uint32_t)(kStages * C::ATile);
+                                const uint64_t adl = p.mn_major ? smem_desc(alo + kk * 1024, 4096, 512, kLayoutSw128Atom32)
+                                                                : smem_desc(alo + kk * 32, 16, 1024, kLayoutSw128);
+                                const uint64_t bdl = smem_desc(bh + (uint32_t)C::BTile + kk * 32, 16, 1024, kLayoutSw128);
+                                tc_mma_tf32(dcor, adl, bd, idesc, acc);
+                                tc_mma_tf32(dcor, ad, bdl, idesc, 1u);
+                            }
+                            tc_mma_tf32(dtm, ad, bd, idesc, acc);
                         }
                         tc_commit(&S->empty[s]);
                     }
@@ -277,14 +304,15 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
                     break;
                 }
                 float4 *a = (float4 *)(sA + s * C::ATile);
+                float4 *alo = (float4 *)(sAlo + s * C::ATile);
 #pragma unroll
                 for (int i = 0; i < C::ATile / 16 / 128; ++i) {
-                    float4 v = a[ct + 128 * i];
-                    v.x = round_tf32(v.x);
-                    v.y = round_tf32(v.y);
-                    v.z = round_tf32(v.z);
-                    v.w = round_tf32(v.w);
-                    a[ct + 128 * i] = v;
+                    const float4 v = a[ct + 128 * i];
+                    const float4 h = make_float4(round_tf32(v.x), round_tf32(v.y), round_tf32(v.z), round_tf32(v.w));
+                    a[ct + 128 * i] = h;
+                    if (SPLIT)
+                        alo[ct + 128 * i] = make_float4(round_tf32(v.x - h.x), round_tf32(v.y - h.y),
+                                                        round_tf32(v.z - h.z), round_tf32(v.w - h.w));
                 }
                 fence_proxy_async();
                 mbar_arrive(&S->conv[s]);
@@ -320,6 +348,22 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
 #pragma unroll
                     for (int c = 0; c < 16; ++c) v[16 + c] = hi[c];
                 }
+                if (SPLIT) {
+                    // chunk = main + corrections, one rounding
+                    uint32_t w[32];
+                    uint32_t t16[16];
+                    tc_ld16(taddr + 64, t16);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) w[c] = t16[c];
+                    if (RP > 16) {
+                        tc_ld16(taddr + 80, t16);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) w[16 + c] = t16[c];
+                    }
+                    tc_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < RP; ++c) v[c] = __float_as_uint(__fadd_rn(__uint_as_float(v[c]), __uint_as_float(w[c])));
+                }
                 tc_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&S->acce[b]);
@@ -336,8 +380,11 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
             if (row < p.out_rows) {
                 if (p.out_mode == 0) {
 #pragma unroll
-                    for (int c = 0; c < RP; ++c)
-                        out[(int64_t)c * p.out_ld + row] = round_tf32(acc[c]);
+                    for (int c = 0; c < RP; ++c) {
+                        const float hi = round_tf32(acc[c]);
+                        out[(int64_t)c * p.out_ld + row] = hi;
+                        if (SPLIT) p.out_lo[(int64_t)mi * p.out_stride + (int64_t)c * p.out_ld + row] = round_tf32(acc[c] - hi);
+                    }
                 } else {
                     float4 *o = (float4 *)(out + (int64_t)row * RP);
 #pragma unroll
@@ -352,20 +399,22 @@ __global__ void __launch_bounds__(kGemmThreads, CPS) k_gemm_tf32(const __grid_co
     __syncthreads();
     tc_fence_after();
     if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TmemCols) : "memory");
     }
 }
 
-template <int RP, int CPS>
+template <int RP, int CPS, bool SPLIT>
 constexpr size_t gemm_smem_bytes()
 {
-    using C = GemmCfg<RP, CPS>;
-    return 1024 + (size_t)C::ST * (C::ATile + C::BTile) + sizeof(GemmSmem<C::ST>);
+    using C = GemmCfg<RP, CPS, SPLIT>;
+    return 1024 + (size_t)C::NP * C::ST * (C::ATile + C::BTile) + sizeof(GemmSmem<C::ST>);
 }
-static_assert(gemm_smem_bytes<16, 1>() <= 227 * 1024, "GEMM shared memory (RP = 16) exceeds 227 KB");
-static_assert(2 * (gemm_smem_bytes<16, 2>() + 1024) <= 228 * 1024,
+static_assert(gemm_smem_bytes<16, 1, false>() <= 227 * 1024, "GEMM shared memory (RP = 16) exceeds 227 KB");
+static_assert(2 * (gemm_smem_bytes<16, 2, false>() + 1024) <= 228 * 1024,
               "two GEMM CTAs (RP = 16) do not fit in one SM's shared memory");
-static_assert(gemm_smem_bytes<32, 1>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
+static_assert(gemm_smem_bytes<32, 1, false>() <= 227 * 1024, "GEMM shared memory (RP = 32) exceeds 227 KB");
+static_assert(gemm_smem_bytes<16, 1, true>() <= 227 * 1024, "split GEMM shared memory (RP = 16) exceeds 227 KB");
+static_assert(gemm_smem_bytes<32, 1, true>() <= 227 * 1024, "split GEMM shared memory (RP = 32) exceeds 227 KB");
 
 // ------------------------------------------------------ CholeskyQR -------
 // Two launches per orthonormalisation.  k_cholqr_factor: CTA (chunk, matrix)
@@ -384,6 +433,7 @@ struct CholMat {
     unsigned int *count;  // chunks done (zero before the launch; the last CTA resets it)
     double *Rinv;         // R^{-1} [32 x 32], upper triangular
     float *Qt;            // mode Q: rounded transposed output [rp x qt_ld] (rows >= r stay zero)
+    float *Qt_lo;         // mode Q, split products: the lo parts of Qt (or null)
     float *Qexact;        // mode Q: optional exact output [rows x r] (V)
     float *U;             // mode U: [rows x r]
     float *R;             // mode U: [r x r]
@@ -601,7 +651,11 @@ __global__ void __launch_bounds__(kCqrThreads) k_cholqr_apply(const __grid_const
             double acc = 0.0;
 #pragma unroll
             for (int k = 0; k <= c; ++k) acc += yv[k] * Ri[k * 32 + c];
-            if (MODE == 0 && t < nrows) M.Qt[(int64_t)c * p.qt_ld + row] = round_tf32((float)acc);
+            if (MODE == 0 && t < nrows) {
+                const float f = (float)acc, hi = round_tf32(f);
+                M.Qt[(int64_t)c * p.qt_ld + row] = hi;
+                if (M.Qt_lo) M.Qt_lo[(int64_t)c * p.qt_ld + row] = round_tf32(f - hi);
+            }
             tile[t * 33 + c] = (float)acc;
         }
     }
@@ -958,15 +1012,17 @@ int64_t rup(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
     int rp;
+    bool split;                           // split (3xTF32) products: lo parts of Q^T and P^T too
     int64_t mp, np;                       // padded leading dims (multiples of 32)
-    size_t qt, pt, pe, z, cnt, gp, ri, total;   // byte offsets inside the workspace
+    size_t qt, pt, qt_lo, pt_lo, pe, z, cnt, gp, ri, total;   // byte offsets inside the workspace
     int chunks;                           // Gram chunks of the tallest block
 };
 
-WsLayout layout(int nmat, int64_t m, int64_t n, int r)
+WsLayout layout(int nmat, int64_t m, int64_t n, int r, bool split)
 {
     WsLayout L{};
     L.rp = r <= 16 ? 16 : 32;
+    L.split = split;
     L.mp = rup(m, 32);
     L.np = rup(n, 32);
     size_t off = 0;
@@ -977,6 +1033,8 @@ WsLayout layout(int nmat, int64_t m, int64_t n, int r)
     };
     L.qt = take((size_t)nmat * L.rp * L.np * 4);
     L.pt = take((size_t)nmat * L.rp * L.mp * 4);
+    L.qt_lo = split ? take((size_t)nmat * L.rp * L.np * 4) : 0;
+    L.pt_lo = split ? take((size_t)nmat * L.rp * L.mp * 4) : 0;
     L.pe = take((size_t)nmat * m * L.rp * 4);
     L.z = take((size_t)nmat * n * L.rp * 4);
     L.cnt = take((size_t)nmat * sizeof(unsigned int));
@@ -987,7 +1045,7 @@ WsLayout layout(int nmat, int64_t m, int64_t n, int r)
     return L;
 }
 
-template <int RP, int CPS>
+template <int RP, int CPS, bool SPLIT>
 cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
 {
     // the shared-memory opt-in is a per-device function attribute: set it once per device
@@ -999,33 +1057,39 @@ cudaError_t gemm_launch_rp(GemmParams &gp, int grid, cudaStream_t stream)
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || !done[dev]) {
-            e = cudaFuncSetAttribute(k_gemm_tf32<RP, CPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)gemm_smem_bytes<RP, CPS>());
+            e = cudaFuncSetAttribute(k_gemm_tf32<RP, CPS, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gemm_smem_bytes<RP, CPS, SPLIT>());
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) done[dev] = true;
         }
     }
-    const char *name = RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>";
-    log_launch(name, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP, CPS>());
+    const char *name = SPLIT ? (RP == 16 ? "k_gemm_tf32<16,split>" : "k_gemm_tf32<32,split>")
+                             : (RP == 16 ? "k_gemm_tf32<16>" : "k_gemm_tf32<32>");
+    log_launch(name, dim3(grid), dim3(kGemmThreads), gemm_smem_bytes<RP, CPS, SPLIT>());
     trace_begin(name, stream);
-    k_gemm_tf32<RP, CPS><<<grid, kGemmThreads, gemm_smem_bytes<RP, CPS>(), stream>>>(gp);
+    k_gemm_tf32<RP, CPS, SPLIT><<<grid, kGemmThreads, gemm_smem_bytes<RP, CPS, SPLIT>(), stream>>>(gp);
     trace_end(stream);
     return cudaGetLastError();
 }
 
 // Resident CTAs per SM for a launch of `total_tiles` tiles (see GemmCfg).
-int gemm_cps(int rp, int64_t total_tiles) { return rp == 16 && total_tiles >= 2 * (int64_t)num_sms() ? 2 : 1; }
+int gemm_cps(int rp, bool split, int64_t total_tiles)
+{
+    return !split && rp == 16 && total_tiles >= 2 * (int64_t)num_sms() ? 2 : 1;
+}
 
-cudaError_t gemm_launch(GemmParams &gp, int total_tiles, int cps, cudaStream_t stream)
+cudaError_t gemm_launch(GemmParams &gp, int total_tiles, int cps, bool split, cudaStream_t stream)
 {
     const int grid = total_tiles < cps * num_sms() ? total_tiles : cps * num_sms();
     if (grid <= 0) return cudaSuccess;
-    if (gp.rp != 16) return gemm_launch_rp<32, 1>(gp, grid, stream);
-    return cps == 2 ? gemm_launch_rp<16, 2>(gp, grid, stream) : gemm_launch_rp<16, 1>(gp, grid, stream);
+    if (split) return gp.rp != 16 ? gemm_launch_rp<32, 1, true>(gp, grid, stream) : gemm_launch_rp<16, 1, true>(gp, grid, stream);
+    if (gp.rp != 16) return gemm_launch_rp<32, 1, false>(gp, grid, stream);
+    return cps == 2 ? gemm_launch_rp<16, 2, false>(gp, grid, stream) : gemm_launch_rp<16, 1, false>(gp, grid, stream);
 }
 
-int gemm_bk(int rp, int cps)
+int gemm_bk(int rp, int cps, bool split)
 {
+    if (split) return rp != 16 ? GemmCfg<32, 1, true>::BK : GemmCfg<16, 1, true>::BK;
     return rp != 16 ? GemmCfg<32, 1>::BK : (cps == 2 ? GemmCfg<16, 2>::BK : GemmCfg<16, 1>::BK);
 }
 
@@ -1056,8 +1120,8 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             gp->wait_ns = 20000000ull;
         }
         bool ok;
-        const int cps = gemm_cps(L.rp, (int64_t)cnt * (((!mn_major ? m : n) + kBM - 1) / kBM));
-        const int bk = gemm_bk(L.rp, cps);
+        const int cps = gemm_cps(L.rp, L.split, (int64_t)cnt * (((!mn_major ? m : n) + kBM - 1) / kBM));
+        const int bk = gemm_bk(L.rp, cps, L.split);
         if (!mn_major) {
             gp->tiles_per_mat = (int)((m + kBM - 1) / kBM);
             gp->ktiles = (int)((n + bk - 1) / bk);
@@ -1065,8 +1129,12 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             gp->out_ld = (int)L.mp;
             ok = make_map3(&gp->tb, ws + L.qt + (size_t)first * L.rp * L.np * 4, n, L.rp, cnt, L.np, L.rp * L.np,
                            kBoxK, L.rp);
+            if (ok && L.split)
+                ok = make_map3(&gp->tb_lo, ws + L.qt_lo + (size_t)first * L.rp * L.np * 4, n, L.rp, cnt, L.np,
+                               L.rp * L.np, kBoxK, L.rp);
             if (out_mode == 0) {
                 gp->out = (float *)(ws + L.pt) + (size_t)first * L.rp * L.mp;
+                gp->out_lo = L.split ? (float *)(ws + L.pt_lo) + (size_t)first * L.rp * L.mp : nullptr;
                 gp->out_stride = L.rp * L.mp;
             } else {
                 gp->out = (float *)(ws + L.pe) + (size_t)first * m * L.rp;
@@ -1079,6 +1147,9 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             gp->out_ld = 0;
             ok = make_map3(&gp->tb, ws + L.pt + (size_t)first * L.rp * L.mp * 4, m, L.rp, cnt, L.mp, L.rp * L.mp,
                            kBoxK, L.rp);
+            if (ok && L.split)
+                ok = make_map3(&gp->tb_lo, ws + L.pt_lo + (size_t)first * L.rp * L.mp * 4, m, L.rp, cnt, L.mp,
+                               L.rp * L.mp, kBoxK, L.rp);
             gp->out = (float *)(ws + L.z) + (size_t)first * n * L.rp;
             gp->out_stride = n * L.rp;
         }
@@ -1091,7 +1162,7 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
             err = cudaErrorInvalidValue;
             break;
         }
-        err = gemm_launch(*gp, cnt * gp->tiles_per_mat, cps, stream);
+        err = gemm_launch(*gp, cnt * gp->tiles_per_mat, cps, L.split, stream);
     }
     delete gp;
     return err;
@@ -1130,6 +1201,7 @@ cudaError_t cholqr_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsL
             c.count = (unsigned int *)(ws + L.cnt) + i;
             c.Rinv = (double *)(ws + L.ri + (size_t)i * 32 * 32 * 8);
             c.Qt = (float *)(ws + L.qt + (size_t)i * L.rp * L.np * 4);
+            c.Qt_lo = L.split ? (float *)(ws + L.qt_lo + (size_t)i * L.rp * L.np * 4) : nullptr;
             c.Qexact = final_v ? mats[i].V : nullptr;
             c.U = mats[i].U;
             c.R = mats[i].R;
@@ -1236,18 +1308,33 @@ cudaError_t apply_pass(const LowrankPlan &pl, const LowrankMat *mats, bool sende
 
 }  // namespace
 
-size_t lowrank_workspace_bytes(int nmat, int64_t m, int64_t n, int r) { return layout(nmat, m, n, r).total; }
+bool lowrank_split(int precision, int64_t m, int64_t n, int r)
+{
+    if (precision == CF_PRECISION_SPLIT) return true;
+    if (precision == CF_PRECISION_TF32) return false;
+    // automatic: split products where the rank is a large fraction of the
+    // smaller dimension, i.e. where a few iterations leave the subspace far
+    // from converged and the result follows every rounding of the products
+    return (int64_t)8 * r > std::min(m, n);
+}
+
+size_t lowrank_workspace_bytes(int nmat, int64_t m, int64_t n, int r, bool split)
+{
+    return layout(nmat, m, n, r, split).total;
+}
 
 cudaError_t run_lowrank(const LowrankPlan &pl, const LowrankMat *mats, cudaStream_t stream)
 {
     if (pl.nmat <= 0) return cudaSuccess;
     if (pl.m > INT32_MAX || pl.n > INT32_MAX) return cudaErrorInvalidValue;
-    const WsLayout L = layout(pl.nmat, pl.m, pl.n, pl.r);
+    const WsLayout L = layout(pl.nmat, pl.m, pl.n, pl.r, pl.split);
     if (pl.ws_bytes < L.total) return cudaErrorInvalidValue;
     char *ws = (char *)pl.ws;
     // Padded rows of Q^T (rows r..rp-1) must be zero: they feed zero columns.
     cudaError_t err = cudaMemsetAsync(ws + L.qt, 0, (size_t)pl.nmat * L.rp * L.np * 4, stream);
     if (err == cudaSuccess) err = cudaMemsetAsync(ws + L.pt, 0, (size_t)pl.nmat * L.rp * L.mp * 4, stream);
+    if (err == cudaSuccess && L.split) err = cudaMemsetAsync(ws + L.qt_lo, 0, (size_t)pl.nmat * L.rp * L.np * 4, stream);
+    if (err == cudaSuccess && L.split) err = cudaMemsetAsync(ws + L.pt_lo, 0, (size_t)pl.nmat * L.rp * L.mp * 4, stream);
     // CholeskyQR chunk counters start at zero (each launch leaves them at zero)
     if (err == cudaSuccess) err = cudaMemsetAsync(ws + L.cnt, 0, (size_t)pl.nmat * sizeof(unsigned int), stream);
     // Line 1: Q = orth(Q0).

@@ -63,23 +63,29 @@ def source_hash(src="cf_quant.cu"):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(kernel, src="cf_quant.cu"):
-    """DRAM bytes per launch (per call for the low-rank call) from a committed
-    ncu summary of the same source file."""
+def recorded_traffic(kernel, src="cf_quant.cu", field="dram_bytes_per_launch"):
+    """A recorded ncu figure of a kernel (by default its DRAM bytes per launch,
+    per call for the whole low-rank call) from profiles/traffic.json, reported
+    only while that capture's source file is the one built here."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         e = d.get(kernel)
-        if e and e.get("source_sha") == source_hash(src):
-            return float(e["dram_bytes_per_launch"])
+        if e and e.get("source_sha") == source_hash(src) and e.get(field) is not None:
+            return float(e[field])
     except Exception:
         pass
     return None
 
 
 class ClockSampler:
-    """Samples SM clock, power and clock-event reasons through NVML."""
+    """Samples SM clock and clock-event reasons through NVML while ``active``.
+
+    The NVML handle is found by the GPU's UUID (else its PCI bus id), since
+    NVML numbers devices physically and ignores CUDA_VISIBLE_DEVICES.  Samples
+    are kept only while ``active`` is set, i.e. inside the timed regions.
+    """
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -91,48 +97,96 @@ class ClockSampler:
         self.samples = []
         self.ok = False
         self.reasons = set()
+        self.active = False
+        self.how = None
         self._stop = threading.Event()
         try:
             import pynvml
 
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.h, self.how = self._handle(pynvml, dev_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
             self.max_mhz = None
 
+    @staticmethod
+    def _handle(nv, dev_index):
+        props = torch.cuda.get_device_properties(dev_index)
+        uuid = getattr(props, "uuid", None)
+        if uuid is not None:
+            want = str(uuid).lower().replace("gpu-", "")
+            for i in range(nv.nvmlDeviceGetCount()):
+                h = nv.nvmlDeviceGetHandleByIndex(i)
+                u = nv.nvmlDeviceGetUUID(h)
+                u = (u.decode() if isinstance(u, bytes) else u).lower().replace("gpu-", "")
+                if u == want:
+                    return h, "uuid"
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            busid = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), bus, getattr(props, "pci_device_id", 0))
+            return nv.nvmlDeviceGetHandleByPciBusId_v2(busid), "pci_bus_id"
+        raise RuntimeError("cannot match the CUDA device to an NVML device")
+
     def _run(self):
         nv = self.nv
         while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append(mhz)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(0.005)
+            if self.active:
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    if self.active:
+                        self.samples.append(mhz)
+                        for bit, name in self.REASONS.items():
+                            if r & bit:
+                                self.reasons.add(name)
+                except Exception:
+                    pass
+            time.sleep(0.002)
 
-    def __enter__(self):
+    def start(self):
         if self.ok:
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
 
-    def __exit__(self, *a):
+    def stop(self):
         if self.ok:
             self._stop.set()
             self.t.join()
+
+    def __enter__(self):
+        self.start()
+        self.active = True
+        return self
+
+    def __exit__(self, *a):
+        self.active = False
+        self.stop()
 
     def summary(self):
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples), "nvml_device": self.how,
+                "window": "every timed region of this run"}
+
+
+class Timed:
+    """Marks a timed region for the clock sampler (samples are kept only inside)."""
+
+    def __init__(self, clk):
+        self.clk = clk
+
+    def __enter__(self):
+        if self.clk is not None:
+            self.clk.active = True
+        return self
+
+    def __exit__(self, *a):
+        if self.clk is not None:
+            self.clk.active = False
 
 
 def dist_init():
@@ -207,6 +261,19 @@ def host_inputs(w, rows, steps, seed=0):
                 for x in synth.activations(sub, s, steps, seed=seed)] for s in range(w.slots)}
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -239,7 +306,8 @@ def run_reference(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w),
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -260,6 +328,7 @@ def run_cf(args, w):
     import activation_residual_compression_02_b200 as cf
 
     dev = torch.device("cuda", torch.cuda.current_device())
+    clk = ClockSampler(torch.cuda.current_device()).start()
     shapes = [(w.rows, w.cols)] * w.slots
     ctx = cf.Context(shapes, bits=w.bits, group=w.group)
     st = cf.QuantState(shapes, w.bits, w.group, device=dev)
@@ -304,7 +373,7 @@ def run_cf(args, w):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with Timed(clk):
         start.record(stream)
         for k in range(args.steps):
             i = args.warmup + 1 + k
@@ -334,13 +403,14 @@ def run_cf(args, w):
         barrier(world)
         torch.cuda.synchronize()
         l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        l0.record(stream)
-        for k in range(args.steps):
-            i = args.warmup + 1 + k
-            if L.cf_loopback(h, c_slots[(i - 1) % len(c_slots)], i, sh) != 0:
-                raise RuntimeError(L.cf_last_error(h).decode())
-        l1.record(stream)
-        torch.cuda.synchronize()
+        with Timed(clk):
+            l0.record(stream)
+            for k in range(args.steps):
+                i = args.warmup + 1 + k
+                if L.cf_loopback(h, c_slots[(i - 1) % len(c_slots)], i, sh) != 0:
+                    raise RuntimeError(L.cf_last_error(h).decode())
+            l1.record(stream)
+            torch.cuda.synchronize()
         lb_ms = max_over_ranks(l0.elapsed_time(l1), world) / args.steps
         lb_bytes = (22.0 + w.bits / 8 + 4 / w.group) * n_elem
         lb = {"ms_per_step": lb_ms, "value": world * x_bytes / (lb_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -375,15 +445,16 @@ def run_cf(args, w):
         barrier(world)
         torch.cuda.synchronize()
         r0, r1, r2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        r0.record(stream)
-        for _ in range(args.steps):
-            deco(r_arr)
-        r1.record(stream)
-        for _ in range(args.steps):
-            deco(c_slots[last])
-            recon_all.copy_(st.cache_all)
-        r2.record(stream)
-        torch.cuda.synchronize()
+        with Timed(clk):
+            r0.record(stream)
+            for _ in range(args.steps):
+                deco(r_arr)
+            r1.record(stream)
+            for _ in range(args.steps):
+                deco(c_slots[last])
+                recon_all.copy_(st.cache_all)
+            r2.record(stream)
+            torch.cuda.synchronize()
         if ctx.check() != 0:
             raise RuntimeError("device status in the recon run")
         r_ms = max_over_ranks(r0.elapsed_time(r1), world) / args.steps
@@ -408,13 +479,14 @@ def run_cf(args, w):
     barrier(world)
     torch.cuda.synchronize()
     wev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for k in range(args.steps):
-        wev[k][0].record(stream)
-        L.cf_compress(h, a0, 0, sh)
-        wev[k][1].record(stream)
-        L.cf_decompress(h, a0, 0, sh)
-        wev[k][2].record(stream)
-    torch.cuda.synchronize()
+    with Timed(clk):
+        for k in range(args.steps):
+            wev[k][0].record(stream)
+            L.cf_compress(h, a0, 0, sh)
+            wev[k][1].record(stream)
+            L.cf_decompress(h, a0, 0, sh)
+            wev[k][2].record(stream)
+        torch.cuda.synchronize()
     ws_ms = sum(e[0].elapsed_time(e[1]) for e in wev) / args.steps
     wr_ms = sum(e[1].elapsed_time(e[2]) for e in wev) / args.steps
     warm = {"sender_ms": ws_ms, "receiver_ms": wr_ms,
@@ -448,19 +520,20 @@ def run_cf(args, w):
         torch.cuda.synchronize()
         q0e, q1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         lev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        q0e.record(stream)
-        for k in range(args.steps):
-            i = args.warmup + 1 + k
-            arr = l_arrays[(i - 1) % len(l_arrays)]
-            lev[k][0].record(stream)
-            if L.cf_compress(lh, arr, i, sh) != 0:
-                raise RuntimeError(L.cf_last_error(lh).decode())
-            lev[k][1].record(stream)
-            if L.cf_decompress(lh, arr, i, sh) != 0:
-                raise RuntimeError(L.cf_last_error(lh).decode())
-            lev[k][2].record(stream)
-        q1e.record(stream)
-        torch.cuda.synchronize()
+        with Timed(clk):
+            q0e.record(stream)
+            for k in range(args.steps):
+                i = args.warmup + 1 + k
+                arr = l_arrays[(i - 1) % len(l_arrays)]
+                lev[k][0].record(stream)
+                if L.cf_compress(lh, arr, i, sh) != 0:
+                    raise RuntimeError(L.cf_last_error(lh).decode())
+                lev[k][1].record(stream)
+                if L.cf_decompress(lh, arr, i, sh) != 0:
+                    raise RuntimeError(L.cf_last_error(lh).decode())
+                lev[k][2].record(stream)
+            q1e.record(stream)
+            torch.cuda.synchronize()
         if lctx.check() != 0:
             raise RuntimeError("device status in the lean run")
         lean_ms = max_over_ranks(q0e.elapsed_time(q1e), world) / args.steps
@@ -506,15 +579,16 @@ def run_cf(args, w):
         hc.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(hc.s_h2d)
-        for t in range(3, 3 + e2e_steps):
-            e2e_step(t)
-        for s_ in (hc.s_codec, hc.s_d2h):
-            ev = torch.cuda.Event()
-            ev.record(s_)
-            hc.s_h2d.wait_event(ev)
-        e1.record(hc.s_h2d)
-        hc.synchronize()
+        with Timed(clk):
+            e0.record(hc.s_h2d)
+            for t in range(3, 3 + e2e_steps):
+                e2e_step(t)
+            for s_ in (hc.s_codec, hc.s_d2h):
+                ev = torch.cuda.Event()
+                ev.record(s_)
+                hc.s_h2d.wait_event(ev)
+            e1.record(hc.s_h2d)
+            hc.synchronize()
         if hc.check() != 0:
             raise RuntimeError("device status after the e2e run")
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
@@ -537,10 +611,26 @@ def run_cf(args, w):
         xs_host = {s: [X[t][s].view(torch.int16).cpu().numpy().view(np.uint16).copy() for t in range(1 + csteps)]
                    for s in range(w.slots)}
         dt, elems = oracle_run(w, xs_host, cores)
-        cpu = {"value": elems * 2 / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+        cpu = {"value": elems * 2 / dt / 1e9, "unit": "GB/s", "cores": cores, "cpu_model": cpu_model(),
+               "kind": "oracle",
                "sample": f"the whole workload ({w.slots} slots x {w.rows} x {w.cols}) for {csteps} compressed "
                          f"steps after the warmup (compress + decompress, {elems} elements), one slot per host "
                          f"thread, {cores} threads, {dt:.1f} s wall"}
+
+    # ---- the other workloads of the codec, as extra keys of this line ----
+    # The CogVideoX-shaped and stress steps (quantised), and the low-rank call
+    # (Algorithm 3 + apply on 57 x 4608 x 3072 fp32), each timed the same way.
+    cog = stress = lowrank = None
+    if not args.no_extra:
+        del X, slot_lists, c_slots, slots0, st
+        torch.cuda.empty_cache()
+        cog = quant_extra(args, synth.COGVIDEOX, world, rank, clk, min(args.steps, 30))
+        stress = quant_extra(args, synth.STRESS, world, rank, clk, min(args.steps, 10))
+        lowrank = lowrank_measure(args, synth.LOWRANK, world, rank, clk, min(args.steps, 20),
+                                  0 if args.no_cpu else 4)
+        if lowrank.get("cpu_baseline"):
+            lowrank["cpu_baseline"]["sample"] += " (a bounded sample: the run stays short)"
+    clk.stop()
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -557,6 +647,7 @@ def run_cf(args, w):
                           "alg_bytes_per_step": (bc + bd) * n_elem},
         "loopback": lb, "lean_state": lean, "recon": rc, "warmup_step": warm,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
+        "cogvideox": cog, "stress": stress, "lowrank": lowrank,
         "clocks": clk.summary(),
     }
     if rank == 0:
@@ -569,19 +660,20 @@ def run_cf(args, w):
     return 0
 
 
-def run_lowrank_bench(args, w):
-    """Algorithm 3 on the low-rank workload (57 fp32 residual matrices of
-    4608 x 3072, r = 16, T = 2, Gaussian start blocks) through cf_lowrank,
-    with the error buffer E = A - U R V^T written (a step of the low-rank
-    codec's sender on given residuals)."""
-    world, rank, local = dist_init()
+def lowrank_measure(args, w, world, rank, clk, steps, cpu_mats, through_slots=False, warm_start=False, precision=0):
+    """Algorithm 3 on the low-rank workload (k fp32 residual matrices of
+    m x n, rank r, T iterations, Gaussian start blocks) through cf_lowrank,
+    with the error buffer E = A - U R V^T written: a step of the low-rank
+    codec's sender on given residuals.  Times `steps` calls with CUDA events,
+    then the same calls again with per-launch tracing (cf_trace).  Returns the
+    fields of a bench line (without the line's own keys)."""
     import activation_residual_compression_02_b200 as cf
 
     dev = torch.device("cuda", torch.cuda.current_device())
     m, n, r, T, k = w.rows, w.cols, w.rank, w.iters, w.slots
-    if args.warm_start:
+    if warm_start:
         T = 1      # each call starts from the previous call's V
-    ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+    ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T, precision=precision)
     ws = torch.empty(ctx.lowrank_workspace_bytes(k, m, n), dtype=torch.uint8, device=dev)
     ctx.set_workspace(ws)
     A = [synth.lowrank_matrix(m, n, r, mat=i, seed=rank, device=dev) for i in range(k)]
@@ -592,36 +684,38 @@ def run_lowrank_bench(args, w):
     E = [torch.empty(m, n, device=dev) for _ in range(k)]
     stream = torch.cuda.current_stream()
     ctx.lowrank(A, Q0, U, R, V, E)
-    start_block = V if args.warm_start else Q0   # warm start: V doubles as the next start block
+    start_block = V if warm_start else Q0   # warm start: V doubles as the next start block
     for _ in range(args.warmup):
         ctx.lowrank(A, start_block, U, R, V, E)
     torch.cuda.synchronize()
     assert ctx.check() == 0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    torch.cuda.synchronize()
+    with Timed(clk):
         start.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             ctx.lowrank(A, start_block, U, R, V, E)
         end.record(stream)
         torch.cuda.synchronize()
     status = ctx.check()
     if status != 0:
         raise RuntimeError(f"device status {status}")
-    ms = max_over_ranks(start.elapsed_time(end), world) / args.steps
+    ms = max_over_ranks(start.elapsed_time(end), world) / steps
 
     # ---- the same calls again with per-launch tracing (cf_trace_*) -------
     # CUDA events around every kernel on the launching stream give each
     # kernel's live duration; the roofline line is the dominant kernel's.
     ctx.trace(True)
-    for _ in range(args.steps):
-        ctx.lowrank(A, start_block, U, R, V, E)
-    torch.cuda.synchronize()
+    with Timed(clk):
+        for _ in range(steps):
+            ctx.lowrank(A, start_block, U, R, V, E)
+        torch.cuda.synchronize()
     trace = ctx.trace_read()
     ctx.trace(False)
     for e in trace:
         e["ms_per_launch"] = max_over_ranks(e["total_ms"] / e["launches"], world)
-        e["launches_per_call"] = e["launches"] // args.steps
+        e["launches_per_call"] = e["launches"] // steps
     dom = max(trace, key=lambda e: e["total_ms"] * 1.0)
     elems = k * m * n
     peak, peak_kind = hbm_peak()
@@ -633,15 +727,16 @@ def run_lowrank_bench(args, w):
         gemm_bytes = elems * 8
     sched_bytes = elems * (4 * (2 * T + 2) + 4)   # A read by each of the 2T+1 products and the apply, E written
     flops = 2.0 * (2 * T + 1) * m * n * r * k + 2.0 * m * n * r * k
+    full_size = (k, m, n, r, w.iters) == (57, 4608, 3072, 16, 2) and not warm_start and precision == 0
 
     # ---- low-rank mode through cf_compress / cf_decompress ---------------
     # The same shapes as bf16 activation slots: each compressed step first
     # materialises A = (X - base) + E in fp32 (k_residual_f32), then runs the
     # call above on it; the receiver adds U R V^T to its cache.
     lr_mode = None
-    if args.through_slots:
+    if through_slots:
         shapes = [(m, n)] * k
-        mctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+        mctx = cf.Context(shapes, mode=cf.CF_MODE_LOWRANK, rank=r, iters=T, precision=precision)
         mws = torch.empty(mctx.workspace_bytes(), dtype=torch.uint8, device=dev)
         mctx.set_workspace(mws)
         wq = synth.FLUX.scaled(slots=k, rows=m, cols=n)
@@ -672,14 +767,15 @@ def run_lowrank_bench(args, w):
             mstep(i)
         torch.cuda.synchronize()
         barrier(world)
-        mev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        for j in range(args.steps):
-            mstep(args.warmup + 1 + j, mev[j])
-        torch.cuda.synchronize()
+        mev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        with Timed(clk):
+            for j in range(steps):
+                mstep(args.warmup + 1 + j, mev[j])
+            torch.cuda.synchronize()
         if mctx.check() != 0:
             raise RuntimeError("device status in the low-rank mode run")
-        c_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in mev) / args.steps, world)
-        d_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in mev) / args.steps, world)
+        c_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in mev) / steps, world)
+        d_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in mev) / steps, world)
         lr_mode = {"compress_ms": c_ms, "decompress_ms": d_ms, "ms_per_step": c_ms + d_ms,
                    "value": world * elems * 2 / ((c_ms + d_ms) * 1e-3) / 1e9, "unit": "GB/s of bf16 activations",
                    "residual_ms_est": c_ms - ms,
@@ -691,13 +787,13 @@ def run_lowrank_bench(args, w):
         del mctx, mws, Xs, mb, me, mc, arrs
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
+    if rank == 0 and world == 1 and cpu_mats > 0:
         import concurrent.futures
 
         import oracle
 
         oracle.build()
-        nsample = k                     # every matrix: about 30 s of host CPU work at full size
+        nsample = min(cpu_mats, k)
         Ah = [A[i].cpu().numpy() for i in range(nsample)]
         Qh = [Q0[i].cpu().numpy() for i in range(nsample)]
 
@@ -710,32 +806,34 @@ def run_lowrank_bench(args, w):
         with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
             list(ex.map(work, range(nsample)))
         dt = time.perf_counter() - t0
-        cpu = {"value": nsample * m * n * 4 / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        cpu = {"value": nsample * m * n * 4 / dt / 1e9, "unit": "GB/s", "cores": threads,
+               "cpu_model": cpu_model(), "kind": "oracle",
                "sample": f"{nsample} of the {k} matrices (Algorithm 3 in fp64 plus the apply), one matrix per host "
                          f"thread, {threads} threads, {dt:.1f} s wall"}
-    line = {
-        "metric": "low-rank codec GB/s of fp32 residual input (Algorithm 3 + apply)", "value":
-            world * elems * 4 / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "tf32/f64", "data": "synthetic",
+    out = {
+        "value": world * elems * 4 / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+        "warmup": args.warmup,
         "config": {"workload": f"lowrank: {k} matrices x {m} x {n} fp32, rank-{r} signal + 0.01 noise, r={r}, "
-                               f"T={T}, " + ("warm start from the previous V" if args.warm_start else "Gaussian Q0")
-                               + ", E = A - U R V^T written",
+                               f"T={T}, " + ("warm start from the previous V" if warm_start else "Gaussian Q0")
+                               + ", E = A - U R V^T written"
+                               + {0: "", 1: ", TF32 products", 2: ", split (3xTF32) products"}[precision],
                    "l2": "inputs larger than L2 (3.2 GB of A per step)"},
         "roofline": {"bound": "hbm", "kernel": dom["kernel"],
                      "achieved": gemm_bytes / (dom["ms_per_launch"] * 1e-3) / 1e9, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": gemm_bytes / (dom["ms_per_launch"] * 1e-3) / 1e9 / peak,
-                     "traffic": (recorded_traffic("lowrank_gemm", "cf_subspace.cu")
-                                 if not args.slots and not args.warm_start else None),
+                     "traffic": recorded_traffic("lowrank_gemm", "cf_subspace.cu") if full_size else None,
+                     "tensor_pipe": recorded_traffic("lowrank_gemm", "cf_subspace.cu", "tensor_pipe_active")
+                     if full_size else None,
                      "alg_bytes_per_launch": gemm_bytes, "ms_per_launch": dom["ms_per_launch"],
                      "note": "the dominant kernel, timed live by per-launch CUDA events (cf_trace); one launch "
                              "is one product with A over all matrices: A read once, the r-column blocks read and "
-                             "written (a read-only stream can exceed the copy peak)"},
+                             "written (a read-only stream can exceed the copy peak); tensor_pipe: the fraction of "
+                             "cycles the tensor pipe was active (ncu sm__pipe_tensor_cycles_active) in the recorded "
+                             "capture of the same source"},
         "roofline_call": {"kernel": "whole cf_lowrank call", "achieved": alg_bytes / (ms * 1e-3) / 1e9,
                           "frac": alg_bytes / (ms * 1e-3) / 1e9 / peak,
-                          "traffic": (recorded_traffic("lowrank_call", "cf_subspace.cu")
-                                      if not args.slots and not args.warm_start else None),
+                          "traffic": recorded_traffic("lowrank_call", "cf_subspace.cu") if full_size else None,
                           "alg_bytes_per_step": alg_bytes, "tflops": flops / (ms * 1e-3) / 1e12,
                           "schedule_bytes_per_step": sched_bytes,
                           "schedule_frac": sched_bytes / (ms * 1e-3) / 1e9 / peak,
@@ -743,14 +841,102 @@ def run_lowrank_bench(args, w):
                                   "the 2T+1 products and in the apply"},
         "kernels": [{"kernel": e["kernel"], "launches_per_call": e["launches_per_call"],
                      "ms_per_launch": e["ms_per_launch"]} for e in trace],
-        "gpu_launches": args.steps * sum(e["launches_per_call"] for e in trace), "e2e": None, "cpu_baseline": cpu,
+        "gpu_launches": steps * sum(e["launches_per_call"] for e in trace), "cpu_baseline": cpu,
         "lowrank_mode": lr_mode,
-        "clocks": clk.summary(),
     }
+    ctx.close()
+    del A, Q0, U, R, V, E, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_lowrank_bench(args, w):
+    """The low-rank workload as the bench line (--workload lowrank)."""
+    world, rank, local = dist_init()
+    clk = ClockSampler(torch.cuda.current_device()).start()
+    out = lowrank_measure(args, w, world, rank, clk, args.steps, 0 if args.no_cpu else w.slots,
+                          through_slots=args.through_slots, warm_start=args.warm_start, precision=args.precision)
+    clk.stop()
+    line = {"metric": "low-rank codec GB/s of fp32 residual input (Algorithm 3 + apply)", "n_gpus": world,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32/f64",
+            "data": "synthetic", "e2e": None, **out, "clocks": clk.summary()}
+    if args.slots:
+        line["roofline"]["traffic"] = None
     if rank == 0:
         print(json.dumps(line), flush=True)
-    ctx.close()
     return 0
+
+
+def quant_extra(args, w, world, rank, clk, steps):
+    """One more quantised workload (compress + decompress per step, every
+    slot in one grouped launch each), timed like the headline: inputs of a
+    few distinct steps resident in HBM and cycled, CUDA events per kernel."""
+    import activation_residual_compression_02_b200 as cf
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shapes = [(w.rows, w.cols)] * w.slots
+    ctx = cf.Context(shapes, bits=w.bits, group=w.group)
+    st = cf.QuantState(shapes, w.bits, w.group, device=dev)
+    nsteps = 4                                # the warmup and three distinct compressed steps, cycled
+    streams = [synth.SlotStream(w, s, seed=rank, device=dev) for s in range(w.slots)]
+    X = [[None] * w.slots for _ in range(nsteps)]
+    for s in range(w.slots):
+        for t in range(nsteps):
+            X[t][s] = streams[s].next().reshape(-1)
+        streams[s].state = None
+    del streams
+    arrs = [ctx._slots(st.slots(X[t])) for t in range(nsteps)]
+    L, h = cf.lib(), ctx.handle
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def step(i, ev=None):
+        arr = arrs[0] if i == 0 else arrs[1 + (i - 1) % (nsteps - 1)]
+        if ev:
+            ev[0].record(stream)
+        if L.cf_compress(h, arr, i, sh) != 0:
+            raise RuntimeError(L.cf_last_error(h).decode())
+        if ev:
+            ev[1].record(stream)
+        if L.cf_decompress(h, arr, i, sh) != 0:
+            raise RuntimeError(L.cf_last_error(h).decode())
+        if ev:
+            ev[2].record(stream)
+
+    for i in range(args.warmup + 1):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Timed(clk):
+        t0.record(stream)
+        for k in range(steps):
+            step(args.warmup + 1 + k, ev[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if ctx.check() != 0:
+        raise RuntimeError(f"device status in the {w.name} run")
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / steps
+    c_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / steps, world)
+    d_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / steps, world)
+    bc, bd = alg_bytes_per_elem(w.bits, w.group)
+    peak, _ = hbm_peak()
+    n = w.elems
+    pair = (bc + bd) * n / (ms * 1e-3) / 1e9
+    out = {"metric": METRIC, "value": world * n * 2 / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+           "steps": steps, "warmup": args.warmup, "config": workload_config(w),
+           "compress": {"ms_per_launch": c_ms, "frac": bc * n / (c_ms * 1e-3) / 1e9 / peak,
+                        "alg_bytes_per_launch": bc * n},
+           "decompress": {"ms_per_launch": d_ms, "frac": bd * n / (d_ms * 1e-3) / 1e9 / peak,
+                          "alg_bytes_per_launch": bd * n},
+           "roofline_step": {"achieved": pair, "frac": pair / peak, "frac_of_8tbs": pair / 8000.0,
+                             "alg_bytes_per_step": (bc + bd) * n},
+           "gpu_launches": 2 * steps}
+    ctx.close()
+    del X, arrs, st
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_exchange_bench(args, w):
@@ -849,7 +1035,11 @@ def main():
     ap.add_argument("--no-loopback", action="store_true")
     ap.add_argument("--no-lean", action="store_true")
     ap.add_argument("--no-recon", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the CogVideoX-shaped, stress and low-rank extra keys of the default line")
     ap.add_argument("--warm-start", action="store_true", help="low-rank: T = 1 from the previous call's V")
+    ap.add_argument("--precision", type=int, default=0, choices=[0, 1, 2],
+                    help="low-rank products: 0 automatic, 1 TF32, 2 split (3xTF32)")
     ap.add_argument("--through-slots", action="store_true",
                     help="low-rank: also time cf_compress / cf_decompress in low-rank mode on bf16 slots")
     ap.add_argument("--exchange", action="store_true",

@@ -94,6 +94,16 @@ typedef enum cf_status {
 
 enum { CF_MODE_QUANT = 0, CF_MODE_LOWRANK = 1 };
 
+/* Arithmetic of the low-rank products with A (A Q and A^T P). */
+enum {
+    CF_PRECISION_AUTO = 0,   /* split products where r > min(m, n) / 8, TF32 elsewhere */
+    CF_PRECISION_TF32 = 1,   /* operands rounded to TF32 (nearest): relative error about 2^-12 per product */
+    CF_PRECISION_SPLIT = 2   /* "3xTF32": each operand as a TF32 hi + lo pair, three MMAs per step; close to
+                                fp32 accuracy, for iterations that follow every rounding (few iterations with a
+                                rank that is a large fraction of the matrix), at about twice the shared-memory
+                                traffic of the TF32 form */
+};
+
 typedef struct cf_config {
     int mode;        /* CF_MODE_QUANT or CF_MODE_LOWRANK */
     int bits;        /* quant: k = 1, 2 or 4 */
@@ -108,6 +118,7 @@ typedef struct cf_config {
                         (default); 1 = from the second compressed step on, start from the slot's V
                         of the previous step (q0 may then be NULL), so that a small `iters`
                         (e.g. 1) tracks a slowly moving subspace with fewer passes over A */
+    int precision;   /* low-rank: CF_PRECISION_AUTO (default), _TF32 or _SPLIT */
 } cf_config;
 
 typedef struct cf_shape {
@@ -138,17 +149,24 @@ typedef struct cf_slot {
  * device has compute capability 10.0 (the only target of sm_100a code), and
  * allocates the device status word on it.
  * nslots may be 0 for a context used only with cf_lowrank.
- * Errors: CF_E_ARG, CF_E_SHAPE, CF_E_NOMEM, CF_E_CUDA; *out is NULL then. */
+ * Errors: CF_E_ARG, CF_E_SHAPE, CF_E_NOMEM (a host or device allocation
+ * failed), CF_E_CUDA; *out is NULL then.
+ * Source: library plumbing with no counterpart in the paper; the
+ * configuration selects the compressor -- the k-bit group quantiser of the
+ * residual (abstract) or rank-r subspace iteration (Algorithm 3). */
 cf_status cf_create(const cf_config *config, int nslots, const cf_shape *shapes, cf_ctx **out);
 
 /* Device workspace cf_compress needs for this context, in bytes (0 in
  * quantised mode; in low-rank mode the fp32 residuals of every slot plus the
- * small per-slot buffers of Algorithm 3). */
+ * small per-slot buffers of Algorithm 3).
+ * Source: library plumbing; the buffers are those of Algorithm 3
+ * (reproducibility table, "Pseudocode" row). */
 size_t cf_workspace_bytes(const cf_ctx *ctx);
 
 /* Register caller-owned device workspace (16-byte aligned) used by
  * cf_compress / cf_lowrank until replaced.  Errors: CF_E_ALIGN, CF_E_NOMEM
- * (smaller than cf_workspace_bytes). */
+ * (smaller than cf_workspace_bytes).
+ * Source: library plumbing, no counterpart in the paper. */
 cf_status cf_set_workspace(cf_ctx *ctx, void *dev_ptr, size_t bytes);
 
 /* Sender side of step `step` for every slot, in one grouped launch.
@@ -162,7 +180,11 @@ cf_status cf_set_workspace(cf_ctx *ctx, void *dev_ptr, size_t bytes);
  * `slots` is a host array of nslots entries; `cuda_stream` a cudaStream_t
  * (NULL = legacy default stream).  Errors before launch: CF_E_ARG,
  * CF_E_ALIGN, CF_E_STATE (step >= 1 before a warmup), CF_E_NOMEM (workspace
- * missing in low-rank mode); CF_E_CUDA if a launch fails. */
+ * missing in low-rank mode); CF_E_CUDA if a launch fails.
+ * Source: abstract (send only the compressed step-wise residual, and feed the
+ * compression error back into the next step); reproducibility table,
+ * "Dataset Splits" row (the uncompressed warmup step sets the base tensor);
+ * "Pseudocode" row, Algorithm 3 (the low-rank mode). */
 cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
 
 /* Receiver side of step `step` for every slot, in one grouped launch.
@@ -176,7 +198,10 @@ cf_status cf_compress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_st
  * cache back (4) and write bf16 (2).  It is meant for the consumer of a
  * received K or V, which reads bf16.  The same holds for cf_loopback.
  * Errors as cf_compress (CF_E_STATE: step >= 1 before a receiver warmup;
- * CF_E_ALIGN: recon not 16-byte aligned). */
+ * CF_E_ALIGN: recon not 16-byte aligned).
+ * Source: abstract (the receiver adds each decompressed residual to the
+ * activation it reconstructed at the previous step); reproducibility table,
+ * "Dataset Splits" row (the warmup step delivers X_0 uncompressed). */
 cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
 
 /* Sender and receiver of step `step` in one pass, for when both sides of a
@@ -188,14 +213,18 @@ cf_status cf_decompress(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_
  * bytes per element less than the pair; step 0, and every step in low-rank
  * mode, run the two sides one after the other.  Uses x, base, err, cache,
  * codes, scales (and q0, U, R, V in low-rank mode).  Errors as cf_compress
- * (CF_E_STATE: step >= 1 before the warmup). */
+ * (CF_E_STATE: step >= 1 before the warmup).
+ * Source: as cf_compress and cf_decompress (abstract; "Dataset Splits" row),
+ * with both sides on one device. */
 cf_status cf_loopback(cf_ctx *ctx, const cf_slot *slots, int step, void *cuda_stream);
 
 /* Workspace cf_lowrank needs for nmat matrices of m x n at this context's
  * rank: the r-column blocks of Algorithm 3 (Q^T, P^T, P, Z, padded to 16 or
  * 32 columns), the fp64 Gram matrices of their 256-row chunks and R^{-1},
  * about 4*rp*(2m + 2n) + 4*r*(r+1)*ceil(max(m, n)/256) + 8 KB bytes per
- * matrix.  Returns 0 for a quantised-mode context or bad sizes. */
+ * matrix.  Returns 0 for a quantised-mode context or bad sizes.
+ * Source: library plumbing; the blocks are those of Algorithm 3
+ * (reproducibility table, "Pseudocode" row). */
 size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_t n);
 
 /* Algorithm 3 (subspace iteration, rank r = config.rank, T = config.iters
@@ -207,11 +236,15 @@ size_t cf_lowrank_workspace_bytes(const cf_ctx *ctx, int nmat, int64_t m, int64_
  *   E_opt NULL or E[i] fp32 [m x n]: E = A - U R V^T       (written)
  *   C_opt NULL or C[i] fp32 [m x n]: C += U R V^T          (updated)
  * Uses the registered workspace (>= cf_lowrank_workspace_bytes).  The two
- * products with A (A Q and A^T P) run on the tensor cores in TF32 with
- * operands rounded to nearest; Gram matrices and Cholesky run in fp64.
+ * products with A (A Q and A^T P) run on the tensor cores, in TF32 with
+ * operands rounded to nearest or split into TF32 hi + lo pairs, as
+ * config.precision selects; Gram matrices and Cholesky run in fp64.
  * Errors before launch: CF_E_ARG, CF_E_SHAPE (m < r, n < r, n % 4),
  * CF_E_ALIGN, CF_E_NOMEM; device-side: CF_E_NONFINITE (Gram matrix not
- * positive definite), CF_E_TIMEOUT, at the next cf_check. */
+ * positive definite), CF_E_TIMEOUT, at the next cf_check.
+ * Source: reproducibility table, "Pseudocode" row, Algorithm 3 (Subspace
+ * Iteration, rank r); E and C are the error feedback and the receiver's
+ * accumulation of the abstract, applied to the rank-r reconstruction. */
 cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *const *A,
                      const float *const *Q0, float *const *U, float *const *R, float *const *V,
                      float *const *E_opt, float *const *C_opt, void *cuda_stream);
@@ -243,15 +276,29 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
  * bytes, and nmat <= 512; otherwise the call returns CF_E_NOMEM and launches
  * nothing.  Eight 4608 x 3072 matrices at r = 16 fit in one call.
  *
- * The call is synchronous: it enqueues the work on `cuda_stream`, waits for
- * it and returns the device status (CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or
- * CF_E_CUDA).  The first call on a device looks up the scratch's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  Every call shares the one scratch array,
- * which keeps the previous call's contents (the call clears what must start
- * at zero), so calls that overlap on the GPU -- on two streams or from two
- * host threads -- race and must be serialised by the caller.  Errors before
- * launch: CF_E_ARG, CF_E_SHAPE, CF_E_ALIGN, CF_E_NOMEM. */
+ * The call runs on the current device; every pointer must be device memory
+ * of that device (else CF_E_ARG).  It is synchronous: it enqueues the work
+ * on `cuda_stream` (a stream of the current device), waits for it and
+ * returns the device status (CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or
+ * CF_E_CUDA).
+ *
+ * First call on a device: it looks up the scratch's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  CUDA loads a library's device code lazily by
+ * default, when it is first used on a device, and the 8 MiB array comes
+ * into existence with it; so the first call into libcf on a device -- this
+ * one or any other -- may itself reserve device memory.  A caller whose
+ * allocation state must not change should make one call (e.g. on a small
+ * matrix) on each device before that region; later calls with the same
+ * rank reserve nothing more.
+ *
+ * Every call shares the one scratch array, which keeps the previous call's
+ * contents (the call clears what must start at zero), so calls that overlap
+ * on the GPU -- on two streams or from two host threads -- race and must be
+ * serialised by the caller.  Errors before launch: CF_E_ARG, CF_E_SHAPE,
+ * CF_E_ALIGN, CF_E_NOMEM.
+ * Source: none in the paper (an integration aid of this library); it
+ * computes what cf_lowrank computes (Algorithm 3, "Pseudocode" row). */
 cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64_t m, int64_t n, const float *const *A,
                              const float *const *Q0, float *const *U, float *const *R, float *const *V,
                              float *const *E_opt, float *const *C_opt, void *cuda_stream);
@@ -260,7 +307,8 @@ cf_status cf_lowrank_noalloc(const cf_config *config, int nmat, int64_t m, int64
  * every kernel this context launches (in cf_compress, cf_decompress,
  * cf_loopback and cf_lowrank) is bracketed by a pair of CUDA events recorded
  * on its stream; the events come from a pool the context keeps.  Not for use
- * while a stream is being captured into a CUDA graph.  Errors: CF_E_ARG. */
+ * while a stream is being captured into a CUDA graph.  Errors: CF_E_ARG.
+ * Source: library plumbing (measurement), no counterpart in the paper. */
 cf_status cf_trace_enable(cf_ctx *ctx, int on);
 
 typedef struct cf_trace_entry {
@@ -272,21 +320,29 @@ typedef struct cf_trace_entry {
 /* Waits for the traced launches, writes per-kernel totals (in order of first
  * launch) to out[0 .. min(count, max_entries)), clears them and returns the
  * number of distinct kernels (which may exceed max_entries), or -CF_E_ARG /
- * -CF_E_CUDA (an event could not be created, recorded or read). */
+ * -CF_E_CUDA (an event could not be created, recorded or read), or
+ * -CF_E_NOMEM.
+ * Source: library plumbing (measurement), no counterpart in the paper. */
 int cf_trace_read(cf_ctx *ctx, cf_trace_entry *out, int max_entries);
 
 /* Synchronise `cuda_stream`, read and clear the device status word.
  * Returns CF_OK, CF_E_NONFINITE, CF_E_TIMEOUT or CF_E_CUDA (an asynchronous
- * CUDA error, e.g. from an earlier launch). */
+ * CUDA error, e.g. from an earlier launch).
+ * Source: library plumbing (error reporting), no counterpart in the paper. */
 cf_status cf_check(cf_ctx *ctx, void *cuda_stream);
 
 /* Payload bytes of slot `slot` per compressed step: rows*cols*k/8 +
  * 4*rows*cols/G (quantised) or 4*r*(rows + r + cols) (low-rank); 0 for a bad
- * slot index. */
+ * slot index.
+ * Source: abstract (only the compressed residual crosses the link); xDiT
+ * issue 573 (residuals plus error feedback cut the traffic 8-16x: 16/k of
+ * the bf16 activations for k = 2 and k = 1, before the scales' 32/G bits
+ * per element). */
 size_t cf_payload_bytes(const cf_ctx *ctx, int slot);
 
 /* Human-readable message of the last error on this context ("" if none).
- * The string is owned by the context. */
+ * The string is owned by the context.
+ * Source: library plumbing, no counterpart in the paper. */
 const char *cf_last_error(const cf_ctx *ctx);
 
 /* Resume a run from caller-saved state (checkpoint / restart).  All codec
@@ -297,11 +353,15 @@ const char *cf_last_error(const cf_ctx *ctx);
  * steps 0..steps_done (the warmup included) have run on both the sender and
  * the receiver side, so the next call may be step steps_done + 1, and a
  * warm-start low-rank context starts Algorithm 3 from the restored V.
- * Enqueues nothing.  Errors: CF_E_ARG (NULL context, steps_done < 0). */
+ * Enqueues nothing.  Errors: CF_E_ARG (NULL context, steps_done < 0).
+ * Source: library plumbing (checkpoint / restart); the state it resumes is
+ * the base tensor ("Dataset Splits" row), the error-feedback buffer and the
+ * receiver's reconstruction (abstract). */
 cf_status cf_resume(cf_ctx *ctx, int64_t steps_done);
 
 /* Free the context (waits for nothing; the caller must not destroy a
- * context while its launches are still running on a stream). */
+ * context while its launches are still running on a stream).
+ * Source: library plumbing, no counterpart in the paper. */
 cf_status cf_destroy(cf_ctx *ctx);
 
 #ifdef __cplusplus

@@ -68,3 +68,20 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "_LIB_PATH", str(tmp_path / "libcf.so"))
     with pytest.raises(ImportError):
         b.lib()
+
+
+def test_every_call_names_its_source():
+    """Each function declared in include/cf.h carries, in the comment right
+    above it, a "Source:" line: the passage of the pages that defines the
+    operation, or the statement that it is library plumbing."""
+    src = open(os.path.join(ROOT, "include", "cf.h")).read()
+    missing = []
+    for m in re.finditer(r"/\*(?:(?!\*/).)*\*/\s*(?:typedef[^;]*;\s*|#define[^\n]*\n\s*)*"
+                         r"(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(cf_\w+)\s*\(", src, flags=re.S):
+        comment = m.group(0)[:m.group(0).rindex("*/")]
+        if "Source:" not in comment:
+            missing.append(m.group(1))
+    found = {m.group(1) for m in re.finditer(r"/\*(?:(?!\*/).)*\*/\s*(?:typedef[^;]*;\s*|#define[^\n]*\n\s*)*"
+                                             r"(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(cf_\w+)\s*\(", src, flags=re.S)}
+    assert found == set(declared_functions()), set(declared_functions()) ^ found
+    assert not missing, missing

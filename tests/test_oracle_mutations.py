@@ -32,6 +32,9 @@ MUTATIONS = [
      False),
     ("A^T dropped from the iteration", "mat_AtP(m, n, r, A, P, Q);", "(void)P;", False),
     ("Cholesky divisor", "R[p * r + q] = v / R[p * r + p];", "R[p * r + q] = v / diag;", False),
+    ("zero-group threshold at FLT_MIN", "CFO_SCALE_MIN = 7.52316384526264e-37f;", "CFO_SCALE_MIN = 1.17549435e-38f;",
+     False),
+    ("zero-group threshold inclusive", "} else if (s < CFO_SCALE_MIN) {", "} else if (s <= CFO_SCALE_MIN) {", False),
 ]
 
 

@@ -17,53 +17,25 @@ import torch
 
 import synth
 
-GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quant_worked_groups.txt")
-
-
-def bf16(values):
-    t = torch.tensor(values, dtype=torch.float32)
-    b = t.to(torch.bfloat16)
-    assert torch.equal(b.float(), t), "fixture values must be exact in bf16"
-    return b.view(torch.int16).numpy().view(np.uint16).copy()
-
-
-def read_golden():
-    cases, cur = {}, None
-    for line in open(GOLDEN):
-        line = line.strip()
-        if not line or line.startswith("#"):
-            continue
-        if line.startswith("["):
-            cur = cases.setdefault(line[1:-1], {})
-            continue
-        k, v = [s.strip() for s in line.split("=", 1)]
-        cur[k] = v
-    return cases
-
-
-def floats(s):
-    return np.array([float(v) for v in s.split(",")], np.float32)
-
-
-CASES = read_golden()
+from goldens import CASES, bf16, floats, num  # noqa: E402
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_hand_worked_group(oracle, name):
     c = CASES[name]
     bits, group, ss = int(c["bits"]), int(c["group"]), int(c["sign_scale"])
-    x = bf16([float(v) for v in c["x"].split(",")])
-    base = bf16([float(v) for v in c["base"].split(",")])
+    x = bf16([num(v) for v in c["x"].split(",")])
+    base = bf16([num(v) for v in c["base"].split(",")])
     if c.get("state") == "bf16":
-        err = bf16([float(v) for v in c["e"].split(",")])
-        cache = bf16([float(v) for v in c["cache"].split(",")])
+        err = bf16([num(v) for v in c["e"].split(",")])
+        cache = bf16([num(v) for v in c["cache"].split(",")])
         codes, scales, flags = oracle.compress_lean(x, base, err, bits, group, ss)
         assert flags == 0
         assert codes.tobytes() == bytes(int(b, 16) for b in c["bytes"].split(","))
-        assert scales.tolist() == [float(c["scale"])]
-        assert np.array_equal(err, bf16([float(v) for v in c["e_new"].split(",")]))
+        assert scales.tolist() == [num(c["scale"])]
+        assert np.array_equal(err, bf16([num(v) for v in c["e_new"].split(",")]))
         oracle.decompress_lean(codes, scales, cache, bits, group)
-        assert np.array_equal(cache, bf16([float(v) for v in c["cache_new"].split(",")]))
+        assert np.array_equal(cache, bf16([num(v) for v in c["cache_new"].split(",")]))
         return
     err = floats(c["e"])
     cache = floats(c["cache"])
@@ -71,7 +43,7 @@ def test_hand_worked_group(oracle, name):
     assert flags == 0
     want_bytes = bytes(int(b, 16) for b in c["bytes"].split(","))
     assert codes.tobytes() == want_bytes
-    assert scales.tolist() == [float(c["scale"])]
+    assert scales.tolist() == [num(c["scale"])]
     # the per-element codes, read back through numpy's own bit routine
     bitstream = np.unpackbits(codes, bitorder="little")
     got = [int(sum(int(bitstream[j * bits + b]) << b for b in range(bits))) for j in range(group)]
@@ -80,7 +52,7 @@ def test_hand_worked_group(oracle, name):
     assert np.array_equal(base, x)
     oracle.decompress(codes, scales, cache, bits, group)
     d_want = floats(c["d"])
-    s = float(c["scale"])
+    s = num(c["scale"])
     if "d_exact_mask" in c:
         mask = np.array([int(v) for v in c["d_exact_mask"].split(",")], bool)
         d_got = cache - floats(c["cache"])
