@@ -81,7 +81,8 @@ def check(oracle, As, Q0s, out, T, idx=None):
 # Ragged shapes in both dimensions (m and n not multiples of the 128-row
 # tile or the 32-column box), full-width rows (n = 3072) and wider (3200),
 # r from 1 to 32 (padded to 16 or 32 columns), T from 0 to 4, all within the
-# 1e-3 bar.  Where Algorithm 3 is still far from converged (r a large
+# 1e-3 bar.  Tall blocks (m = 8320, 8200) give the CholeskyQR of P 33 Gram
+# chunks per matrix.  Where Algorithm 3 is still far from converged (r a large
 # fraction of the smaller dimension with few iterations, e.g. 192 x 128 at
 # r = 32, T = 2) the result follows every rounding of the products: TF32
 # operands gave 1.6e-3 there in a CPU simulation of the kernels, so the
@@ -89,7 +90,7 @@ def check(oracle, As, Q0s, out, T, idx=None):
 @pytest.mark.parametrize("m,n,r,T", [(256, 256, 16, 2), (300, 200, 16, 2), (4444 // 4, 1920 // 4, 16, 2),
                                      (200, 72, 8, 2), (160, 96, 24, 1), (320, 256, 32, 2), (192, 128, 32, 4),
                                      (192, 128, 32, 2), (130, 64, 16, 0), (128, 128, 1, 3), (700, 1000, 16, 2),
-                                     (300, 3072, 16, 2), (256, 3200, 8, 1)])
+                                     (300, 3072, 16, 2), (256, 3200, 8, 1), (8320, 256, 16, 1), (8200, 96, 24, 1)])
 def test_lowrank_matches_oracle(cf, oracle, m, n, r, T):
     k = 3
     As = [synth.lowrank_matrix(m, n, r, mat=i, noise=0.01) for i in range(k)]
