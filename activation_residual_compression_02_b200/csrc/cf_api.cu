@@ -50,6 +50,7 @@ struct cf_ctx {
     bool warm_sender = false;
     bool warm_receiver = false;
     int64_t lowrank_steps = 0;   // compressed low-rank steps done (for warm_start)
+    bool starve_once = false;    // failure-detection test: the next cf_lowrank withholds its loads
     int device = 0;
     std::string err;
 };
@@ -431,6 +432,12 @@ try {
     if (!ctx) return CF_E_NOMEM;
     ctx->cfg = *config;
     ctx->device = dev;
+    // Failure-detection test hook, read once here: with CF_TEST_STARVE_GEMM=1
+    // in the environment when the context is created, the context's first
+    // cf_lowrank call issues no loads in its products, so their bounded waits
+    // run out and the next cf_check reports CF_E_TIMEOUT (no GPU fault).
+    const char *starve = getenv("CF_TEST_STARVE_GEMM");
+    ctx->starve_once = config->mode == CF_MODE_LOWRANK && starve && starve[0] == '1';
     try {
         ctx->shapes.assign(shapes, shapes + nslots);
     } catch (const std::bad_alloc &) {
@@ -560,6 +567,8 @@ try {
     plan.r = r;
     plan.T = ctx->cfg.iters;
     plan.split = split;
+    plan.starve = ctx->starve_once;
+    ctx->starve_once = false;
     plan.ws = ctx->ws;
     plan.ws_bytes = ctx->ws_bytes;
     plan.status = ctx->d_status;

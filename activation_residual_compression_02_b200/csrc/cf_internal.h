@@ -69,6 +69,7 @@ struct LowrankPlan {
     int64_t m, n;
     int r, T;
     bool split;        // split (3xTF32) products, see lowrank_split
+    bool starve;       // failure-detection test only: the products' loads are withheld (bounded waits time out)
     void *ws;          // device workspace
     size_t ws_bytes;
     uint32_t *status;

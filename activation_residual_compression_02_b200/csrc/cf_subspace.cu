@@ -1110,12 +1110,11 @@ cudaError_t gemm_pass(const LowrankPlan &pl, const LowrankMat *mats, const WsLay
         gp->out_mode = out_mode;
         gp->status = pl.status;
         gp->wait_ns = kWaitNs;
-        // Fault injection for the failure-detection test: with
-        // CF_TEST_STARVE_GEMM=1 the producer loads nothing, so the consumers'
-        // bounded waits on the "tile landed" barriers run out (after 20 ms) and
-        // the kernel returns with the timeout bit set in the status word.
-        const char *starve = getenv("CF_TEST_STARVE_GEMM");
-        if (starve && starve[0] == '1') {
+        // Fault injection for the failure-detection test (see LowrankPlan::starve):
+        // the producer loads nothing, so the consumers' bounded waits on the
+        // "tile landed" barriers run out (after 20 ms) and the kernel returns
+        // with the timeout bit set in the status word.
+        if (pl.starve) {
             gp->starve = 1;
             gp->wait_ns = 20000000ull;
         }

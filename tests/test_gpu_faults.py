@@ -1,11 +1,12 @@
 """Failure detection on the GPU without a fault.
 
 Every mbarrier wait in the tcgen05 GEMM is bounded.  The fault-injection hook
-CF_TEST_STARVE_GEMM=1 makes the TMA producer issue no loads, so the consumers
-wait on barriers that nothing completes; the wait gives up after 20 ms, the
-kernel drains, frees its tensor memory and returns, and cf_check reports
-CF_E_TIMEOUT.  The context and the device stay usable: the next call, without
-the hook, succeeds and matches the oracle.
+CF_TEST_STARVE_GEMM=1, read when a low-rank context is created, makes the TMA
+producer of that context's first cf_lowrank call issue no loads, so the
+consumers wait on barriers that nothing completes; the wait gives up after
+20 ms, the kernel drains, frees its tensor memory and returns, and cf_check
+reports CF_E_TIMEOUT.  The context and the device stay usable: the next call
+on the same context succeeds and matches the oracle.
 """
 import os
 
@@ -32,16 +33,17 @@ def test_bounded_wait_times_out_and_context_survives(cf, oracle):
     m, n, r, T = 256, 192, 16, 2
     A = [synth.lowrank_matrix(m, n, r, mat=11, device="cuda")]
     Q0 = [synth.q0(n, r, seed=0, mat=11, device="cuda")]
-    ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+    # the hook is read when the context is created and starves its first call only
+    os.environ["CF_TEST_STARVE_GEMM"] = "1"
+    try:
+        ctx = cf.Context([], mode=cf.CF_MODE_LOWRANK, rank=r, iters=T)
+    finally:
+        del os.environ["CF_TEST_STARVE_GEMM"]
     ws = torch.empty(ctx.lowrank_workspace_bytes(1, m, n), dtype=torch.uint8, device="cuda")
     ctx.set_workspace(ws)
     U, R, V = [torch.empty(m, r, device="cuda")], [torch.empty(r, r, device="cuda")], [torch.empty(n, r, device="cuda")]
-    os.environ["CF_TEST_STARVE_GEMM"] = "1"
-    try:
-        ctx.lowrank(A, Q0, U, R, V)
-        status = ctx.check()
-    finally:
-        del os.environ["CF_TEST_STARVE_GEMM"]
+    ctx.lowrank(A, Q0, U, R, V)
+    status = ctx.check()
     assert status == cf.CF_E_TIMEOUT
     # the status word was cleared by the read, and the context still works
     ctx.lowrank(A, Q0, U, R, V)
