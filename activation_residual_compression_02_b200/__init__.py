@@ -13,7 +13,7 @@ builds the library and marshals arguments.
 from ._cf import (  # noqa: F401
     CF_E_ALIGN, CF_E_ARG, CF_E_CUDA, CF_E_NOMEM, CF_E_NONFINITE, CF_E_SHAPE, CF_E_STATE, CF_E_TIMEOUT,
     CF_MODE_LOWRANK, CF_MODE_QUANT, CF_OK, CF_PRECISION_AUTO, CF_PRECISION_SPLIT, CF_PRECISION_TF32, EXPORTED,
-    CfError, Context, Slot, cf_check, cf_compress, cf_config, cf_create, cf_decompress, cf_destroy, cf_loopback, cf_lowrank, cf_lowrank_noalloc, cf_payload_bytes, lib,
+    KV, CfError, Context, Slot, cf_check, cf_compress, cf_config, cf_create, cf_kv, cf_decompress, cf_destroy, cf_loopback, cf_lowrank, cf_lowrank_noalloc, cf_payload_bytes, lib,
     NOALLOC_SCRATCH_BYTES,
 )
 from .state import HostStreamCodec, QuantState, alloc_quant_state  # noqa: F401

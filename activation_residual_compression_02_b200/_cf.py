@@ -23,7 +23,8 @@ CF_PRECISION_AUTO, CF_PRECISION_TF32, CF_PRECISION_SPLIT = 0, 1, 2
 
 EXPORTED = ["cf_create", "cf_workspace_bytes", "cf_set_workspace", "cf_compress", "cf_decompress",
             "cf_lowrank_workspace_bytes", "cf_lowrank", "cf_check", "cf_payload_bytes", "cf_last_error",
-            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback", "cf_resume", "cf_trace_enable", "cf_trace_read"]
+            "cf_destroy", "cf_lowrank_noalloc", "cf_loopback", "cf_resume", "cf_trace_enable", "cf_trace_read",
+            "cf_attention"]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -46,6 +47,11 @@ class cf_slot(ctypes.Structure):
                 ("cache", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("q0", ctypes.c_void_p), ("U", ctypes.c_void_p), ("R", ctypes.c_void_p), ("V", ctypes.c_void_p),
                 ("recon", ctypes.c_void_p)]
+
+
+class cf_kv(ctypes.Structure):
+    _fields_ = [("bf16", ctypes.c_void_p), ("cache_in", ctypes.c_void_p), ("cache_out", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
 
 
 class CfError(RuntimeError):
@@ -99,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.cf_trace_read.restype = I
         L.cf_lowrank_noalloc.argtypes = [ctypes.POINTER(cf_config), I, I64, I64, PP, PP, PP, PP, PP, PP, PP, P]
         L.cf_lowrank_noalloc.restype = I
+        L.cf_attention.argtypes = [P, I64, I64, I64, P, ctypes.POINTER(cf_kv), ctypes.POINTER(cf_kv), P, P]
+        L.cf_attention.restype = I
         _lib = L
     return _lib
 
@@ -140,6 +148,33 @@ class Slot:
 
     def to_c(self) -> cf_slot:
         return cf_slot(*[_ptr(getattr(self, f)) for f in Slot.__slots__])
+
+
+class KV:
+    """K or V of a received shard for ``Context.attention`` (``cf_kv``): either
+    ``bf16`` [lk, cols], or the receiver's ``cache_in`` [lk, cols] fp32 with
+    this step's ``codes`` and ``scales`` (dequantise-on-load; ``cache_out``
+    [lk, cols] fp32 receives the updated cache)."""
+
+    __slots__ = ("bf16", "cache_in", "cache_out", "codes", "scales")
+
+    def __init__(self, bf16=None, cache_in=None, cache_out=None, codes=None, scales=None):
+        self.bf16, self.cache_in, self.cache_out, self.codes, self.scales = bf16, cache_in, cache_out, codes, scales
+
+    def to_c(self) -> cf_kv:
+        return cf_kv(*[_ptr(getattr(self, f)) for f in KV.__slots__])
+
+    def check(self, lk: int, cols: int, bits: int, group: int, name: str):
+        want = {"bf16": (torch.bfloat16, lk * cols), "cache_in": (torch.float32, lk * cols),
+                "cache_out": (torch.float32, lk * cols), "codes": (torch.uint8, lk * cols * bits // 8),
+                "scales": (torch.float32, lk * cols // group if group else 0)}
+        for f in KV.__slots__:
+            t = getattr(self, f)
+            if t is None:
+                continue
+            dt, n = want[f]
+            if t.dtype != dt or t.numel() != n:
+                raise ValueError(f"{name}.{f} must be {dt} with {n} elements, not {t.dtype} with {t.numel()}")
 
 
 class Context:
@@ -218,6 +253,23 @@ class Context:
         st = lib().cf_lowrank(self._h, nmat, m, n, _parr(A), _parr(Q0), _parr(U), _parr(R), _parr(V), _parr(E),
                               _parr(C), _stream_handle(stream))
         self._raise(st, "cf_lowrank")
+
+    def attention(self, q: torch.Tensor, k: KV, v: KV, out: torch.Tensor, lk: Optional[int] = None,
+                  stream: Optional[torch.cuda.Stream] = None):
+        """cf_attention: out = softmax(q k^T / 8) v per head of 64 channels.
+        q and out are bf16 [lq, cols]; lk defaults to the rows of k's tensors."""
+        if q.dim() != 2 or q.dtype != torch.bfloat16 or out.dtype != torch.bfloat16 or out.shape != q.shape:
+            raise ValueError("q and out must be bf16 [lq, cols] of the same shape")
+        lq, cols = int(q.shape[0]), int(q.shape[1])
+        if lk is None:
+            t = k.bf16 if k.bf16 is not None else k.cache_in
+            lk = int(t.numel() // cols) if t is not None else 0
+        for kv, name in ((k, "k"), (v, "v")):
+            kv.check(lk, cols, self.cfg.bits, self.cfg.group, name)
+        kc, vc = k.to_c(), v.to_c()
+        st = lib().cf_attention(self._h, lq, lk, cols, _ptr(q), ctypes.byref(kc), ctypes.byref(vc), _ptr(out),
+                                _stream_handle(stream))
+        self._raise(st, "cf_attention")
 
     def trace(self, on: bool = True):
         """Time every kernel launch of this context with CUDA events (cf_trace_enable)."""

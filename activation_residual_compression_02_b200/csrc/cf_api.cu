@@ -582,6 +582,80 @@ try {
     return CF_E_ARG;
 }
 
+namespace {
+bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return a && b && x < y + nb && y < x + na;
+}
+}  // namespace
+
+cf_status cf_attention(cf_ctx *ctx, int64_t lq, int64_t lk, int64_t cols, const void *q, const cf_kv *k,
+                       const cf_kv *v, void *out, void *cuda_stream)
+try {
+    if (!ctx) return CF_E_ARG;
+    DeviceGuard device(ctx);
+    TraceGuard trace(ctx);
+    if (lq < 0 || lk < 1 || cols < 64 || cols % 64 != 0)
+        return fail(ctx, CF_E_SHAPE, "need lq >= 0, lk >= 1 and cols a positive multiple of 64 (heads of 64)");
+    if (lq > ((int64_t)1 << 40) / cols || lk > ((int64_t)1 << 40) / cols || cols / 64 > 65535 ||
+        lq > INT32_MAX || lk > INT32_MAX)
+        return fail(ctx, CF_E_SHAPE, "shard too large");
+    if (lq == 0) return CF_OK;
+    if (!q || !k || !v || !out) return fail(ctx, CF_E_ARG, "q, k, v and out must be non-NULL");
+    if (!aligned16(q) || !aligned16(out)) return fail(ctx, CF_E_ALIGN, "q and out must be 16-byte aligned");
+    const bool deq = k->bf16 == nullptr;
+    if ((v->bf16 == nullptr) != deq) return fail(ctx, CF_E_ARG, "k and v must come in the same form");
+    cf::AttnArgs a{};
+    a.q = q;
+    a.out = out;
+    a.lq = lq;
+    a.lk = lk;
+    a.cols = cols;
+    a.dequantise = deq;
+    a.status = ctx->d_status;
+    const cf_kv *kv[2] = {k, v};
+    const size_t state_bytes = (size_t)lk * (size_t)cols * 4;
+    for (int i = 0; i < 2; ++i) {
+        const cf_kv &t = *kv[i];
+        if (!deq) {
+            if (!aligned16(t.bf16)) return fail(ctx, CF_E_ALIGN, "k/v bf16 must be 16-byte aligned");
+            a.kv[i] = t.bf16;
+            continue;
+        }
+        if (ctx->cfg.mode != CF_MODE_QUANT || ctx->cfg.state_bf16)
+            return fail(ctx, CF_E_ARG, "dequantise-on-load needs a quantised-mode context with fp32 state");
+        if (cols % ctx->cfg.group != 0) return fail(ctx, CF_E_SHAPE, "cols must be a multiple of the group size");
+        if (!t.cache_in || !t.codes || !t.scales)
+            return fail(ctx, CF_E_ARG, "dequantise-on-load needs cache_in, codes and scales");
+        if (!aligned16(t.cache_in) || !aligned16(t.cache_out) || !aligned16(t.codes) || !aligned16(t.scales))
+            return fail(ctx, CF_E_ALIGN, "k/v state and payload must be 16-byte aligned");
+        a.cache_in[i] = t.cache_in;
+        a.cache_out[i] = t.cache_out;
+        a.codes[i] = t.codes;
+        a.scales[i] = t.scales;
+    }
+    if (deq) {
+        // the CTAs of the first query block write C_t while the others still read C_{t-1}
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 2; ++j)
+                if (ranges_overlap(a.cache_out[i], state_bytes, a.cache_in[j], state_bytes))
+                    return fail(ctx, CF_E_ARG, "cache_out must not overlap cache_in");
+        if (ranges_overlap(a.cache_out[0], state_bytes, a.cache_out[1], state_bytes))
+            return fail(ctx, CF_E_ARG, "the cache_out of k and v overlap");
+        a.bits = ctx->cfg.bits;
+        a.group = ctx->cfg.group;
+    }
+    cudaError_t e = cf::launch_attention(a, (cudaStream_t)cuda_stream);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "cf_attention");
+    ctx->err.clear();
+    return CF_OK;
+} catch (const std::bad_alloc &) {
+    return CF_E_NOMEM;
+} catch (...) {
+    return CF_E_ARG;
+}
+
 cf_status cf_check(cf_ctx *ctx, void *cuda_stream)
 {
     if (!ctx) return CF_E_ARG;

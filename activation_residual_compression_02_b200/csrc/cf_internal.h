@@ -93,6 +93,24 @@ cudaError_t run_lowrank_decompress(const LowrankPlan &plan, const LowrankMat *ma
 cudaError_t launch_residual_f32(const void *const *x, void *const *base, const float *const *err,
                                 float *const *a_out, const int64_t *n, int nslots, cudaStream_t stream);
 
+// Attention over a received K/V shard (cf_attention): heads of 64 channels,
+// K and V as bf16 (kv) or dequantised on load from cache_in + codes/scales
+// (dequantise = true), the new cache written to cache_out when non-null.
+struct AttnArgs {
+    const void *q;
+    const void *kv[2];
+    const float *cache_in[2];
+    float *cache_out[2];
+    const uint8_t *codes[2];
+    const float *scales[2];
+    void *out;
+    int64_t lq, lk, cols;
+    int bits, group;
+    bool dequantise;
+    uint32_t *status;
+};
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);
+
 int num_sms();
 
 // Host-side launch log: with CF_LOG=1 in the environment (read once), every

@@ -249,6 +249,43 @@ cf_status cf_lowrank(cf_ctx *ctx, int nmat, int64_t m, int64_t n, const float *c
                      const float *const *Q0, float *const *U, float *const *R, float *const *V,
                      float *const *E_opt, float *const *C_opt, void *cuda_stream);
 
+/* K or V of a received shard for cf_attention, in one of two forms:
+ *   bf16 != NULL : the tensor in bf16, e.g. a slot's recon (bf16 of the
+ *                  receiver's cache, written by cf_decompress in its pass);
+ *   bf16 == NULL : dequantise-on-load -- the receiver's cache C_{t-1} and
+ *                  this step's payload; the attention forms
+ *                  C_t = C_{t-1} + deq(codes, scales) exactly as cf_decompress
+ *                  does, uses bf16(C_t) and writes C_t to cache_out (if not
+ *                  NULL), so the receiver needs no separate decompress. */
+typedef struct cf_kv {
+    const void *bf16;         /* bf16 [rows*cols], or NULL for dequantise-on-load */
+    const float *cache_in;    /* fp32 [rows*cols]: C_{t-1} (read only) */
+    float *cache_out;         /* fp32 [rows*cols]: C_t, or NULL; must not overlap any cache_in */
+    const uint8_t *codes;     /* this step's codes (the context's k), rows*cols*k/8 bytes */
+    const float *scales;      /* this step's scales (the context's G), rows*cols/G */
+} cf_kv;
+
+/* Attention of a shard's queries over a received K/V shard, per head of 64
+ * channels: for head h (channels [64 h, 64 h + 64) of the token-major
+ * layout), out_h = softmax(q_h k_h^T / 8) v_h.
+ *   q, out  bf16 [lq x cols] (16-byte aligned); k, v of [lk x cols], both in
+ *   the same cf_kv form; cols a multiple of 64 (and of G when dequantising).
+ * The products run on the tensor cores in bf16 with fp32 accumulation, the
+ * softmax in fp32 (base 2, online over blocks of 128 keys, P rounded to bf16).
+ * Dequantise-on-load needs a quantised-mode context with fp32 state (its k
+ * and G describe the payload); the bf16 form only uses the context's status
+ * word.  The two forms give bit-identical outputs for the same C_t.
+ * Stream-ordered; allocates nothing.  Errors before launch: CF_E_ARG (NULL
+ * pointer, mixed forms, overlapping caches, wrong context), CF_E_SHAPE (lk <
+ * 1, cols not a multiple of 64 or of G), CF_E_ALIGN; device-side:
+ * CF_E_TIMEOUT at the next cf_check.
+ * Source: reproducibility table, "Pseudocode" row, Algorithms 1 and 2 (each
+ * device attends over the key/value blocks it receives from the others);
+ * abstract (the receiver adds each decompressed residual to its
+ * reconstruction). */
+cf_status cf_attention(cf_ctx *ctx, int64_t lq, int64_t lk, int64_t cols, const void *q, const cf_kv *k,
+                       const cf_kv *v, void *out, void *cuda_stream);
+
 /* Bytes of device scratch that the library keeps on every GPU it is loaded
  * on, for cf_lowrank_noalloc (status word plus the Algorithm 3 buffers). */
 #define CF_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)

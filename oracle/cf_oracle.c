@@ -483,3 +483,47 @@ int cfo_decompress_lean(int64_t n, int k, int G, const uint8_t *codes, const flo
     }
     return CFO_OK;
 }
+
+/* ------------------------------------------------------------ attention -- */
+
+/* "Accelerating Parallel Diffusion Model Serving with Residual Compression",
+ * reproducibility table, "Pseudocode" row, Algorithms 1 and 2: each device
+ * attends with its queries over the key/value blocks it receives.  Standard
+ * scaled dot-product attention per head of 64 channels (channels
+ * [64 h, 64 h + 64) of the token-major layout), in fp64:
+ *   score(i, j) = (q_i . k_j) / 8          (8 = sqrt(64))
+ *   w(i, j)     = exp(score(i, j) - max_j score(i, j)) / sum_j (same)
+ *   out(i, c)   = sum_j w(i, j) v(j, c)
+ * q, k, v are bf16 bit patterns; out is fp64 [lq x cols]. */
+int cfo_attention(int64_t lq, int64_t lk, int64_t cols, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  double *out)
+{
+    if (lq < 0 || lk < 1 || cols < 64 || cols % 64 != 0) return CFO_E_ARG;
+    double *w = (double *)malloc((size_t)lk * sizeof(double));
+    if (!w) return CFO_E_NOMEM;
+    for (int64_t h = 0; h < cols / 64; ++h) {
+        const int64_t c0 = h * 64;
+        for (int64_t i = 0; i < lq; ++i) {
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < lk; ++j) {
+                double s = 0.0;
+                for (int c = 0; c < 64; ++c)
+                    s += (double)bf16_to_float(q[i * cols + c0 + c]) * (double)bf16_to_float(k[j * cols + c0 + c]);
+                w[j] = s / 8.0;
+                if (w[j] > mx) mx = w[j];
+            }
+            double z = 0.0;
+            for (int64_t j = 0; j < lk; ++j) {
+                w[j] = exp(w[j] - mx);
+                z += w[j];
+            }
+            for (int c = 0; c < 64; ++c) {
+                double o = 0.0;
+                for (int64_t j = 0; j < lk; ++j) o += w[j] * (double)bf16_to_float(v[j * cols + c0 + c]);
+                out[i * cols + c0 + c] = o / z;
+            }
+        }
+    }
+    free(w);
+    return CFO_OK;
+}

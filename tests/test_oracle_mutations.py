@@ -14,7 +14,8 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "cf_oracle.c")
-PINS = [os.path.join(ROOT, "tests", "test_oracle_quant.py"), os.path.join(ROOT, "tests", "test_oracle_lowrank.py")]
+PINS = [os.path.join(ROOT, "tests", "test_oracle_quant.py"), os.path.join(ROOT, "tests", "test_oracle_lowrank.py"),
+        os.path.join(ROOT, "tests", "test_oracle_attention.py")]
 
 # (name, text in cf_oracle.c, replacement, replace every occurrence)
 MUTATIONS = [
@@ -35,6 +36,9 @@ MUTATIONS = [
     ("zero-group threshold at FLT_MIN", "CFO_SCALE_MIN = 7.52316384526264e-37f;", "CFO_SCALE_MIN = 1.17549435e-38f;",
      False),
     ("zero-group threshold inclusive", "} else if (s < CFO_SCALE_MIN) {", "} else if (s <= CFO_SCALE_MIN) {", False),
+    ("attention scale 1/64", "w[j] = s / 8.0;", "w[j] = s / 64.0;", False),
+    ("softmax max not taken out", "w[j] = exp(w[j] - mx);", "w[j] = exp(w[j]);", False),
+    ("softmax not normalised", "out[i * cols + c0 + c] = o / z;", "out[i * cols + c0 + c] = o;", False),
 ]
 
 
