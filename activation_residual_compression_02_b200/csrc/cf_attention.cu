@@ -30,9 +30,15 @@
 //   warp 4     allocates TMEM (S: 128 columns, O: 64) and issues
 //              tcgen05.mma.kind::f16 (bf16 operands, fp32 accumulators):
 //              S = Q K^T, then O += P V;
-//   warps 5-7  load Q once, then K and V blocks into a two-deep ring
-//              (K-major, 128-byte swizzle; V transposed in registers so that
-//              every operand is K-major).
+//   warps 5-7  load Q once (TMA), then K and V blocks into a two-deep ring:
+//              in the bf16 form by TMA (a [128 x 64] box with the 128-byte
+//              swizzle lands in the layout the MMA reads); in the other, the
+//              fp32 cache rows of 32-key sub-chunks by TMA and their codes and
+//              scales by cp.async into a ring of staging slots, three
+//              sub-chunks ahead of the one being dequantised and stored
+//              swizzled.  Q and K are K-major operands;
+//              V is read MN-major (the channels of a key are contiguous), so
+//              no operand is transposed.
 // Every mbarrier wait is bounded; on expiry the CTA raises an abort flag and
 // the status word's timeout bit, drains its MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -57,8 +63,18 @@ constexpr int kLoaders = 96;           // warps 5-7
 constexpr int kRing = 2;               // K/V blocks in flight
 constexpr int kTileBytes = 128 * kHeadDim * 2;   // a 128 x 64 bf16 tile: 16 KB
 constexpr uint64_t kAttnWaitNs = 2000000000ull;
+// Dequantise-on-load staging: sub-chunks of 32 keys (K and V: fp32 cache,
+// codes, scales) stream through a ring of kSlots shared-memory slots.
+constexpr int kSub = 32;
+constexpr int kSlots = 4;
+constexpr int kSlotC = 2 * kSub * kHeadDim * 4;     // 16 KB of cache
+constexpr int kSlotCodes = 2 * kSub * 32;           // up to 32 code bytes per key row (k = 4)
+constexpr int kSlotScales = 2 * kSub * 8 * 4;       // up to 8 scales per key row (G = 8)
+constexpr int kSlotBytes = kSlotC + kSlotCodes + kSlotScales;
 
 struct AttnSmem {
+    uint64_t st_full[kSlots];     // staging slot landed (TMA bytes + every loader's cp.async)
+    uint64_t st_free[kSlots];     // staging slot read by the three loader warps
     uint64_t q_full;
     uint64_t ld_full[kRing];
     uint64_t ld_free[kRing];
@@ -72,7 +88,10 @@ struct AttnSmem {
     float lut[16];
 };
 
-struct AttnParams {
+struct __align__(64) AttnParams {
+    CUtensorMap tq;               // Q, bf16 [lq x cols], box 64 x 128
+    CUtensorMap tk, tv;           // K, V (bf16 form), same boxes
+    CUtensorMap tc[2];            // cache_in of K and V (dequantise form), fp32, box 64 x 32
     const uint16_t *q;            // bf16 [lq x cols]
     const uint16_t *kv[2];        // bf16 [lk x cols] (form 0)
     const float *cache_in[2];     // fp32 [lk x cols] (form 1)
@@ -82,6 +101,7 @@ struct AttnParams {
     uint16_t *out;                // bf16 [lq x cols]
     int lq, lk, cols;
     int group;
+    int group_lg;                 // log2(group)
     float scale_log2;             // log2(e) / sqrt(64)
     uint32_t *status;
     unsigned long long wait_ns;
@@ -100,10 +120,21 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M = 128.
-__device__ __forceinline__ uint32_t instr_desc_bf16(int n)
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, A K-major, B K-major
+// or MN-major (b_mn), M = 128.
+__device__ __forceinline__ uint32_t instr_desc_bf16(int n, int b_mn)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBlockQ >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(kBlockQ >> 4) << 24);
+}
+
+// 2^x on the special-function unit (ex2.approx: a relative error near 2^-22,
+// below the bf16 rounding P gets next).
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
@@ -128,7 +159,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// K-major [rows x 64] bf16 tile, 128-byte swizzle: 8-row groups 1 KB apart.
 __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, kLayoutSw128); }
+// MN-major [keys x 64] bf16 tile (V: 64 channels of a key contiguous), 128-byte
+// swizzle: one 64-wide atom along N, 8-key groups 1 KB apart along K.  Both
+// offsets are 1 KB, so the single N atom reads the same either way.
+__device__ __forceinline__ uint64_t vdesc(uint32_t saddr) { return smem_desc(saddr, 1024, 1024, kLayoutSw128); }
 
 // A bounded wait whose outcome is the same for every lane of the warp, so that
 // the warp never splits across the .sync.aligned tcgen05 instructions after it.
@@ -139,70 +175,83 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-// Eight consecutive channels of K or V at flat element index i0 (a multiple
-// of 8), as four bf16 pairs.  FORM 0 reads bf16; FORM 1 forms C + deq as the
-// receiver's decompress does and, when `wb` is set, writes it to cache_out.
-template <int FORM, int K>
-__device__ __forceinline__ void load8(const AttnParams &p, int which, int64_t i0, bool wb, const float *lut,
-                                      uint32_t (&w)[4])
+__device__ __forceinline__ void cp_async(void *dst, const void *src, int bytes)
 {
-    if constexpr (FORM == 0) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.kv[which] + i0));
-        w[0] = v.x;
-        w[1] = v.y;
-        w[2] = v.z;
-        w[3] = v.w;
-    } else {
-        const int64_t v8 = i0 >> 3;
-        uint32_t code;
-        if constexpr (K == 4)
-            code = __ldg(reinterpret_cast<const uint32_t *>(p.codes[which]) + v8);
-        else if constexpr (K == 2)
-            code = __ldg(reinterpret_cast<const uint16_t *>(p.codes[which]) + v8);
-        else
-            code = __ldg(p.codes[which] + v8);
-        const float s = __ldg(p.scales[which] + i0 / p.group);
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(p.cache_in[which] + i0));
-        const float4 b = __ldg(reinterpret_cast<const float4 *>(p.cache_in[which] + i0) + 1);
-        const float cin[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        float c[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t cj = (code >> (K * j)) & ((1u << K) - 1u);
-            const float d = (K >= 2) ? __fmul_rn(lut[cj], s) : (cj ? s : -s);
-            c[j] = __fadd_rn(cin[j], d);
-        }
-        if (wb) {
-            float4 *o = reinterpret_cast<float4 *>(p.cache_out[which] + i0);
-            o[0] = make_float4(c[0], c[1], c[2], c[3]);
-            o[1] = make_float4(c[4], c[5], c[6], c[7]);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) w[j] = bf16x2(c[2 * j], c[2 * j + 1]);
-    }
+    if (bytes == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    else if (bytes == 8)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+
+// Loads from shared memory by 32-bit shared-window address (the staging and
+// tile pointers are derived by arithmetic, which would otherwise make them
+// generic accesses).
+__device__ __forceinline__ float4 lds128(uint32_t a)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a)
+{
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds8(uint32_t a)
+{
+    unsigned short v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(a));
+    return v & 0xffu;
+}
+// The mbarrier gets one arrival once this thread's earlier cp.async copies
+// have landed (the arrival counts towards the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <int FORM, int K>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_constant__ AttnParams p)
 {
     extern __shared__ __align__(1024) uint8_t attn_smem[];
     uint8_t *base = (uint8_t *)(((uintptr_t)attn_smem + 1023) & ~(uintptr_t)1023);
-    uint8_t *sQ = base;                                    // [128 x 64] bf16
-    uint8_t *sK = sQ + kTileBytes;                         // kRing x [128 keys x 64]
-    uint8_t *sV = sK + kRing * kTileBytes;                 // kRing x 2 x [64 dims x 64 keys] (V transposed)
-    uint8_t *sP = sV + kRing * kTileBytes;                 // 2 x [128 queries x 64 keys]
-    AttnSmem *S = reinterpret_cast<AttnSmem *>(sP + 2 * kTileBytes);
+    uint8_t *sQ = base;                                    // [128 queries x 64] K-major
+    uint8_t *sK = sQ + kTileBytes;                         // kRing x [128 keys x 64] K-major
+    uint8_t *sV = sK + kRing * kTileBytes;                 // kRing x [128 keys x 64] (read MN-major)
+    uint8_t *sP = sV + kRing * kTileBytes;                 // 2 x [128 queries x 64 keys] K-major
+    uint8_t *sStage = sP + 2 * kTileBytes;                 // dequantise-on-load: kSlots staging slots
+    AttnSmem *S = reinterpret_cast<AttnSmem *>(sStage + (FORM == 1 ? kSlots * kSlotBytes : 0));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb = blockIdx.x, head = blockIdx.y;
     const int q0 = qb * kBlockQ;
     const int nkb = (p.lk + kBlockK - 1) / kBlockK;
     const int col0 = head * kHeadDim;
+    constexpr uint32_t kLdArrivals = FORM == 0 ? 1u : (uint32_t)kLoaders;
 
     if (threadIdx.x == 0) {
-        mbar_init(&S->q_full, kLoaders);
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&S->st_full[i], kLoaders + 1);   // every loader's cp.async arrival + the TMA thread's
+            mbar_init(&S->st_free[i], kLoaders / 32);  // one arrival per loader warp
+        }
+        mbar_init(&S->q_full, 1);
         for (int b = 0; b < kRing; ++b) {
-            mbar_init(&S->ld_full[b], kLoaders);
+            mbar_init(&S->ld_full[b], kLdArrivals);
             mbar_init(&S->ld_free[b], 1);
         }
         mbar_init(&S->s_full, 1);
@@ -234,60 +283,126 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
     if (warp >= 5) {
         // ------------------------------------------------------- loaders --
         const int lt = threadIdx.x - 160;   // 0..kLoaders-1
-        // Q: 128 rows x 8 pieces; rows past lq are zero
-        for (int u = lt; u < kBlockQ * 8; u += kLoaders) {
-            const int row = u >> 3, ch = u & 7;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (q0 + row < p.lq) v = __ldg(reinterpret_cast<const uint4 *>(p.q + (int64_t)(q0 + row) * p.cols + col0 + 8 * ch));
-            *reinterpret_cast<uint4 *>(sQ + sw128(row, ch)) = v;
+        if (lt == 0) {
+            // Q by TMA; rows past lq read as zero
+            mbar_expect_tx(&S->q_full, (uint32_t)kTileBytes);
+            tma_load_2d(sQ, &p.tq, col0, q0, &S->q_full);
         }
-        fence_proxy_async();
-        mbar_arrive(&S->q_full);
-        const bool wb = FORM == 1 && qb == 0;
-        for (int j = 0; j < nkb; ++j) {
-            const int b = j % kRing;
-            if (j >= kRing && !warp_wait(&S->ld_free[b], (uint32_t)((j / kRing) - 1) & 1u, abort_flag, p.status, wait_ns))
-                break;
-            const int k0 = j * kBlockK;
-            uint8_t *tk = sK + b * kTileBytes;
-            uint8_t *tv = sV + b * kTileBytes;
-            // K: 128 keys x 8 pieces of 8 channels, K-major as loaded
-            for (int u = lt; u < kBlockK * 8; u += kLoaders) {
-                const int row = u >> 3, ch = u & 7;
-                uint32_t w[4] = {0u, 0u, 0u, 0u};
-                if (k0 + row < p.lk) load8<FORM, K>(p, 0, (int64_t)(k0 + row) * p.cols + col0 + 8 * ch, wb, S->lut, w);
-                *reinterpret_cast<uint4 *>(tk + sw128(row, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            // V: 8-key x 8-channel blocks, transposed in registers so that V^T
-            // (channels x keys) is K-major like the other operands
-            for (int bi = lt; bi < (kBlockK / 8) * 8; bi += kLoaders) {
-                const int kg = bi >> 3, dg = bi & 7;    // keys 8 kg .. 8 kg + 7, channels 8 dg .. 8 dg + 7
-                uint32_t in[8][4];
-#pragma unroll
-                for (int r = 0; r < 8; ++r) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) in[r][c] = 0u;
-                    const int key = k0 + 8 * kg + r;
-                    if (key < p.lk) load8<FORM, K>(p, 1, (int64_t)key * p.cols + col0 + 8 * dg, wb, S->lut, in[r]);
-                }
-                uint8_t *blk = tv + (kg >> 3) * (kTileBytes / 2);   // keys 0-63 or 64-127 of the block
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
-                    uint4 o;
-                    o.x = __byte_perm(in[0][c >> 1], in[1][c >> 1], sel);
-                    o.y = __byte_perm(in[2][c >> 1], in[3][c >> 1], sel);
-                    o.z = __byte_perm(in[4][c >> 1], in[5][c >> 1], sel);
-                    o.w = __byte_perm(in[6][c >> 1], in[7][c >> 1], sel);
-                    *reinterpret_cast<uint4 *>(blk + sw128(8 * dg + c, kg & 7)) = o;
+        if constexpr (FORM == 0) {
+            // K and V boxes by TMA (keys past lk read as zero), one thread
+            if (lt == 0) {
+                for (int j = 0; j < nkb; ++j) {
+                    const int b = j % kRing;
+                    if (j >= kRing &&
+                        !wait_bounded(&S->ld_free[b], (uint32_t)((j / kRing) - 1) & 1u, abort_flag, p.status, wait_ns))
+                        break;
+                    mbar_expect_tx(&S->ld_full[b], 2u * kTileBytes);
+                    tma_load_2d(sK + b * kTileBytes, &p.tk, col0, j * kBlockK, &S->ld_full[b]);
+                    tma_load_2d(sV + b * kTileBytes, &p.tv, col0, j * kBlockK, &S->ld_full[b]);
                 }
             }
-            fence_proxy_async();
-            mbar_arrive(&S->ld_full[b]);
+        } else {
+            // Dequantise-on-load.  Sub-chunk g (keys 32 g .. 32 g + 31 of K and
+            // V) is staged in slot g % kSlots: the fp32 cache rows by TMA (one
+            // 64 x 32 box per tensor, keys past lk zero-filled), the code bytes
+            // and scales by cp.async; the slot's mbarrier completes when all
+            // have landed.  Staging runs three sub-chunks ahead of the one being
+            // dequantised into the bf16 tiles of its key block.
+            const bool wb = qb == 0;                      // the first query block writes the new cache
+            const int ngs = nkb * (kBlockK / kSub);
+            constexpr int kCodeRow = 8 * K;                // code bytes per key row of a head (64 channels)
+            constexpr int kCodePiece = kCodeRow >= 16 ? 16 : kCodeRow;
+            constexpr int kCodePieces = kCodeRow / kCodePiece;
+            const int ns = p.group >= kHeadDim ? 1 : kHeadDim / p.group;   // scales per key row of a head
+            const int sc_piece = ns >= 4 ? 16 : 4 * ns;
+            const int sc_lg = ns == 8 ? 1 : 0;             // two 16-byte pieces at G = 8
+            const int cpg = p.cols / p.group, c0g = col0 / p.group;      // scale index = key * cpg + c0g
+            const uint32_t stage0 = smem_u32(sStage);
+            auto issue = [&](int g) {                     // every loader thread; the slot is free
+                const int k0 = g * kSub, slot = g & (kSlots - 1);
+                uint8_t *st = sStage + slot * kSlotBytes;
+                if (lt == 0) {
+                    mbar_expect_tx(&S->st_full[slot], 2u * kSub * kHeadDim * 4);
+                    tma_load_2d(st, &p.tc[0], col0, k0, &S->st_full[slot]);
+                    tma_load_2d(st + kSub * 256, &p.tc[1], col0, k0, &S->st_full[slot]);
+                }
+                for (int u = lt; u < 2 * kSub * kCodePieces; u += kLoaders) {
+                    const int w = u / (kSub * kCodePieces), rem = u - w * (kSub * kCodePieces);
+                    const int r = rem / kCodePieces, q = rem - r * kCodePieces;
+                    if (k0 + r < p.lk)
+                        cp_async(st + kSlotC + w * (kSub * 32) + r * 32 + q * kCodePiece,
+                                 p.codes[w] + ((int64_t)(k0 + r) * p.cols + col0) * K / 8 + q * kCodePiece, kCodePiece);
+                }
+                for (int u = lt; u < (2 * kSub) << sc_lg; u += kLoaders) {
+                    const int wr = u >> sc_lg, q = u & ((1 << sc_lg) - 1);
+                    const int w = wr >> 5, r = wr & (kSub - 1);
+                    if (k0 + r < p.lk)
+                        cp_async(st + kSlotC + kSlotCodes + w * (kSub * 32) + r * 32 + q * sc_piece,
+                                 p.scales[w] + (int64_t)(k0 + r) * cpg + c0g + q * (sc_piece / 4), sc_piece);
+                }
+                cp_async_arrive(&S->st_full[slot]);
+            };
+            bool ok = true;
+            for (int g = 0; g < kSlots - 1 && g < ngs; ++g) issue(g);
+            const uint32_t lut = smem_u32(S->lut);
+            for (int g = 0; g < ngs && ok; ++g) {
+                const int j = g / (kBlockK / kSub), sub = g % (kBlockK / kSub), b = j % kRing;
+                const int slot = g & (kSlots - 1);
+                // stage sub-chunk g + 3 into the slot of sub-chunk g - 1 once every loader warp has read it
+                const int gn = g + kSlots - 1;
+                if (gn < ngs) {
+                    if (gn >= kSlots && !warp_wait(&S->st_free[gn & (kSlots - 1)], (uint32_t)((gn / kSlots) - 1) & 1u,
+                                                   abort_flag, p.status, wait_ns))
+                        break;
+                    issue(gn);
+                }
+                if (!warp_wait(&S->st_full[slot], (uint32_t)(g / kSlots) & 1u, abort_flag, p.status, wait_ns)) break;
+                if (sub == 0 && j >= kRing &&
+                    !warp_wait(&S->ld_free[b], (uint32_t)((j / kRing) - 1) & 1u, abort_flag, p.status, wait_ns))
+                    break;
+                const uint32_t st = stage0 + (uint32_t)(slot * kSlotBytes);
+                const uint32_t tk = smem_u32(sK + b * kTileBytes), tv = smem_u32(sV + b * kTileBytes);
+                for (int u = lt; u < 2 * kSub * 8; u += kLoaders) {
+                    const int w = u >> 8, r = (u >> 3) & (kSub - 1), pc = u & 7;
+                    const int key = g * kSub + r;
+                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                    if (key < p.lk) {
+                        const uint32_t cs = st + (uint32_t)(w * (kSub * 256) + r * 256 + 32 * pc);
+                        const float4 a = lds128(cs), bb = lds128(cs + 16);
+                        const uint32_t cb = st + (uint32_t)(kSlotC + w * (kSub * 32) + r * 32 + K * pc);
+                        const uint32_t code = K == 4 ? lds32(cb) : (K == 2 ? lds16(cb) : lds8(cb));
+                        const float sc = __uint_as_float(lds32(st + (uint32_t)(kSlotC + kSlotCodes + w * (kSub * 32) +
+                                                                               r * 32 + 4 * ((8 * pc) >> p.group_lg))));
+                        const float cin[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+                        float c[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            // the decompress arithmetic: one binary32 multiply and one add, never fused
+                            const uint32_t ce = (code >> (K * e)) & ((1u << K) - 1u);
+                            const float d = (K >= 2) ? __fmul_rn(__uint_as_float(lds32(lut + 4 * ce)), sc) : (ce ? sc : -sc);
+                            c[e] = __fadd_rn(cin[e], d);
+                        }
+                        if (wb) {
+                            float4 *dst = reinterpret_cast<float4 *>(p.cache_out[w] + (int64_t)key * p.cols + col0 + 8 * pc);
+                            dst[0] = make_float4(c[0], c[1], c[2], c[3]);
+                            dst[1] = make_float4(c[4], c[5], c[6], c[7]);
+                        }
+                        o = make_uint4(bf16x2(c[0], c[1]), bf16x2(c[2], c[3]), bf16x2(c[4], c[5]), bf16x2(c[6], c[7]));
+                    }
+                    sts128((w ? tv : tk) + sw128(sub * kSub + r, pc), o);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S->st_free[slot]);
+                if (sub == kBlockK / kSub - 1) {
+                    fence_proxy_async();
+                    mbar_arrive(&S->ld_full[b]);
+                }
+            }
+            cp_wait_all();
         }
     } else if (warp == 4) {
         // ---------------------------------------------------- MMA issuer --
-        const uint32_t idS = instr_desc_bf16(kBlockK), idO = instr_desc_bf16(kHeadDim);
+        const uint32_t idS = instr_desc_bf16(kBlockK, 0), idO = instr_desc_bf16(kHeadDim, 1);
         const uint32_t aQ = smem_u32(sQ);
         bool ok = warp_wait(&S->q_full, 0u, abort_flag, p.status, wait_ns) &&
                   warp_wait(&S->ld_full[0], 0u, abort_flag, p.status, wait_ns);
@@ -324,8 +439,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
                 const uint32_t aP = smem_u32(sP), bV = smem_u32(sV + (j % kRing) * kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < kBlockK / 16; ++kk) {
+                    // keys 16 kk .. 16 kk + 15: P's K-major half kk / 4, V's 8-key groups 2 kk and 2 kk + 1
                     const uint32_t half = (uint32_t)(kk >> 2), off = 32u * (uint32_t)(kk & 3);
-                    mma_bf16(tO, kdesc(aP + half * kTileBytes + off), kdesc(bV + half * (kTileBytes / 2) + off), idO,
+                    mma_bf16(tO, kdesc(aP + half * kTileBytes + off), vdesc(bV + 2048u * (uint32_t)kk), idO,
                              (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(&S->pv_done);
@@ -352,31 +468,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
                 break;
             }
             tc_fence_after();
-            float s[kBlockK];
+            uint32_t sv[kBlockK];
 #pragma unroll
             for (int c = 0; c < kBlockK; c += 16) {
                 uint32_t v[16];
                 tc_ld16(tS + lanebase + (uint32_t)c, v);
-                tc_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) s[c + e] = __uint_as_float(v[e]);
+                for (int e = 0; e < 16; ++e) sv[c + e] = v[e];
             }
+            tc_wait_ld();
             tc_fence_before();
             mbar_arrive(&S->s_free);
             // scores in base 2; keys past lk do not count
             const int kvalid = p.lk - j * kBlockK;
+            float s[kBlockK];
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < kBlockK; ++c) {
-                s[c] = c < kvalid ? s[c] * p.scale_log2 : -INFINITY;
+                s[c] = c < kvalid ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
                 mx = fmaxf(mx, s[c]);
             }
             const float m_new = fmaxf(m, mx);
-            const float alpha = exp2f(m - m_new);     // 0 on the first block (m = -inf)
+            const float alpha = ex2(m - m_new);       // 0 on the first block (m = -inf)
             float sum = 0.0f;
 #pragma unroll
             for (int c = 0; c < kBlockK; ++c) {
-                s[c] = exp2f(s[c] - m_new);
+                s[c] = ex2(s[c] - m_new);
                 sum += s[c];
             }
             l = l * alpha + sum;
@@ -398,13 +515,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
                 *reinterpret_cast<uint4 *>(sP + (c >> 6) * kTileBytes + sw128(row, (c & 63) >> 3)) = w;
             }
             if (j > 0) {
+                uint32_t ov[kHeadDim];
 #pragma unroll
                 for (int c = 0; c < kHeadDim; c += 16) {
                     uint32_t v[16];
                     tc_ld16(tO + lanebase + (uint32_t)c, v);
-                    tc_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                    for (int e = 0; e < 16; ++e) ov[c + e] = v[e];
+                }
+                tc_wait_ld();
+#pragma unroll
+                for (int c = 0; c < kHeadDim; c += 16) {
+                    uint32_t v[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(ov[c + e]) * alpha);
                     tmem_st16(tO + lanebase + (uint32_t)c, v);
                 }
                 tmem_wait_st();
@@ -416,16 +540,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
         if (ok && warp_wait(&S->pv_done, (uint32_t)(nkb - 1) & 1u, abort_flag, p.status, wait_ns)) {
             tc_fence_after();
             const float inv = 1.0f / l;
-            uint32_t o[kHeadDim / 2];
+            uint32_t ov[kHeadDim];
 #pragma unroll
             for (int c = 0; c < kHeadDim; c += 16) {
                 uint32_t v[16];
                 tc_ld16(tO + lanebase + (uint32_t)c, v);
-                tc_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; e += 2)
-                    o[(c + e) >> 1] = bf16x2(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
+                for (int e = 0; e < 16; ++e) ov[c + e] = v[e];
             }
+            tc_wait_ld();
+            uint32_t o[kHeadDim / 2];
+#pragma unroll
+            for (int c = 0; c < kHeadDim; c += 2)
+                o[c >> 1] = bf16x2(__uint_as_float(ov[c]) * inv, __uint_as_float(ov[c + 1]) * inv);
             if (q0 + row < p.lq) {
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)(q0 + row) * p.cols + col0);
 #pragma unroll
@@ -442,8 +569,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
     }
 }
 
-constexpr size_t kAttnSmemBytes = 1024 + (size_t)(1 + 2 * kRing + 2) * kTileBytes + sizeof(AttnSmem);
-static_assert(kAttnSmemBytes <= 227 * 1024, "attention shared memory exceeds 227 KB");
+template <int FORM>
+constexpr size_t attn_smem_bytes()
+{
+    return 1024 + (size_t)(1 + 2 * kRing + 2) * kTileBytes + (FORM == 1 ? (size_t)kSlots * kSlotBytes : 0) +
+           sizeof(AttnSmem);
+}
+static_assert(attn_smem_bytes<1>() <= 227 * 1024, "attention shared memory exceeds 227 KB");
 
 template <int FORM, int K>
 cudaError_t attn_launch_k(const AttnParams &p, cudaStream_t stream)
@@ -457,16 +589,16 @@ cudaError_t attn_launch_k(const AttnParams &p, cudaStream_t stream)
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || !done[dev]) {
             e = cudaFuncSetAttribute(k_attention<FORM, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)kAttnSmemBytes);
+                                     (int)attn_smem_bytes<FORM>());
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) done[dev] = true;
         }
     }
     const dim3 grid((unsigned)((p.lq + kBlockQ - 1) / kBlockQ), (unsigned)(p.cols / kHeadDim));
     const char *name = FORM == 0 ? "k_attention<bf16>" : "k_attention<dequantise>";
-    log_launch(name, grid, dim3(kAttnThreads), kAttnSmemBytes);
+    log_launch(name, grid, dim3(kAttnThreads), attn_smem_bytes<FORM>());
     trace_begin(name, stream);
-    k_attention<FORM, K><<<grid, kAttnThreads, kAttnSmemBytes, stream>>>(p);
+    k_attention<FORM, K><<<grid, kAttnThreads, attn_smem_bytes<FORM>(), stream>>>(p);
     trace_end(stream);
     return cudaGetLastError();
 }
@@ -489,9 +621,25 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream)
     p.lk = (int)a.lk;
     p.cols = (int)a.cols;
     p.group = a.group;
+    p.group_lg = 0;
+    while (p.group > 0 && (1 << (p.group_lg + 1)) <= p.group) ++p.group_lg;
     p.scale_log2 = 1.4426950408889634f / 8.0f;   // log2(e) / sqrt(64)
     p.status = a.status;
     p.wait_ns = kAttnWaitNs;
+    // Q (both forms) and bf16 K, V by TMA: [rows x cols] bf16, a 64-channel x 128-row box
+    if (!make_map_bf16(&p.tq, a.q, (uint64_t)a.cols, (uint64_t)a.lq, (uint64_t)a.cols, kHeadDim, kBlockQ))
+        return cudaErrorInvalidValue;
+    if (!a.dequantise &&
+        (!make_map_bf16(&p.tk, a.kv[0], (uint64_t)a.cols, (uint64_t)a.lk, (uint64_t)a.cols, kHeadDim, kBlockK) ||
+         !make_map_bf16(&p.tv, a.kv[1], (uint64_t)a.cols, (uint64_t)a.lk, (uint64_t)a.cols, kHeadDim, kBlockK)))
+        return cudaErrorInvalidValue;
+    // the caches (dequantise form): fp32 [lk x cols], a 64-channel x 32-key box, no swizzle
+    if (a.dequantise &&
+        (!make_map(&p.tc[0], a.cache_in[0], (uint64_t)a.cols, (uint64_t)a.lk, (uint64_t)a.cols, kHeadDim, kSub,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+         !make_map(&p.tc[1], a.cache_in[1], (uint64_t)a.cols, (uint64_t)a.lk, (uint64_t)a.cols, kHeadDim, kSub,
+                   CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return cudaErrorInvalidValue;
     if (!a.dequantise) return attn_launch_k<0, 2>(p, stream);
     switch (a.bits) {
     case 1: return attn_launch_k<1, 1>(p, stream);

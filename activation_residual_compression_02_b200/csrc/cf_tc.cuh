@@ -138,6 +138,22 @@ static inline bool make_map(CUtensorMap *map, const void *ptr, uint64_t inner, u
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor map: dims {inner, outer}, row pitch in elements, box {bx, by},
+// 128-byte swizzle (bx * 2 <= 128).
+static inline bool make_map_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer,
+                                 uint64_t pitch_elems, uint32_t bx, uint32_t by)
+{
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch_elems * 2};
+    cuuint32_t box[2] = {bx, by};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D fp32 tensor map over `count` equally spaced [outer x inner] blocks
 // (pitch in elements, block stride in elements), box {bx, by, 1}.
 static inline bool make_map3(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t count, uint64_t pitch_elems,

@@ -57,6 +57,15 @@ def alg_bytes_per_elem(bits, group):
     return 2 + 2 + 4 + 2 + 4 + payload, payload + 4 + 4
 
 
+def bf16_peak():
+    """Dense bf16 tensor peak (TFLOP/s): the measured burst figure, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def source_hash(src="cf_quant.cu"):
     p = os.path.join(ROOT, "activation_residual_compression_02_b200", "csrc", src)
     with open(p, "rb") as f:
@@ -1020,6 +1029,126 @@ def run_exchange_bench(args, w):
     return 0
 
 
+def run_attention_bench(args, w):
+    """The consumer of the compressed K/V exchange (Algorithms 1 and 2): one
+    step of attention over a received shard for every layer of the workload
+    (the layer's K and V slots, 4444 tokens x 1920 channels = 30 heads of 64
+    for the CogVideoX-shaped shard), three ways:
+      recon       cf_decompress of every K/V slot writing bf16(C) in the same
+                  pass, then cf_attention on those bf16 tensors;
+      cast        cf_decompress, a separate torch cast of each cache to bf16,
+                  then cf_attention;
+      dequantise  cf_attention reading the caches and the step's payload,
+                  dequantising on load and writing the new caches (no
+                  decompress launch).
+    Reports ms per step of each and the attention's TFLOP/s."""
+    world, rank, local = dist_init()
+    import activation_residual_compression_02_b200 as cf
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    clk = ClockSampler(torch.cuda.current_device()).start()
+    layers = w.slots
+    shapes = [(w.rows, w.cols)] * (2 * layers)        # K and V of every layer
+    ctx = cf.Context(shapes, bits=w.bits, group=w.group)
+    st = cf.QuantState(shapes, w.bits, w.group, device=dev, recon=True)
+    streams = [synth.SlotStream(w, s_, seed=rank, device=dev) for s_ in range(2 * layers)]
+    x0 = [s_.next().reshape(-1) for s_ in streams]
+    sl = st.slots(x0)
+    ctx.compress(sl, 0)
+    ctx.decompress(sl, 0)
+    del x0
+    x1 = [s_.next().reshape(-1) for s_ in streams]
+    del streams
+    sl = st.slots(x1)
+    ctx.compress(sl, 1)                                 # the step's payload
+    before = st.cache_all.clone()                       # the receiver's caches before the step
+    c_before = [before[c.storage_offset() - st.cache_all.storage_offset():][:c.numel()] for c in st.cache]
+    new_all = torch.empty_like(st.cache_all)
+    c_new = [new_all[c.storage_offset() - st.cache_all.storage_offset():][:c.numel()] for c in st.cache]
+    cast_all = torch.empty(st.cache_all.numel(), dtype=torch.bfloat16, device=dev)
+    c_cast = [cast_all[c.storage_offset() - st.cache_all.storage_offset():][:c.numel()] for c in st.cache]
+    gq = torch.Generator(device=dev)
+    gq.manual_seed(synth.mix_seed(rank, 99))
+    q = [torch.randn(w.rows, w.cols, generator=gq, device=dev).to(torch.bfloat16) for _ in range(layers)]
+    out = [torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
+    rc_slots = ctx._slots(sl)
+    plain = st.slots(x1)
+    for sl_ in plain:
+        sl_.recon = None
+    plain_slots = ctx._slots(plain)
+    L, h = cf.lib(), ctx.handle
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def decompress(arr):
+        if L.cf_decompress(h, arr, 1, sh) != 0:
+            raise RuntimeError(L.cf_last_error(h).decode())
+
+    def attn_bf16(kv_k, kv_v):
+        for l_ in range(layers):
+            ctx.attention(q[l_], cf.KV(bf16=kv_k[l_]), cf.KV(bf16=kv_v[l_]), out[l_], stream=stream)
+
+    def path_recon():
+        decompress(rc_slots)
+        attn_bf16(st.recon[0::2], st.recon[1::2])
+
+    def path_cast():
+        decompress(plain_slots)
+        cast_all.copy_(st.cache_all)
+        attn_bf16(c_cast[0::2], c_cast[1::2])
+
+    def path_dequantise():
+        for l_ in range(layers):
+            kv = [cf.KV(cache_in=c_before[2 * l_ + i], cache_out=c_new[2 * l_ + i], codes=st.codes[2 * l_ + i],
+                        scales=st.scales[2 * l_ + i]) for i in range(2)]
+            ctx.attention(q[l_], kv[0], kv[1], out[l_], stream=stream)
+
+    def attention_only():
+        attn_bf16(st.recon[0::2], st.recon[1::2])
+
+    def time_it(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with Timed(clk):
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+    ms = {name: time_it(fn) for name, fn in (("attention_only", attention_only), ("recon", path_recon),
+                                             ("cast", path_cast), ("dequantise", path_dequantise))}
+    if ctx.check() != 0:
+        raise RuntimeError("device status in the attention run")
+    clk.stop()
+    flops = 4.0 * w.rows * w.rows * w.cols * layers     # Q K^T and P V: 2 * 2 * lq * lk * 64 per head
+    peak = bf16_peak()
+    line = {
+        "metric": "ring-attention step over a received K/V shard (every layer): ms per step", "value": ms["recon"],
+        "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms["recon"],
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {layers} layers, K and V slots of {w.rows} tokens x {w.cols} channels "
+                               f"({w.cols // 64} heads of 64), k={w.bits}, G={w.group}; queries {w.rows} x {w.cols}",
+                   "l2": "inputs larger than L2 (every layer's caches, payloads and queries)"},
+        "paths_ms": ms,
+        "attention": {"tflops": flops / (ms["attention_only"] * 1e-3) / 1e12,
+                      "frac_of_bf16_peak": flops / (ms["attention_only"] * 1e-3) / 1e12 / peak[0],
+                      "peak_tflops": peak[0], "peak_kind": peak[1], "flops_per_step": flops},
+        "dequantise_vs_recon": ms["dequantise"] / ms["recon"],
+        "note": "recon: cf_decompress writing bf16(C) in its pass + cf_attention on bf16; cast: cf_decompress + "
+                "torch cast of each cache + cf_attention; dequantise: cf_attention reading C_{t-1}, codes and scales "
+                "and writing C_t (no decompress launch)",
+        "gpu_launches": args.steps * (1 + layers), "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1042,6 +1171,8 @@ def main():
                     help="low-rank products: 0 automatic, 1 TF32, 2 split (3xTF32)")
     ap.add_argument("--through-slots", action="store_true",
                     help="low-rank: also time cf_compress / cf_decompress in low-rank mode on bf16 slots")
+    ap.add_argument("--attention", action="store_true",
+                    help="time attention over the received K/V of every layer: recon, cast and dequantise-on-load")
     ap.add_argument("--exchange", action="store_true",
                     help="time the compressed K/V all-gather of patch parallelism instead of the codec alone")
     ap.add_argument("--buckets", type=int, default=None,
@@ -1058,6 +1189,8 @@ def main():
         return run_lowrank_bench(args, w)
     if args.exchange:
         return run_exchange_bench(args, w)
+    if args.attention:
+        return run_attention_bench(args, w if args.workload != "flux" else synth.COGVIDEOX)
     return run_cf(args, w)
 
 
