@@ -22,23 +22,27 @@
 //     the first query block write C_t to cache_out, so no separate decompress
 //     runs.  The two forms give bit-identical outputs.
 //
-// One CTA per (128-query block, head), 8 warps (two per SM sub-partition, so
-// that a thread may hold up to 255 registers):
-//   warps 0-3  softmax: thread t owns query row t (TMEM lane t); online
-//              softmax in base 2 over 128-key blocks, P written to shared
-//              memory in bf16, O rescaled in TMEM;
-//   warp 4     allocates TMEM (S: 128 columns, O: 64) and issues
-//              tcgen05.mma.kind::f16 (bf16 operands, fp32 accumulators):
-//              S = Q K^T, then O += P V;
-//   warps 5-7  load Q once (TMA), then K and V blocks into a two-deep ring:
-//              in the bf16 form by TMA (a [128 x 64] box with the 128-byte
-//              swizzle lands in the layout the MMA reads); in the other, the
-//              fp32 cache rows of 32-key sub-chunks by TMA and their codes and
-//              scales by cp.async into a ring of staging slots, three
-//              sub-chunks ahead of the one being dequantised and stored
-//              swizzled.  Q and K are K-major operands;
-//              V is read MN-major (the channels of a key are contiguous), so
-//              no operand is transposed.
+// One CTA per (256-query block, head): two 128-query tiles, t = 0 and 1, whose
+// softmax work alternates with the other tile's products on the tensor cores.
+//   warps 0-3, 4-7  softmax of tile 0, tile 1: thread r of a tile owns query
+//              row r (TMEM lane r); online softmax in base 2 over 128-key
+//              blocks, P written to tensor memory in bf16; O rescaled in
+//              TMEM only when a row's running maximum grows by more than 2^8
+//              (otherwise the stale maximum is kept: the normalisation at the
+//              end divides by a sum taken against the same maximum);
+//   warp 8     allocates TMEM (S_t: 128 columns each, O_t: 64, P_t: 64) and
+//              issues tcgen05.mma.kind::f16 (bf16 operands, fp32
+//              accumulators): S_t = Q_t K^T from shared memory, then
+//              O_t += P_t V with P_t read from tensor memory;
+//   warps 9..  load Q once (TMA), then K and V blocks into a ring shared by
+//              both tiles: in the bf16 form by TMA (a [128 x 64] box with the
+//              128-byte swizzle lands in the layout the MMA reads); in the
+//              other, the fp32 cache rows of 32-key sub-chunks by TMA and
+//              their codes and scales by cp.async into a ring of staging
+//              slots, three sub-chunks ahead of the one being dequantised
+//              and stored swizzled.  Q and K are K-major operands; V is read
+//              MN-major (the channels of a key are contiguous), so no operand
+//              is transposed.
 // Every mbarrier wait is bounded; on expiry the CTA raises an abort flag and
 // the status word's timeout bit, drains its MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -56,13 +60,18 @@ using namespace ptx;
 using namespace tc;
 
 constexpr int kHeadDim = 64;
-constexpr int kBlockQ = 128;           // queries per CTA (MMA M)
+constexpr int kBlockQ = 128;           // queries per tile (MMA M)
+constexpr int kTiles = 2;              // query tiles per CTA
 constexpr int kBlockK = 128;           // keys per block (S's N, PV's K)
-constexpr int kAttnThreads = 256;      // 8 warps
-constexpr int kLoaders = 96;           // warps 5-7
-constexpr int kRing = 2;               // K/V blocks in flight
+constexpr int kMmaWarp = 8;
+constexpr int kLoader0 = 288;          // first loader thread (warp 9)
 constexpr int kTileBytes = 128 * kHeadDim * 2;   // a 128 x 64 bf16 tile: 16 KB
+constexpr int kMaxRing = 3;
 constexpr uint64_t kAttnWaitNs = 2000000000ull;
+// Tensor memory columns: S_t at 128 t, O_t at 256 + 64 t, P_t at 384 + 64 t.
+constexpr uint32_t kTmemCols = 512;
+// Rescale O only when the running maximum grows by more than 2^8 (base 2).
+constexpr float kRescaleLog2 = 8.0f;
 // Dequantise-on-load staging: sub-chunks of 32 keys (K and V: fp32 cache,
 // codes, scales) stream through a ring of kSlots shared-memory slots.
 constexpr int kSub = 32;
@@ -72,16 +81,24 @@ constexpr int kSlotCodes = 2 * kSub * 32;           // up to 32 code bytes per k
 constexpr int kSlotScales = 2 * kSub * 8 * 4;       // up to 8 scales per key row (G = 8)
 constexpr int kSlotBytes = kSlotC + kSlotCodes + kSlotScales;
 
+// Per form: loader warps, threads and K/V ring depth.
+template <int FORM>
+struct AttnCfg {
+    static constexpr int kLoaders = FORM == 0 ? 32 : 96;
+    static constexpr int kThreads = kLoader0 + kLoaders;
+    static constexpr int kRing = FORM == 0 ? 3 : 2;
+};
+
 struct AttnSmem {
     uint64_t st_full[kSlots];     // staging slot landed (TMA bytes + every loader's cp.async)
     uint64_t st_free[kSlots];     // staging slot read by the three loader warps
     uint64_t q_full;
-    uint64_t ld_full[kRing];
-    uint64_t ld_free[kRing];
-    uint64_t s_full;
-    uint64_t s_free;
-    uint64_t p_full;
-    uint64_t pv_done;
+    uint64_t ld_full[kMaxRing];   // K and V of a block in the ring
+    uint64_t ld_free[kMaxRing];   // both tiles' products with that block done
+    uint64_t s_full[kTiles];      // S_t computed
+    uint64_t s_free[kTiles];      // S_t read by the tile's four softmax warps
+    uint64_t p_full[kTiles];      // P_t (and any O_t rescale) in tensor memory
+    uint64_t pv_done[kTiles];     // O_t += P_t V complete
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -144,6 +161,19 @@ __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t adesc, uint64_t bd
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// The same with the A operand in tensor memory: lane i holds row i of A, and
+// each 32-bit column two consecutive K elements (the lower one in the low
+// half), so one K = 16 step reads 8 columns.
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
 
@@ -226,20 +256,21 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v)
 __device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <int FORM, int K>
-__global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_constant__ AttnParams p)
+__global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const __grid_constant__ AttnParams p)
 {
+    constexpr int kRing = AttnCfg<FORM>::kRing;
+    constexpr int kLoaders = AttnCfg<FORM>::kLoaders;
     extern __shared__ __align__(1024) uint8_t attn_smem[];
     uint8_t *base = (uint8_t *)(((uintptr_t)attn_smem + 1023) & ~(uintptr_t)1023);
-    uint8_t *sQ = base;                                    // [128 queries x 64] K-major
-    uint8_t *sK = sQ + kTileBytes;                         // kRing x [128 keys x 64] K-major
+    uint8_t *sQ = base;                                    // kTiles x [128 queries x 64] K-major
+    uint8_t *sK = sQ + kTiles * kTileBytes;                // kRing x [128 keys x 64] K-major
     uint8_t *sV = sK + kRing * kTileBytes;                 // kRing x [128 keys x 64] (read MN-major)
-    uint8_t *sP = sV + kRing * kTileBytes;                 // 2 x [128 queries x 64 keys] K-major
-    uint8_t *sStage = sP + 2 * kTileBytes;                 // dequantise-on-load: kSlots staging slots
+    uint8_t *sStage = sV + kRing * kTileBytes;             // dequantise-on-load: kSlots staging slots
     AttnSmem *S = reinterpret_cast<AttnSmem *>(sStage + (FORM == 1 ? kSlots * kSlotBytes : 0));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb = blockIdx.x, head = blockIdx.y;
-    const int q0 = qb * kBlockQ;
+    const int q0 = qb * (kTiles * kBlockQ);
     const int nkb = (p.lk + kBlockK - 1) / kBlockK;
     const int col0 = head * kHeadDim;
     constexpr uint32_t kLdArrivals = FORM == 0 ? 1u : (uint32_t)kLoaders;
@@ -254,10 +285,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
             mbar_init(&S->ld_full[b], kLdArrivals);
             mbar_init(&S->ld_free[b], 1);
         }
-        mbar_init(&S->s_full, 1);
-        mbar_init(&S->s_free, 128);
-        mbar_init(&S->p_full, 128);
-        mbar_init(&S->pv_done, 1);
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(&S->s_full[t], 1);
+            mbar_init(&S->s_free[t], 4);               // one arrival per softmax warp of the tile
+            mbar_init(&S->p_full[t], 4);
+            mbar_init(&S->pv_done[t], 1);
+        }
         mbar_init(&S->drain, 1);
         S->abort_flag = 0;
         mbar_init_fence();
@@ -266,9 +299,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
         const int L = (1 << (K - 1)) - 1;
         S->lut[threadIdx.x] = (K >= 2) ? __fdiv_rn((float)((int)threadIdx.x - L), (float)L) : 0.0f;
     }
-    if (warp == 4) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S->tmem_base)),
-                     "r"(256)
+                     "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -276,17 +309,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    const uint32_t tS = tmem, tO = tmem + 128;   // S: columns 0..127, O: 128..191
     volatile int *abort_flag = &S->abort_flag;
     const unsigned long long wait_ns = p.wait_ns;
 
-    if (warp >= 5) {
+    if (threadIdx.x >= kLoader0) {
         // ------------------------------------------------------- loaders --
-        const int lt = threadIdx.x - 160;   // 0..kLoaders-1
+        const int lt = threadIdx.x - kLoader0;   // 0..kLoaders-1
         if (lt == 0) {
-            // Q by TMA; rows past lq read as zero
-            mbar_expect_tx(&S->q_full, (uint32_t)kTileBytes);
-            tma_load_2d(sQ, &p.tq, col0, q0, &S->q_full);
+            // Q of both tiles by TMA; rows past lq read as zero
+            mbar_expect_tx(&S->q_full, (uint32_t)(kTiles * kTileBytes));
+            for (int t = 0; t < kTiles; ++t) tma_load_2d(sQ + t * kTileBytes, &p.tq, col0, q0 + t * kBlockQ, &S->q_full);
         }
         if constexpr (FORM == 0) {
             // K and V boxes by TMA (keys past lk read as zero), one thread
@@ -342,10 +374,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
                 }
                 cp_async_arrive(&S->st_full[slot]);
             };
-            bool ok = true;
             for (int g = 0; g < kSlots - 1 && g < ngs; ++g) issue(g);
             const uint32_t lut = smem_u32(S->lut);
-            for (int g = 0; g < ngs && ok; ++g) {
+            for (int g = 0; g < ngs; ++g) {
                 const int j = g / (kBlockK / kSub), sub = g % (kBlockK / kSub), b = j % kRing;
                 const int slot = g & (kSlots - 1);
                 // stage sub-chunk g + 3 into the slot of sub-chunk g - 1 once every loader warp has read it
@@ -400,52 +431,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
             }
             cp_wait_all();
         }
-    } else if (warp == 4) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- MMA issuer --
+        // Per key block j: S_0(j + 1) as soon as tile 0's softmax has read
+        // S_0(j), O_0 += P_0(j) V(j) once P_0(j) is in tensor memory, then the
+        // same for tile 1; so the tensor cores work on one tile while the
+        // other tile's softmax runs.
         const uint32_t idS = instr_desc_bf16(kBlockK, 0), idO = instr_desc_bf16(kHeadDim, 1);
-        const uint32_t aQ = smem_u32(sQ);
+        auto issue_s = [&](int t, int b) {       // S_t = Q_t K_b^T (lane 0)
+            const uint32_t aQ = smem_u32(sQ + t * kTileBytes), bK = smem_u32(sK + b * kTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < kHeadDim / 16; ++kk)
+                mma_bf16(tmem + 128u * (uint32_t)t, kdesc(aQ + 32 * kk), kdesc(bK + 32 * kk), idS, kk > 0);
+            tc_commit(&S->s_full[t]);
+        };
+        auto issue_pv = [&](int t, int b, bool first) {   // O_t += P_t V_b (lane 0)
+            const uint32_t bV = smem_u32(sV + b * kTileBytes);
+            const uint32_t tO = tmem + 256u + 64u * (uint32_t)t, tP = tmem + 384u + 64u * (uint32_t)t;
+#pragma unroll
+            for (int kk = 0; kk < kBlockK / 16; ++kk)
+                // keys 16 kk .. 16 kk + 15: P's columns 8 kk .., V's 8-key groups 2 kk and 2 kk + 1
+                mma_bf16_ta(tO, tP + 8u * (uint32_t)kk, vdesc(bV + 2048u * (uint32_t)kk), idO,
+                            (!first || kk > 0) ? 1u : 0u);
+            tc_commit(&S->pv_done[t]);
+        };
         bool ok = warp_wait(&S->q_full, 0u, abort_flag, p.status, wait_ns) &&
                   warp_wait(&S->ld_full[0], 0u, abort_flag, p.status, wait_ns);
         if (ok) {
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t bK = smem_u32(sK);
-#pragma unroll
-                for (int kk = 0; kk < kHeadDim / 16; ++kk) mma_bf16(tS, kdesc(aQ + 32 * kk), kdesc(bK + 32 * kk), idS, kk > 0);
-                tc_commit(&S->s_full);
+                issue_s(0, 0);
+                issue_s(1, 0);
             }
             __syncwarp();
         }
         for (int j = 0; j < nkb && ok; ++j) {
+            const int b = j % kRing, b1 = (j + 1) % kRing;
+            const uint32_t par = (uint32_t)j & 1u;
             if (j + 1 < nkb) {
-                const int b1 = (j + 1) % kRing;
                 ok = warp_wait(&S->ld_full[b1], (uint32_t)((j + 1) / kRing) & 1u, abort_flag, p.status, wait_ns) &&
-                     warp_wait(&S->s_free, (uint32_t)j & 1u, abort_flag, p.status, wait_ns);
+                     warp_wait(&S->s_free[0], par, abort_flag, p.status, wait_ns);
                 if (!ok) break;
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t bK = smem_u32(sK + b1 * kTileBytes);
-#pragma unroll
-                    for (int kk = 0; kk < kHeadDim / 16; ++kk)
-                        mma_bf16(tS, kdesc(aQ + 32 * kk), kdesc(bK + 32 * kk), idS, kk > 0);
-                    tc_commit(&S->s_full);
-                }
+                if (lane == 0) issue_s(0, b1);
                 __syncwarp();
             }
-            ok = warp_wait(&S->p_full, (uint32_t)j & 1u, abort_flag, p.status, wait_ns);
+            ok = warp_wait(&S->p_full[0], par, abort_flag, p.status, wait_ns);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) issue_pv(0, b, j == 0);
+            __syncwarp();
+            if (j + 1 < nkb) {
+                ok = warp_wait(&S->s_free[1], par, abort_flag, p.status, wait_ns);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) issue_s(1, b1);
+                __syncwarp();
+            }
+            ok = warp_wait(&S->p_full[1], par, abort_flag, p.status, wait_ns);
             if (!ok) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t aP = smem_u32(sP), bV = smem_u32(sV + (j % kRing) * kTileBytes);
-#pragma unroll
-                for (int kk = 0; kk < kBlockK / 16; ++kk) {
-                    // keys 16 kk .. 16 kk + 15: P's K-major half kk / 4, V's 8-key groups 2 kk and 2 kk + 1
-                    const uint32_t half = (uint32_t)(kk >> 2), off = 32u * (uint32_t)(kk & 3);
-                    mma_bf16(tO, kdesc(aP + half * kTileBytes + off), vdesc(bV + 2048u * (uint32_t)kk), idO,
-                             (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc_commit(&S->pv_done);
-                tc_commit(&S->ld_free[j % kRing]);
+                issue_pv(1, b, j == 0);
+                tc_commit(&S->ld_free[b]);
             }
             __syncwarp();
         }
@@ -456,95 +504,110 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
             wait_bounded(&S->drain, 0u, &no_abort, p.status, kAttnWaitNs);
         }
         __syncwarp();
-    } else {
+    } else if (warp < kMmaWarp) {
         // ------------------------------------------------------- softmax --
-        const int row = threadIdx.x;                        // query row of this thread = TMEM lane
-        const uint32_t lanebase = (uint32_t)(32 * warp) << 16;
-        float m = -INFINITY, l = 0.0f;
+        const int t = warp >> 2;                            // query tile
+        const int row = 32 * (warp & 3) + lane;             // query row of the tile = TMEM lane
+        const uint32_t lanebase = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t tS = tmem + 128u * (uint32_t)t + lanebase;
+        const uint32_t tO = tmem + 256u + 64u * (uint32_t)t + lanebase;
+        const uint32_t tP = tmem + 384u + 64u * (uint32_t)t + lanebase;
+        const float c2 = p.scale_log2;
+        float m = -INFINITY, l = 0.0f;                      // reference maximum (raw score) and sum against it
         bool ok = true;
         for (int j = 0; j < nkb; ++j) {
-            if (!warp_wait(&S->s_full, (uint32_t)j & 1u, abort_flag, p.status, wait_ns)) {
+            if (!warp_wait(&S->s_full[t], (uint32_t)j & 1u, abort_flag, p.status, wait_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t sv[kBlockK];
+            float s[kBlockK];
 #pragma unroll
             for (int c = 0; c < kBlockK; c += 16) {
                 uint32_t v[16];
-                tc_ld16(tS + lanebase + (uint32_t)c, v);
+                tc_ld16(tS + (uint32_t)c, v);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sv[c + e] = v[e];
+                for (int e = 0; e < 16; ++e) s[c + e] = __uint_as_float(v[e]);
             }
             tc_wait_ld();
             tc_fence_before();
-            mbar_arrive(&S->s_free);
-            // scores in base 2; keys past lk do not count
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->s_free[t]);
+            // keys past lk do not count (the last block only; uniform across the CTA)
             const int kvalid = p.lk - j * kBlockK;
-            float s[kBlockK];
-            float mx = -INFINITY;
+            if (kvalid < kBlockK) {
 #pragma unroll
-            for (int c = 0; c < kBlockK; ++c) {
-                s[c] = c < kvalid ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[c]);
+                for (int c = 0; c < kBlockK; ++c) s[c] = c < kvalid ? s[c] : -INFINITY;
             }
-            const float m_new = fmaxf(m, mx);
-            const float alpha = ex2(m - m_new);       // 0 on the first block (m = -inf)
-            float sum = 0.0f;
+            float mx[8];
 #pragma unroll
-            for (int c = 0; c < kBlockK; ++c) {
-                s[c] = ex2(s[c] - m_new);
-                sum += s[c];
+            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < kBlockK; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+            const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            // move the reference maximum only when it grows by more than 2^8 in base 2
+            const bool grow = (m_blk - m) * c2 > kRescaleLog2;   // true on the first block (m = -inf)
+            const bool rescale = __any_sync(0xffffffffu, grow) && j > 0;
+            float alpha = 1.0f;
+            if (grow) {
+                alpha = ex2((m - m_blk) * c2);                    // 0 on the first block
+                m = m_blk;
             }
-            l = l * alpha + sum;
-            m = m_new;
-            uint32_t pw[kBlockK / 2];   // P in bf16 pairs: half the registers across the wait below
-#pragma unroll
-            for (int c = 0; c < kBlockK; c += 2) pw[c >> 1] = bf16x2(s[c], s[c + 1]);
+            const float mc = m * c2;
             if (j > 0) {
-                // P and O are free once the previous block's P V has completed
-                if (!warp_wait(&S->pv_done, (uint32_t)(j - 1) & 1u, abort_flag, p.status, wait_ns)) {
+                // P_t and O_t are free once the previous block's P V has completed
+                if (!warp_wait(&S->pv_done[t], (uint32_t)(j - 1) & 1u, abort_flag, p.status, wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
             }
+            // P = 2^(s c2 - m c2) in 32-key chunks, each packed to bf16 pairs and
+            // stored to tensor memory as soon as it is formed
+            float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kBlockK; c += 8) {
-                const uint4 w = make_uint4(pw[c >> 1], pw[(c >> 1) + 1], pw[(c >> 1) + 2], pw[(c >> 1) + 3]);
-                *reinterpret_cast<uint4 *>(sP + (c >> 6) * kTileBytes + sw128(row, (c & 63) >> 3)) = w;
-            }
-            if (j > 0) {
-                uint32_t ov[kHeadDim];
+            for (int q = 0; q < kBlockK; q += 32) {
+                uint32_t v[16];
 #pragma unroll
-                for (int c = 0; c < kHeadDim; c += 16) {
-                    uint32_t v[16];
-                    tc_ld16(tO + lanebase + (uint32_t)c, v);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) ov[c + e] = v[e];
+                for (int e = 0; e < 16; ++e) {
+                    const float x0 = ex2(fmaf(s[q + 2 * e], c2, -mc)), x1 = ex2(fmaf(s[q + 2 * e + 1], c2, -mc));
+                    sm[(2 * e) & 7] += x0;
+                    sm[(2 * e + 1) & 7] += x1;
+                    v[e] = bf16x2(x0, x1);
                 }
-                tc_wait_ld();
-#pragma unroll
-                for (int c = 0; c < kHeadDim; c += 16) {
-                    uint32_t v[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(ov[c + e]) * alpha);
-                    tmem_st16(tO + lanebase + (uint32_t)c, v);
-                }
-                tmem_wait_st();
+                tmem_st16(tP + (uint32_t)(q >> 1), v);
             }
-            fence_proxy_async();
+            l = l * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+            if (rescale) {
+#pragma unroll
+                for (int c = 0; c < kHeadDim; c += 32) {
+                    uint32_t v0[16], v1[16];
+                    tc_ld16(tO + (uint32_t)c, v0);
+                    tc_ld16(tO + (uint32_t)c + 16u, v1);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
+                        v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
+                    }
+                    tmem_st16(tO + (uint32_t)c, v0);
+                    tmem_st16(tO + (uint32_t)c + 16u, v1);
+                }
+            }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&S->p_full);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S->p_full[t]);
         }
-        if (ok && warp_wait(&S->pv_done, (uint32_t)(nkb - 1) & 1u, abort_flag, p.status, wait_ns)) {
+        if (ok && warp_wait(&S->pv_done[t], (uint32_t)(nkb - 1) & 1u, abort_flag, p.status, wait_ns)) {
             tc_fence_after();
             const float inv = 1.0f / l;
             uint32_t ov[kHeadDim];
 #pragma unroll
             for (int c = 0; c < kHeadDim; c += 16) {
                 uint32_t v[16];
-                tc_ld16(tO + lanebase + (uint32_t)c, v);
+                tc_ld16(tO + (uint32_t)c, v);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) ov[c + e] = v[e];
             }
@@ -553,8 +616,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
 #pragma unroll
             for (int c = 0; c < kHeadDim; c += 2)
                 o[c >> 1] = bf16x2(__uint_as_float(ov[c]) * inv, __uint_as_float(ov[c + 1]) * inv);
-            if (q0 + row < p.lq) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)(q0 + row) * p.cols + col0);
+            const int qrow = q0 + t * kBlockQ + row;
+            if (qrow < p.lq) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)qrow * p.cols + col0);
 #pragma unroll
                 for (int c = 0; c < kHeadDim / 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
             }
@@ -564,18 +628,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attention(const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256) : "memory");
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
 template <int FORM>
 constexpr size_t attn_smem_bytes()
 {
-    return 1024 + (size_t)(1 + 2 * kRing + 2) * kTileBytes + (FORM == 1 ? (size_t)kSlots * kSlotBytes : 0) +
-           sizeof(AttnSmem);
+    return 1024 + (size_t)(kTiles + 2 * AttnCfg<FORM>::kRing) * kTileBytes +
+           (FORM == 1 ? (size_t)kSlots * kSlotBytes : 0) + sizeof(AttnSmem);
 }
+static_assert(attn_smem_bytes<0>() <= 227 * 1024, "attention shared memory exceeds 227 KB");
 static_assert(attn_smem_bytes<1>() <= 227 * 1024, "attention shared memory exceeds 227 KB");
+// One CTA per SM: the 512 tensor-memory columns it allocates are the SM's all.
+static_assert(attn_smem_bytes<0>() > 114 * 1024 && attn_smem_bytes<1>() > 114 * 1024,
+              "a second resident CTA would wait for tensor memory");
 
 template <int FORM, int K>
 cudaError_t attn_launch_k(const AttnParams &p, cudaStream_t stream)
@@ -594,11 +662,12 @@ cudaError_t attn_launch_k(const AttnParams &p, cudaStream_t stream)
             if (dev >= 0 && dev < 64) done[dev] = true;
         }
     }
-    const dim3 grid((unsigned)((p.lq + kBlockQ - 1) / kBlockQ), (unsigned)(p.cols / kHeadDim));
+    constexpr int kQ = kTiles * kBlockQ;
+    const dim3 grid((unsigned)((p.lq + kQ - 1) / kQ), (unsigned)(p.cols / kHeadDim));
     const char *name = FORM == 0 ? "k_attention<bf16>" : "k_attention<dequantise>";
-    log_launch(name, grid, dim3(kAttnThreads), attn_smem_bytes<FORM>());
+    log_launch(name, grid, dim3(AttnCfg<FORM>::kThreads), attn_smem_bytes<FORM>());
     trace_begin(name, stream);
-    k_attention<FORM, K><<<grid, kAttnThreads, attn_smem_bytes<FORM>(), stream>>>(p);
+    k_attention<FORM, K><<<grid, AttnCfg<FORM>::kThreads, attn_smem_bytes<FORM>(), stream>>>(p);
     trace_end(stream);
     return cudaGetLastError();
 }
