@@ -30,11 +30,15 @@
 //              TMEM only when a row's running maximum grows by more than 2^8
 //              (otherwise the stale maximum is kept: the normalisation at the
 //              end divides by a sum taken against the same maximum);
-//   warp 8     allocates TMEM (S_t: 128 columns each, O_t: 64, P_t: 64) and
+//   warp 8(-9) allocates TMEM (S_t: 128 columns each, O_t: 64, P_t: 64) and
 //              issues tcgen05.mma.kind::f16 (bf16 operands, fp32
 //              accumulators): S_t = Q_t K^T from shared memory, then
-//              O_t += P_t V with P_t read from tensor memory;
-//   warps 9..  load Q once (TMA), then K and V blocks into a ring shared by
+//              O_t += P_t V with P_t read from tensor memory.  In the bf16
+//              form warps 8 and 9 each issue one tile's products (a single
+//              issuing thread, at a few hundred cycles per group of MMAs and
+//              commit, would bound the kernel); in the other, warp 8 issues
+//              both;
+//   the rest   load Q once (TMA), then K and V blocks into a ring shared by
 //              both tiles: in the bf16 form by TMA (a [128 x 64] box with the
 //              128-byte swizzle lands in the layout the MMA reads); in the
 //              other, the fp32 cache rows of 32-key sub-chunks by TMA and
@@ -64,7 +68,6 @@ constexpr int kBlockQ = 128;           // queries per tile (MMA M)
 constexpr int kTiles = 2;              // query tiles per CTA
 constexpr int kBlockK = 128;           // keys per block (S's N, PV's K)
 constexpr int kMmaWarp = 8;
-constexpr int kLoader0 = 288;          // first loader thread (warp 9)
 constexpr int kTileBytes = 128 * kHeadDim * 2;   // a 128 x 64 bf16 tile: 16 KB
 constexpr int kMaxRing = 3;
 constexpr uint64_t kAttnWaitNs = 2000000000ull;
@@ -81,9 +84,12 @@ constexpr int kSlotCodes = 2 * kSub * 32;           // up to 32 code bytes per k
 constexpr int kSlotScales = 2 * kSub * 8 * 4;       // up to 8 scales per key row (G = 8)
 constexpr int kSlotBytes = kSlotC + kSlotCodes + kSlotScales;
 
-// Per form: loader warps, threads and K/V ring depth.
+// Per form: MMA issuer warps (one per tile in the bf16 form, whose issue
+// rate would otherwise bound it), loader warps, threads and K/V ring depth.
 template <int FORM>
 struct AttnCfg {
+    static constexpr int kIssuers = FORM == 0 ? 2 : 1;
+    static constexpr int kLoader0 = 32 * (kMmaWarp + kIssuers);   // first loader thread
     static constexpr int kLoaders = FORM == 0 ? 32 : 96;
     static constexpr int kThreads = kLoader0 + kLoaders;
     static constexpr int kRing = FORM == 0 ? 3 : 2;
@@ -99,7 +105,7 @@ struct AttnSmem {
     uint64_t s_free[kTiles];      // S_t read by the tile's four softmax warps
     uint64_t p_full[kTiles];      // P_t (and any O_t rescale) in tensor memory
     uint64_t pv_done[kTiles];     // O_t += P_t V complete
-    uint64_t drain;
+    uint64_t drain[kTiles];
     uint32_t tmem_base;
     int abort_flag;
     float lut[16];
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
         mbar_init(&S->q_full, 1);
         for (int b = 0; b < kRing; ++b) {
             mbar_init(&S->ld_full[b], kLdArrivals);
-            mbar_init(&S->ld_free[b], 1);
+            mbar_init(&S->ld_free[b], AttnCfg<FORM>::kIssuers);   // one commit per issuer
         }
         for (int t = 0; t < kTiles; ++t) {
             mbar_init(&S->s_full[t], 1);
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
             mbar_init(&S->p_full[t], 4);
             mbar_init(&S->pv_done[t], 1);
         }
-        mbar_init(&S->drain, 1);
+        for (int t = 0; t < kTiles; ++t) mbar_init(&S->drain[t], 1);
         S->abort_flag = 0;
         mbar_init_fence();
     }
@@ -312,6 +318,7 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
     volatile int *abort_flag = &S->abort_flag;
     const unsigned long long wait_ns = p.wait_ns;
 
+    constexpr int kLoader0 = AttnCfg<FORM>::kLoader0;
     if (threadIdx.x >= kLoader0) {
         // ------------------------------------------------------- loaders --
         const int lt = threadIdx.x - kLoader0;   // 0..kLoaders-1
@@ -431,7 +438,7 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
             }
             cp_wait_all();
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp >= kMmaWarp) {
         // ---------------------------------------------------- MMA issuer --
         // Per key block j: S_0(j + 1) as soon as tile 0's softmax has read
         // S_0(j), O_0 += P_0(j) V(j) once P_0(j) is in tensor memory, then the
@@ -457,51 +464,85 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
         };
         bool ok = warp_wait(&S->q_full, 0u, abort_flag, p.status, wait_ns) &&
                   warp_wait(&S->ld_full[0], 0u, abort_flag, p.status, wait_ns);
-        if (ok) {
-            tc_fence_after();
-            if (lane == 0) {
-                issue_s(0, 0);
-                issue_s(1, 0);
-            }
-            __syncwarp();
-        }
-        for (int j = 0; j < nkb && ok; ++j) {
-            const int b = j % kRing, b1 = (j + 1) % kRing;
-            const uint32_t par = (uint32_t)j & 1u;
-            if (j + 1 < nkb) {
-                ok = warp_wait(&S->ld_full[b1], (uint32_t)((j + 1) / kRing) & 1u, abort_flag, p.status, wait_ns) &&
-                     warp_wait(&S->s_free[0], par, abort_flag, p.status, wait_ns);
-                if (!ok) break;
+        if constexpr (AttnCfg<FORM>::kIssuers == 2) {
+            // one issuer per tile: S_t(j + 1) once the tile's softmax has read
+            // S_t(j), O_t += P_t(j) V(j) once P_t(j) is in tensor memory
+            const int t = warp - kMmaWarp;
+            if (ok) {
                 tc_fence_after();
-                if (lane == 0) issue_s(0, b1);
+                if (lane == 0) issue_s(t, 0);
                 __syncwarp();
             }
-            ok = warp_wait(&S->p_full[0], par, abort_flag, p.status, wait_ns);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) issue_pv(0, b, j == 0);
-            __syncwarp();
-            if (j + 1 < nkb) {
-                ok = warp_wait(&S->s_free[1], par, abort_flag, p.status, wait_ns);
+            for (int j = 0; j < nkb && ok; ++j) {
+                const int b = j % kRing, b1 = (j + 1) % kRing;
+                const uint32_t par = (uint32_t)j & 1u;
+                if (j + 1 < nkb) {
+                    ok = warp_wait(&S->ld_full[b1], (uint32_t)((j + 1) / kRing) & 1u, abort_flag, p.status, wait_ns) &&
+                         warp_wait(&S->s_free[t], par, abort_flag, p.status, wait_ns);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) issue_s(t, b1);
+                    __syncwarp();
+                }
+                ok = warp_wait(&S->p_full[t], par, abort_flag, p.status, wait_ns);
                 if (!ok) break;
                 tc_fence_after();
-                if (lane == 0) issue_s(1, b1);
+                if (lane == 0) {
+                    issue_pv(t, b, j == 0);
+                    tc_commit(&S->ld_free[b]);
+                }
                 __syncwarp();
             }
-            ok = warp_wait(&S->p_full[1], par, abort_flag, p.status, wait_ns);
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
-                issue_pv(1, b, j == 0);
-                tc_commit(&S->ld_free[b]);
+        } else {
+            // one issuer for both tiles: S_0(j + 1), O_0 += P_0(j) V(j), then
+            // the same for tile 1
+            if (ok) {
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_s(0, 0);
+                    issue_s(1, 0);
+                }
+                __syncwarp();
             }
-            __syncwarp();
+            for (int j = 0; j < nkb && ok; ++j) {
+                const int b = j % kRing, b1 = (j + 1) % kRing;
+                const uint32_t par = (uint32_t)j & 1u;
+                if (j + 1 < nkb) {
+                    ok = warp_wait(&S->ld_full[b1], (uint32_t)((j + 1) / kRing) & 1u, abort_flag, p.status, wait_ns) &&
+                         warp_wait(&S->s_free[0], par, abort_flag, p.status, wait_ns);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) issue_s(0, b1);
+                    __syncwarp();
+                }
+                ok = warp_wait(&S->p_full[0], par, abort_flag, p.status, wait_ns);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) issue_pv(0, b, j == 0);
+                __syncwarp();
+                if (j + 1 < nkb) {
+                    ok = warp_wait(&S->s_free[1], par, abort_flag, p.status, wait_ns);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) issue_s(1, b1);
+                    __syncwarp();
+                }
+                ok = warp_wait(&S->p_full[1], par, abort_flag, p.status, wait_ns);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_pv(1, b, j == 0);
+                    tc_commit(&S->ld_free[b]);
+                }
+                __syncwarp();
+            }
         }
         // Drain: every MMA this thread issued has completed before TMEM is freed.
         if (lane == 0) {
-            tc_commit(&S->drain);
+            uint64_t *dr = &S->drain[warp - kMmaWarp];
+            tc_commit(dr);
             volatile int no_abort = 0;
-            wait_bounded(&S->drain, 0u, &no_abort, p.status, kAttnWaitNs);
+            wait_bounded(dr, 0u, &no_abort, p.status, kAttnWaitNs);
         }
         __syncwarp();
     } else if (warp < kMmaWarp) {
