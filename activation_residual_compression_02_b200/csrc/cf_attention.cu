@@ -105,6 +105,7 @@ struct AttnSmem {
     uint64_t s_free[kTiles];      // S_t read by the tile's four softmax warps
     uint64_t p_full[kTiles];      // P_t (and any O_t rescale) in tensor memory
     uint64_t pv_done[kTiles];     // O_t += P_t V complete
+    uint64_t turn[kTiles][4];     // per sub-partition: tile t may run its exponentials
     uint64_t drain[kTiles];
     uint32_t tmem_base;
     int abort_flag;
@@ -204,11 +205,22 @@ __device__ __forceinline__ uint64_t vdesc(uint32_t saddr) { return smem_desc(sad
 
 // A bounded wait whose outcome is the same for every lane of the warp, so that
 // the warp never splits across the .sync.aligned tcgen05 instructions after it.
+// The first test is inline (a barrier already past costs one try_wait); only a
+// wait that has to spin calls the bounded loop.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, uint32_t *status,
                                           unsigned long long ns)
 {
-    const bool ok = wait_bounded(bar, parity, abort_flag, status, ns);
+    bool ok = mbar_try_wait(smem_u32(bar), parity);
+    if (!ok) ok = wait_bounded(bar, parity, abort_flag, status, ns);
     return __all_sync(0xffffffffu, ok);
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 __device__ __forceinline__ void cp_async(void *dst, const void *src, int bytes)
@@ -296,6 +308,7 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
             mbar_init(&S->s_free[t], 4);               // one arrival per softmax warp of the tile
             mbar_init(&S->p_full[t], 4);
             mbar_init(&S->pv_done[t], 1);
+            for (int w = 0; w < 4; ++w) mbar_init(&S->turn[t][w], 1);
         }
         for (int t = 0; t < kTiles; ++t) mbar_init(&S->drain[t], 1);
         S->abort_flag = 0;
@@ -580,13 +593,15 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
 #pragma unroll
                 for (int c = 0; c < kBlockK; ++c) s[c] = c < kvalid ? s[c] : -INFINITY;
             }
-            float mx[8];
+            float mx[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+            for (int e = 0; e < 4; ++e) mx[e] = fmaxf(s[2 * e], s[2 * e + 1]);
 #pragma unroll
-            for (int c = 8; c < kBlockK; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-            const float m_blk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int c = 8; c < kBlockK; c += 8) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) mx[e] = fmax3(mx[e], s[c + 2 * e], s[c + 2 * e + 1]);
+            }
+            const float m_blk = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
             // move the reference maximum only when it grows by more than 2^8 in base 2
             const bool grow = (m_blk - m) * c2 > kRescaleLog2;   // true on the first block (m = -inf)
             const bool rescale = __any_sync(0xffffffffu, grow) && j > 0;
@@ -604,6 +619,15 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
                 }
                 tc_fence_after();
             }
+            // The two tiles' warps on this sub-partition take turns at the
+            // exponentials (tile 0 first in every block; the turn passes when
+            // half of a block's are done), so that one tile's loads, maximum
+            // and waits overlap the other's use of the unit.
+            if ((t == 1 || j > 0) &&
+                !warp_wait(&S->turn[t][warp & 3], (uint32_t)(t == 1 ? j : j - 1) & 1u, abort_flag, p.status, wait_ns)) {
+                ok = false;
+                break;
+            }
             // P = 2^(s c2 - m c2) in 32-key chunks, each packed to bf16 pairs and
             // stored to tensor memory as soon as it is formed
             float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -618,6 +642,10 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
                     v[e] = bf16x2(x0, x1);
                 }
                 tmem_st16(tP + (uint32_t)(q >> 1), v);
+                if (q == 32 * 2) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&S->turn[t ^ 1][warp & 3]);
+                }
             }
             l = l * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
             if (rescale) {
