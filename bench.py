@@ -627,9 +627,10 @@ def run_cf(args, w):
                          f"thread, {cores} threads, {dt:.1f} s wall"}
 
     # ---- the other workloads of the codec, as extra keys of this line ----
-    # The CogVideoX-shaped and stress steps (quantised), and the low-rank call
-    # (Algorithm 3 + apply on 57 x 4608 x 3072 fp32), each timed the same way.
-    cog = stress = lowrank = None
+    # The CogVideoX-shaped and stress steps (quantised), the low-rank call
+    # (Algorithm 3 + apply on 57 x 4608 x 3072 fp32), and the attention that
+    # consumes a received CogVideoX-shaped K/V shard, each timed the same way.
+    cog = stress = lowrank = attention = None
     if not args.no_extra:
         del X, slot_lists, c_slots, slots0, st
         torch.cuda.empty_cache()
@@ -639,6 +640,8 @@ def run_cf(args, w):
                                   0 if args.no_cpu else 4)
         if lowrank.get("cpu_baseline"):
             lowrank["cpu_baseline"]["sample"] += " (a bounded sample: the run stays short)"
+        torch.cuda.empty_cache()
+        attention = attention_measure(args, synth.COGVIDEOX, world, rank, clk, min(args.steps, 10))
     clk.stop()
 
     line = {
@@ -656,7 +659,7 @@ def run_cf(args, w):
                           "alg_bytes_per_step": (bc + bd) * n_elem},
         "loopback": lb, "lean_state": lean, "recon": rc, "warmup_step": warm,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
-        "cogvideox": cog, "stress": stress, "lowrank": lowrank,
+        "cogvideox": cog, "stress": stress, "lowrank": lowrank, "attention": attention,
         "clocks": clk.summary(),
     }
     if rank == 0:
@@ -1029,7 +1032,20 @@ def run_exchange_bench(args, w):
     return 0
 
 
-def run_attention_bench(args, w):
+# The exponential unit bounds attention with heads of 64: one 2^x per score
+# against 4 * 64 flops of the two products.  A microbenchmark of the softmax
+# loop (registers only) measured 8.7 cycles per warp-wide ex2 on one
+# sub-partition, with one warp or two; at 4 sub-partitions x 148 SMs and the
+# 1965 MHz clock that is 4.28e12 exponentials/s, i.e. 1095 TFLOP/s of attention.
+XU_CLK_PER_WARP_EX2 = 8.7
+
+
+def xu_bound_tflops(head_dim=64, sm_mhz=1965.0, sms=148):
+    ex2_per_s = sms * 4 * 32 / XU_CLK_PER_WARP_EX2 * sm_mhz * 1e6
+    return ex2_per_s * 4 * head_dim / 1e12
+
+
+def attention_measure(args, w, world, rank, clk, steps):
     """The consumer of the compressed K/V exchange (Algorithms 1 and 2): one
     step of attention over a received shard for every layer of the workload
     (the layer's K and V slots, 4444 tokens x 1920 channels = 30 heads of 64
@@ -1041,12 +1057,11 @@ def run_attention_bench(args, w):
       dequantise  cf_attention reading the caches and the step's payload,
                   dequantising on load and writing the new caches (no
                   decompress launch).
-    Reports ms per step of each and the attention's TFLOP/s."""
-    world, rank, local = dist_init()
+    Returns ms per step of each and the attention kernel's TFLOP/s against
+    the measured bf16 peak and the exponential-unit bound."""
     import activation_residual_compression_02_b200 as cf
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    clk = ClockSampler(torch.cuda.current_device()).start()
     layers = w.slots
     shapes = [(w.rows, w.cols)] * (2 * layers)        # K and V of every layer
     ctx = cf.Context(shapes, bits=w.bits, group=w.group)
@@ -1114,35 +1129,58 @@ def run_attention_bench(args, w):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with Timed(clk):
             e0.record(stream)
-            for _ in range(args.steps):
+            for _ in range(steps):
                 fn()
             e1.record(stream)
             torch.cuda.synchronize()
-        return max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        return max_over_ranks(e0.elapsed_time(e1), world) / steps
 
     ms = {name: time_it(fn) for name, fn in (("attention_only", attention_only), ("recon", path_recon),
                                              ("cast", path_cast), ("dequantise", path_dequantise))}
     if ctx.check() != 0:
         raise RuntimeError("device status in the attention run")
-    clk.stop()
     flops = 4.0 * w.rows * w.rows * w.cols * layers     # Q K^T and P V: 2 * 2 * lq * lk * 64 per head
     peak = bf16_peak()
-    line = {
-        "metric": "ring-attention step over a received K/V shard (every layer): ms per step", "value": ms["recon"],
-        "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms["recon"],
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name}: {layers} layers, K and V slots of {w.rows} tokens x {w.cols} channels "
-                               f"({w.cols // 64} heads of 64), k={w.bits}, G={w.group}; queries {w.rows} x {w.cols}",
-                   "l2": "inputs larger than L2 (every layer's caches, payloads and queries)"},
-        "paths_ms": ms,
-        "attention": {"tflops": flops / (ms["attention_only"] * 1e-3) / 1e12,
-                      "frac_of_bf16_peak": flops / (ms["attention_only"] * 1e-3) / 1e12 / peak[0],
-                      "peak_tflops": peak[0], "peak_kind": peak[1], "flops_per_step": flops},
+    tf = flops / (ms["attention_only"] * 1e-3) / 1e12
+    xu = xu_bound_tflops()
+    ctx.close()
+    return {
+        "workload": f"{w.name}: {layers} layers, K and V slots of {w.rows} tokens x {w.cols} channels "
+                    f"({w.cols // 64} heads of 64), k={w.bits}, G={w.group}; queries {w.rows} x {w.cols}",
+        "steps": steps, "paths_ms": ms, "ms_per_step": ms["recon"],
+        "roofline": {"bound": "tensor", "kernel": "k_attention<bf16>", "achieved": tf, "peak": peak[0],
+                     "peak_kind": peak[1], "unit": "TFLOP/s", "frac": tf / peak[0],
+                     "traffic": recorded_traffic("attention", "cf_attention.cu"),
+                     "tensor_pipe": recorded_traffic("attention", "cf_attention.cu", "tensor_pipe_active"),
+                     "xu_pipe": recorded_traffic("attention", "cf_attention.cu", "xu_pipe_active"),
+                     "flops_per_step": flops, "xu_bound": xu, "frac_of_xu_bound": tf / xu,
+                     "xu_bound_how": "4 sub-partitions x 148 SMs x 32 lanes / 8.7 cycles per warp-wide ex2 "
+                                     "(measured) x 1965 MHz x 256 flops per exponential (heads of 64)"},
         "dequantise_vs_recon": ms["dequantise"] / ms["recon"],
         "note": "recon: cf_decompress writing bf16(C) in its pass + cf_attention on bf16; cast: cf_decompress + "
                 "torch cast of each cache + cf_attention; dequantise: cf_attention reading C_{t-1}, codes and scales "
                 "and writing C_t (no decompress launch)",
-        "gpu_launches": args.steps * (1 + layers), "clocks": clk.summary(),
+        "gpu_launches_per_step": {"attention_only": layers, "recon": 1 + layers, "cast": 1 + layers,
+                                  "dequantise": layers},
+    }
+
+
+def run_attention_bench(args, w):
+    """`--attention`: the attention measurement as the headline of its own line."""
+    world, rank, local = dist_init()
+    clk = ClockSampler(torch.cuda.current_device()).start()
+    r = attention_measure(args, w, world, rank, clk, args.steps)
+    clk.stop()
+    line = {
+        "metric": "attention step over a received K/V shard (every layer, recon path): ms per step",
+        "value": r["ms_per_step"], "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": r["ms_per_step"], "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": r["workload"], "l2": "inputs larger than L2 (every layer's caches, payloads and "
+                                                     "queries)"},
+        "paths_ms": r["paths_ms"], "roofline": r["roofline"], "dequantise_vs_recon": r["dequantise_vs_recon"],
+        "note": r["note"], "gpu_launches": args.steps * r["gpu_launches_per_step"]["recon"],
+        "clocks": clk.summary(),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
