@@ -68,7 +68,7 @@ def lib() -> ctypes.CDLL:
         _lib.cfo_compress_lean.argtypes = [I64, I, I, I, P, P, P, P, P, U32P]
         _lib.cfo_decompress_lean.argtypes = [I64, I, I, P, P, P]
         _lib.cfo_to_bf16.argtypes = [I64, P, P]
-        _lib.cfo_attention.argtypes = [I64, I64, I64, P, P, P, P]
+        _lib.cfo_attention.argtypes = [I64, I64, I64, P, P, P, P, P]
     return _lib
 
 
@@ -281,15 +281,19 @@ def lowrank_apply(A: np.ndarray, U: np.ndarray, R: np.ndarray, V: np.ndarray,
 
 # ----------------------------------------------------------------- attention
 
-def attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, cols: int) -> np.ndarray:
+def attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, cols: int, lse: bool = False):
     """softmax(q k^T / 8) v per head of 64 channels, in fp64.
 
     q [lq, cols], k and v [lk, cols] as raw bf16 bit patterns (token-major);
-    returns fp64 [lq, cols]."""
+    returns fp64 [lq, cols], and with ``lse`` also the fp64 log-sum-exp of the
+    scaled scores [lq, cols // 64] (the weight of this K/V block when partial
+    results over several blocks are merged)."""
     q = np.ascontiguousarray(_u16(q_bits)).reshape(-1, cols)
     k = np.ascontiguousarray(_u16(k_bits)).reshape(-1, cols)
     v = np.ascontiguousarray(_u16(v_bits)).reshape(-1, cols)
     assert k.shape == v.shape
     out = np.empty((q.shape[0], cols), np.float64)
-    _check(lib().cfo_attention(q.shape[0], k.shape[0], cols, _ptr(q), _ptr(k), _ptr(v), _ptr(out)), "attention")
-    return out
+    ls = np.empty((q.shape[0], cols // 64), np.float64) if lse else None
+    _check(lib().cfo_attention(q.shape[0], k.shape[0], cols, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                               _ptr(ls) if lse else None), "attention")
+    return (out, ls) if lse else out

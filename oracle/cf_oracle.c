@@ -494,9 +494,14 @@ int cfo_decompress_lean(int64_t n, int k, int G, const uint8_t *codes, const flo
  *   score(i, j) = (q_i . k_j) / 8          (8 = sqrt(64))
  *   w(i, j)     = exp(score(i, j) - max_j score(i, j)) / sum_j (same)
  *   out(i, c)   = sum_j w(i, j) v(j, c)
- * q, k, v are bf16 bit patterns; out is fp64 [lq x cols]. */
+ *   lse(i)      = log sum_j exp(score(i, j))   (if lse is not NULL)
+ * The log-sum-exp of a row is what merges partial results over several K/V
+ * blocks (ring attention, Algorithm 2): the softmax over their union weighs
+ * each block's output by exp(lse_block - lse_union).
+ * q, k, v are bf16 bit patterns; out is fp64 [lq x cols], lse fp64
+ * [lq x cols / 64] (query-major). */
 int cfo_attention(int64_t lq, int64_t lk, int64_t cols, const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                  double *out)
+                  double *out, double *lse)
 {
     if (lq < 0 || lk < 1 || cols < 64 || cols % 64 != 0) return CFO_E_ARG;
     double *w = (double *)malloc((size_t)lk * sizeof(double));
@@ -522,6 +527,7 @@ int cfo_attention(int64_t lq, int64_t lk, int64_t cols, const uint16_t *q, const
                 for (int64_t j = 0; j < lk; ++j) o += w[j] * (double)bf16_to_float(v[j * cols + c0 + c]);
                 out[i * cols + c0 + c] = o / z;
             }
+            if (lse) lse[i * (cols / 64) + h] = mx + log(z);
         }
     }
     free(w);

@@ -121,3 +121,60 @@ def test_key_order_does_not_matter(oracle):
     out = oracle.attention(q, k, v, cols)
     out2 = oracle.attention(q, k[perm], v[perm], cols)
     assert np.allclose(out, out2, rtol=0, atol=1e-12)
+
+
+# ---- the log-sum-exp of a row: what merges partial results over K/V blocks --
+
+
+def test_lse_of_a_single_key_is_its_score(oracle):
+    """With one key the sum has one term: lse = score = (q . k) / 8, here with
+    values chosen so that the dot product is exact (q . k = 2 * 3 + 0.5 * -4)."""
+    cols = 2 * H
+    q = np.zeros((1, cols), np.float32)
+    k = np.zeros((1, cols), np.float32)
+    q[0, 5], k[0, 5] = 2.0, 3.0
+    q[0, H + 7], k[0, H + 7] = 0.5, -4.0
+    _, lse = oracle.attention(bits(q), bits(k), rand_bf16((1, cols), 20), cols, lse=True)
+    assert lse.shape == (1, 2)
+    assert lse[0, 0] == 6.0 / 8.0
+    assert lse[0, 1] == -2.0 / 8.0
+
+
+def test_lse_of_identical_keys_adds_log_count(oracle):
+    """n equal scores s: lse = s + ln n."""
+    cols = H
+    q = np.zeros((3, cols), np.float32)
+    q[:, 2] = [1.0, -2.0, 0.25]
+    k = np.zeros((13, cols), np.float32)
+    k[:, 2] = 4.0
+    _, lse = oracle.attention(bits(q), bits(k), rand_bf16((13, cols), 21), cols, lse=True)
+    want = np.array([4.0, -8.0, 1.0]) / 8.0 + math.log(13.0)
+    assert np.allclose(lse[:, 0], want, rtol=1e-15, atol=1e-15)
+
+
+def test_lse_of_a_dominant_key_is_its_score(oracle):
+    """Scores 1000 and 0 (five times): lse = 1000 + ln(1 + 5 e^-1000) = 1000
+    in fp64, with no overflow on the way."""
+    cols = H
+    q = np.zeros((1, cols), np.float32)
+    q[0, 0] = 80.0
+    k = np.zeros((6, cols), np.float32)
+    k[3, 0] = 100.0
+    _, lse = oracle.attention(bits(q), bits(k), rand_bf16((6, cols), 22), cols, lse=True)
+    assert lse[0, 0] == 1000.0
+
+
+def test_two_blocks_merge_by_lse_into_the_whole(oracle):
+    """Attention over the keys of two blocks equals the two blocks' outputs
+    weighted by exp(lse_b - lse), lse = ln(e^lse_1 + e^lse_2): the merge a
+    ring step does (Algorithm 2) with each block's partial result."""
+    cols = 2 * H
+    q, k, v = rand_bf16((7, cols), 23, 2.0), rand_bf16((50, cols), 24, 2.0), rand_bf16((50, cols), 25)
+    whole, lse = oracle.attention(q, k, v, cols, lse=True)
+    o1, l1 = oracle.attention(q, k[:19], v[:19], cols, lse=True)
+    o2, l2 = oracle.attention(q, k[19:], v[19:], cols, lse=True)
+    merged_lse = np.logaddexp(l1, l2)
+    assert np.allclose(merged_lse, lse, rtol=0, atol=1e-12)
+    w1 = np.repeat(np.exp(l1 - merged_lse), H, axis=1)
+    w2 = np.repeat(np.exp(l2 - merged_lse), H, axis=1)
+    assert np.allclose(w1 * o1 + w2 * o2, whole, rtol=0, atol=1e-12)

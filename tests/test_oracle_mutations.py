@@ -39,6 +39,10 @@ MUTATIONS = [
     ("attention scale 1/64", "w[j] = s / 8.0;", "w[j] = s / 64.0;", False),
     ("softmax max not taken out", "w[j] = exp(w[j] - mx);", "w[j] = exp(w[j]);", False),
     ("softmax not normalised", "out[i * cols + c0 + c] = o / z;", "out[i * cols + c0 + c] = o;", False),
+    ("log-sum-exp without the maximum", "lse[i * (cols / 64) + h] = mx + log(z);",
+     "lse[i * (cols / 64) + h] = log(z);", False),
+    ("log-sum-exp in base 2", "lse[i * (cols / 64) + h] = mx + log(z);",
+     "lse[i * (cols / 64) + h] = mx + log2(z);", False),
 ]
 
 
