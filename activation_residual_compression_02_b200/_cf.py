@@ -105,7 +105,7 @@ def lib() -> ctypes.CDLL:
         L.cf_trace_read.restype = I
         L.cf_lowrank_noalloc.argtypes = [ctypes.POINTER(cf_config), I, I64, I64, PP, PP, PP, PP, PP, PP, PP, P]
         L.cf_lowrank_noalloc.restype = I
-        L.cf_attention.argtypes = [P, I64, I64, I64, P, ctypes.POINTER(cf_kv), ctypes.POINTER(cf_kv), P, P]
+        L.cf_attention.argtypes = [P, I64, I64, I64, P, ctypes.POINTER(cf_kv), ctypes.POINTER(cf_kv), P, P, P]
         L.cf_attention.restype = I
         _lib = L
     return _lib
@@ -255,12 +255,17 @@ class Context:
         self._raise(st, "cf_lowrank")
 
     def attention(self, q: torch.Tensor, k: KV, v: KV, out: torch.Tensor, lk: Optional[int] = None,
-                  stream: Optional[torch.cuda.Stream] = None):
+                  stream: Optional[torch.cuda.Stream] = None, lse: Optional[torch.Tensor] = None):
         """cf_attention: out = softmax(q k^T / 8) v per head of 64 channels.
-        q and out are bf16 [lq, cols]; lk defaults to the rows of k's tensors."""
+        q and out are bf16 [lq, cols]; lk defaults to the rows of k's tensors;
+        lse (optional) is fp32 [lq, cols // 64] and receives each row's
+        log-sum-exp of the scaled scores (to merge partial results over blocks)."""
         if q.dim() != 2 or q.dtype != torch.bfloat16 or out.dtype != torch.bfloat16 or out.shape != q.shape:
             raise ValueError("q and out must be bf16 [lq, cols] of the same shape")
         lq, cols = int(q.shape[0]), int(q.shape[1])
+        if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (lq, cols // 64)
+                                or not lse.is_contiguous()):
+            raise ValueError("lse must be a contiguous fp32 [lq, cols // 64] tensor")
         if lk is None:
             t = k.bf16 if k.bf16 is not None else k.cache_in
             lk = int(t.numel() // cols) if t is not None else 0
@@ -268,7 +273,7 @@ class Context:
             kv.check(lk, cols, self.cfg.bits, self.cfg.group, name)
         kc, vc = k.to_c(), v.to_c()
         st = lib().cf_attention(self._h, lq, lk, cols, _ptr(q), ctypes.byref(kc), ctypes.byref(vc), _ptr(out),
-                                _stream_handle(stream))
+                                _ptr(lse) if lse is not None else None, _stream_handle(stream))
         self._raise(st, "cf_attention")
 
     def trace(self, on: bool = True):

@@ -591,7 +591,7 @@ bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb)
 }  // namespace
 
 cf_status cf_attention(cf_ctx *ctx, int64_t lq, int64_t lk, int64_t cols, const void *q, const cf_kv *k,
-                       const cf_kv *v, void *out, void *cuda_stream)
+                       const cf_kv *v, void *out, float *lse, void *cuda_stream)
 try {
     if (!ctx) return CF_E_ARG;
     DeviceGuard device(ctx);
@@ -604,11 +604,13 @@ try {
     if (lq == 0) return CF_OK;
     if (!q || !k || !v || !out) return fail(ctx, CF_E_ARG, "q, k, v and out must be non-NULL");
     if (!aligned16(q) || !aligned16(out)) return fail(ctx, CF_E_ALIGN, "q and out must be 16-byte aligned");
+    if (lse && ((uintptr_t)lse & 3u) != 0) return fail(ctx, CF_E_ALIGN, "lse must be 4-byte aligned");
     const bool deq = k->bf16 == nullptr;
     if ((v->bf16 == nullptr) != deq) return fail(ctx, CF_E_ARG, "k and v must come in the same form");
     cf::AttnArgs a{};
     a.q = q;
     a.out = out;
+    a.lse = lse;
     a.lq = lq;
     a.lk = lk;
     a.cols = cols;

@@ -123,6 +123,7 @@ struct __align__(64) AttnParams {
     const uint8_t *codes[2];      // k-bit stream (form 1)
     const float *scales[2];       // fp32 per group (form 1)
     uint16_t *out;                // bf16 [lq x cols]
+    float *lse;                   // fp32 [lq x cols/64] or null
     int lq, lk, cols;
     int group;
     int group_lg;                 // log2(group)
@@ -690,6 +691,8 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)qrow * p.cols + col0);
 #pragma unroll
                 for (int c = 0; c < kHeadDim / 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                // log sum_j e^(s_j / 8) = ln 2 * (m log2(e) / 8 + log2 l): l was summed against the reference m
+                if (p.lse) p.lse[(int64_t)qrow * (p.cols / kHeadDim) + head] = (m * c2 + log2f(l)) * 0.69314718055994531f;
             }
         }
     }
@@ -755,6 +758,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream)
         p.scales[i] = a.scales[i];
     }
     p.out = static_cast<uint16_t *>(a.out);
+    p.lse = a.lse;
     p.lq = (int)a.lq;
     p.lk = (int)a.lk;
     p.cols = (int)a.cols;

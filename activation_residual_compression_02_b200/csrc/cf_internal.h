@@ -95,7 +95,8 @@ cudaError_t launch_residual_f32(const void *const *x, void *const *base, const f
 
 // Attention over a received K/V shard (cf_attention): heads of 64 channels,
 // K and V as bf16 (kv) or dequantised on load from cache_in + codes/scales
-// (dequantise = true), the new cache written to cache_out when non-null.
+// (dequantise = true), the new cache written to cache_out when non-null;
+// the log-sum-exp of every row and head to lse when non-null.
 struct AttnArgs {
     const void *q;
     const void *kv[2];
@@ -104,6 +105,7 @@ struct AttnArgs {
     const uint8_t *codes[2];
     const float *scales[2];
     void *out;
+    float *lse;          // [lq x cols/64] or null
     int64_t lq, lk, cols;
     int bits, group;
     bool dequantise;

@@ -270,6 +270,11 @@ typedef struct cf_kv {
  * layout), out_h = softmax(q_h k_h^T / 8) v_h.
  *   q, out  bf16 [lq x cols] (16-byte aligned); k, v of [lk x cols], both in
  *   the same cf_kv form; cols a multiple of 64 (and of G when dequantising).
+ *   lse     fp32 [lq x cols/64] (query-major, 4-byte aligned) or NULL: the
+ *   natural log of sum_j exp(q_h . k_j / 8) of every row and head.  A ring
+ *   step that attends over one received block at a time merges the partial
+ *   outputs with it: over the union of blocks b, out = sum_b exp(lse_b -
+ *   lse) out_b with lse = log sum_b exp(lse_b).
  * The products run on the tensor cores in bf16 with fp32 accumulation, the
  * softmax in fp32 (base 2, online over blocks of 128 keys, P rounded to bf16).
  * Dequantise-on-load needs a quantised-mode context with fp32 state (its k
@@ -277,14 +282,15 @@ typedef struct cf_kv {
  * word.  The two forms give bit-identical outputs for the same C_t.
  * Stream-ordered; allocates nothing.  Errors before launch: CF_E_ARG (NULL
  * pointer, mixed forms, overlapping caches, wrong context), CF_E_SHAPE (lk <
- * 1, cols not a multiple of 64 or of G), CF_E_ALIGN; device-side:
+ * 1, cols not a multiple of 64 or of G), CF_E_ALIGN (q, out, k, v or lse
+ * misaligned); device-side:
  * CF_E_TIMEOUT at the next cf_check.
  * Source: reproducibility table, "Pseudocode" row, Algorithms 1 and 2 (each
  * device attends over the key/value blocks it receives from the others);
  * abstract (the receiver adds each decompressed residual to its
  * reconstruction). */
 cf_status cf_attention(cf_ctx *ctx, int64_t lq, int64_t lk, int64_t cols, const void *q, const cf_kv *k,
-                       const cf_kv *v, void *out, void *cuda_stream);
+                       const cf_kv *v, void *out, float *lse, void *cuda_stream);
 
 /* Bytes of device scratch that the library keeps on every GPU it is loaded
  * on, for cf_lowrank_noalloc (status word plus the Algorithm 3 buffers). */

@@ -13,7 +13,13 @@ and the abstract (the receiver accumulates the decompressed residuals).
   step's payload, must write exactly the cache the oracle's decompress gives
   (bit for bit) and produce exactly the output of the bf16 form fed the
   receiver's recon after the same step.
+* The log-sum-exp of every row is compared with the oracle's within 2e-4
+  (the scores are exact products of bf16 values summed in fp32, the sum of
+  the exponentials is fp32), and two shards merged by it must give the
+  attention over their union (a ring step, Algorithm 2).
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -99,10 +105,14 @@ def test_attention_dequantise_matches_decompress_path(cf, oracle, bits, group, l
     out_b = torch.empty_like(out_a)
     new = [torch.full((lk * cols,), 12345.0, device="cuda") for _ in range(2)]
     kv = [cf.KV(cache_in=before[i], cache_out=new[i], codes=st.codes[i], scales=st.scales[i]) for i in range(2)]
-    ctx.attention(q, kv[0], kv[1], out_b)
+    lse_a = torch.empty(lq, cols // 64, device="cuda")
+    lse_b = torch.full((lq, cols // 64), 7.0, device="cuda")
+    ctx.attention(q, cf.KV(bf16=st.recon[0]), cf.KV(bf16=st.recon[1]), out_a, lse=lse_a)
+    ctx.attention(q, kv[0], kv[1], out_b, lse=lse_b)
     torch.cuda.synchronize()
     assert ctx.check() == cf.CF_OK
     assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+    assert torch.equal(lse_a, lse_b)
     for i in range(2):
         c = before[i].cpu().numpy().copy()
         oracle.decompress(st.codes[i].cpu().numpy(), st.scales[i].cpu().numpy(), c, bits, group)
@@ -136,6 +146,45 @@ def test_attention_full_size_cogvideox_shard(cf, oracle):
     qs = q[rows]
     want = oracle.attention(u16(qs), u16(st.recon[0]), u16(st.recon[1]), cols)
     assert rel_per_head(out_b[rows].float().cpu().double().numpy(), want, cols) <= 1e-2
+
+
+@pytest.mark.parametrize("lq,lk,cols,scale", [(300, 260, 128, 1.0), (129, 1000, 192, 3.0), (1, 1, 64, 1.0),
+                                              (256, 4444, 64, 1.0)])
+def test_attention_lse_matches_oracle(cf, oracle, lq, lk, cols, scale):
+    q, k, v = bf16_rand((lq, cols), 31, scale), bf16_rand((lk, cols), 32, scale), bf16_rand((lk, cols), 33)
+    ctx = cf.Context([], mode=cf.CF_MODE_QUANT)
+    out = torch.empty(lq, cols, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(lq, cols // 64, device="cuda")
+    ctx.attention(q.cuda(), cf.KV(bf16=k.cuda()), cf.KV(bf16=v.cuda()), out, lse=lse)
+    assert ctx.check() == cf.CF_OK
+    want_out, want_lse = oracle.attention(u16(q), u16(k), u16(v), cols, lse=True)
+    assert rel_per_head(out.float().cpu().double().numpy(), want_out, cols) <= 1e-2
+    got = lse.cpu().double().numpy()
+    assert np.max(np.abs(got - want_lse) / np.maximum(1.0, np.abs(want_lse))) <= 2e-4
+
+
+def test_ring_step_merges_two_shards_by_lse(cf, oracle):
+    """A device that receives K/V in two blocks (a ring, Algorithm 2) attends
+    over each and merges the partial outputs by their log-sum-exp; the result
+    is the attention over the union of the blocks."""
+    lq, cols = 300, 128
+    q = bf16_rand((lq, cols), 41, 2.0)
+    ks = [bf16_rand((n, cols), 42 + i, 2.0) for i, n in enumerate((1000, 777))]
+    vs = [bf16_rand((n, cols), 52 + i) for i, n in enumerate((1000, 777))]
+    ctx = cf.Context([], mode=cf.CF_MODE_QUANT)
+    outs, lses = [], []
+    for kb, vb in zip(ks, vs):
+        o = torch.empty(lq, cols, dtype=torch.bfloat16, device="cuda")
+        ls = torch.empty(lq, cols // 64, device="cuda")
+        ctx.attention(q.cuda(), cf.KV(bf16=kb.cuda()), cf.KV(bf16=vb.cuda()), o, lse=ls)
+        outs.append(o.double().cpu())
+        lses.append(ls.double().cpu())
+    assert ctx.check() == cf.CF_OK
+    lse = torch.logaddexp(lses[0], lses[1])
+    merged = sum(torch.exp(l_ - lse).repeat_interleave(64, dim=1) * o for l_, o in zip(lses, outs))
+    want_out, want_lse = oracle.attention(u16(q), u16(torch.cat(ks)), u16(torch.cat(vs)), cols, lse=True)
+    assert rel_per_head(merged.numpy(), want_out, cols) <= 1e-2
+    assert np.max(np.abs(lse.numpy() - want_lse)) <= 2e-4
 
 
 def test_attention_is_deterministic(cf):
@@ -176,6 +225,15 @@ def test_attention_arguments_checked(cf):
         kv = cf.KV(cache_in=c_in, codes=codes, scales=scales)
         lean.attention(q, kv, kv, out)
     assert e.value.status == cf.CF_E_ARG
+    raw = torch.empty(8 * 2 + 1, device="cuda")
+    with pytest.raises(cf.CfError) as e:        # lse must be 4-byte aligned
+        L = cf.lib()
+        st = L.cf_attention(ctx.handle, 8, lk, cols, q.data_ptr(), ctypes.byref(cf.KV(bf16=k).to_c()),
+                            ctypes.byref(cf.KV(bf16=k).to_c()), out.data_ptr(), raw.data_ptr() + 2, None)
+        ctx._raise(st, "cf_attention")
+    assert e.value.status == cf.CF_E_ALIGN
+    with pytest.raises(ValueError):             # lse of the wrong shape
+        ctx.attention(q, cf.KV(bf16=k), cf.KV(bf16=k), out, lse=torch.empty(8, 3, device="cuda"))
     # no queries: nothing to do
     ctx.attention(q[:0], cf.KV(bf16=k), cf.KV(bf16=k), out[:0], lk=lk)
     assert ctx.check() == cf.CF_OK
