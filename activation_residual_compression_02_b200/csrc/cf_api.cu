@@ -51,6 +51,7 @@ struct cf_ctx {
     bool warm_receiver = false;
     int64_t lowrank_steps = 0;   // compressed low-rank steps done (for warm_start)
     bool starve_once = false;    // failure-detection test: the next cf_lowrank withholds its loads
+    bool starve_attention_once = false;   // the same for the next cf_attention
     int device = 0;
     std::string err;
 };
@@ -438,6 +439,10 @@ try {
     // run out and the next cf_check reports CF_E_TIMEOUT (no GPU fault).
     const char *starve = getenv("CF_TEST_STARVE_GEMM");
     ctx->starve_once = config->mode == CF_MODE_LOWRANK && starve && starve[0] == '1';
+    // Likewise CF_TEST_STARVE_ATTENTION=1: the context's first cf_attention call
+    // issues no loads and gives up on its waits after 20 ms.
+    const char *starve_attn = getenv("CF_TEST_STARVE_ATTENTION");
+    ctx->starve_attention_once = starve_attn && starve_attn[0] == '1';
     try {
         ctx->shapes.assign(shapes, shapes + nslots);
     } catch (const std::bad_alloc &) {
@@ -648,6 +653,8 @@ try {
         a.bits = ctx->cfg.bits;
         a.group = ctx->cfg.group;
     }
+    a.starve = ctx->starve_attention_once;
+    ctx->starve_attention_once = false;
     cudaError_t e = cf::launch_attention(a, (cudaStream_t)cuda_stream);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "cf_attention");
     ctx->err.clear();

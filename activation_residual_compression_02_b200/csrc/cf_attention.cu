@@ -130,6 +130,7 @@ struct __align__(64) AttnParams {
     float scale_log2;             // log2(e) / sqrt(64)
     uint32_t *status;
     unsigned long long wait_ns;
+    int starve;                   // failure-detection test: the loaders issue nothing
 };
 
 // Byte offset of 16-byte piece `chunk` (0..7) of row `row` in a [rows x 64]
@@ -336,6 +337,10 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
     if (threadIdx.x >= kLoader0) {
         // ------------------------------------------------------- loaders --
         const int lt = threadIdx.x - kLoader0;   // 0..kLoaders-1
+        // Fault injection for the failure-detection test: with nothing loaded,
+        // the MMA issuers' bounded wait on Q runs out, they raise the abort
+        // flag and every other wait of the CTA gives up.
+        if (p.starve) goto loaders_done;
         if (lt == 0) {
             // Q of both tiles by TMA; rows past lq read as zero
             mbar_expect_tx(&S->q_full, (uint32_t)(kTiles * kTileBytes));
@@ -452,6 +457,7 @@ __global__ void __launch_bounds__(AttnCfg<FORM>::kThreads, 1) k_attention(const 
             }
             cp_wait_all();
         }
+    loaders_done:;
     } else if (warp >= kMmaWarp) {
         // ---------------------------------------------------- MMA issuer --
         // Per key block j: S_0(j + 1) as soon as tile 0's softmax has read
@@ -768,6 +774,10 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream)
     p.scale_log2 = 1.4426950408889634f / 8.0f;   // log2(e) / sqrt(64)
     p.status = a.status;
     p.wait_ns = kAttnWaitNs;
+    if (a.starve) {
+        p.starve = 1;
+        p.wait_ns = 20000000ull;
+    }
     // Q (both forms) and bf16 K, V by TMA: [rows x cols] bf16, a 64-channel x 128-row box
     if (!make_map_bf16(&p.tq, a.q, (uint64_t)a.cols, (uint64_t)a.lq, (uint64_t)a.cols, kHeadDim, kBlockQ))
         return cudaErrorInvalidValue;

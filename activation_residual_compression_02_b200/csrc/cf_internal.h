@@ -109,6 +109,7 @@ struct AttnArgs {
     int64_t lq, lk, cols;
     int bits, group;
     bool dequantise;
+    bool starve;         // failure-detection test only: no loads, 20 ms waits (they time out)
     uint32_t *status;
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t stream);

@@ -280,7 +280,10 @@ typedef struct cf_kv {
  * Dequantise-on-load needs a quantised-mode context with fp32 state (its k
  * and G describe the payload); the bf16 form only uses the context's status
  * word.  The two forms give bit-identical outputs for the same C_t.
- * Stream-ordered; allocates nothing.  Errors before launch: CF_E_ARG (NULL
+ * Stream-ordered; allocates nothing.  Every wait in the kernel is bounded
+ * (failure-detection test hook: CF_TEST_STARVE_ATTENTION=1 in the environment
+ * when the context is created makes its first cf_attention call time out).
+ * Errors before launch: CF_E_ARG (NULL
  * pointer, mixed forms, overlapping caches, wrong context), CF_E_SHAPE (lk <
  * 1, cols not a multiple of 64 or of G), CF_E_ALIGN (q, out, k, v or lse
  * misaligned); device-side:
