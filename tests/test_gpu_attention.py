@@ -96,7 +96,9 @@ def codec_step(cf, bits, group, lk, cols, seed):
 
 @pytest.mark.parametrize("bits,group,lq,lk,cols", [(4, 64, 300, 333, 128), (2, 64, 128, 1111, 192),
                                                    (2, 128, 100, 700, 256), (1, 128, 65, 260, 256),
-                                                   (2, 64, 129, 129, 64)])
+                                                   (2, 64, 129, 129, 64), (4, 8, 100, 300, 128),
+                                                   (2, 16, 64, 200, 64), (1, 32, 130, 261, 192),
+                                                   (4, 256, 40, 97, 256)])
 def test_attention_dequantise_matches_decompress_path(cf, oracle, bits, group, lq, lk, cols):
     ctx, before, st = codec_step(cf, bits, group, lk, cols, seed=7)
     q = bf16_rand((lq, cols), 11).cuda()
