@@ -189,6 +189,24 @@ def test_ring_step_merges_two_shards_by_lse(cf, oracle):
     assert np.max(np.abs(lse.numpy() - want_lse)) <= 2e-4
 
 
+def test_attention_large_shard_sampled_rows(cf, oracle):
+    """100,003 keys (past 2^16, ragged against the 128-key blocks) and 70,000
+    queries (274 query blocks): sampled rows of every head and their
+    log-sum-exp against the oracle."""
+    lq, lk, cols = 70000, 100003, 128
+    q, k, v = bf16_rand((lq, cols), 61), bf16_rand((lk, cols), 62), bf16_rand((lk, cols), 63)
+    ctx = cf.Context([], mode=cf.CF_MODE_QUANT)
+    out = torch.empty(lq, cols, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(lq, cols // 64, device="cuda")
+    ctx.attention(q.cuda(), cf.KV(bf16=k.cuda()), cf.KV(bf16=v.cuda()), out, lse=lse)
+    assert ctx.check() == cf.CF_OK
+    rows = [0, 255, 256, 34999, 69887, 69888, 69999]
+    want_out, want_lse = oracle.attention(u16(q[rows]), u16(k), u16(v), cols, lse=True)
+    assert rel_per_head(out[rows].float().cpu().double().numpy(), want_out, cols) <= 1e-2
+    got = lse[rows].cpu().double().numpy()
+    assert np.max(np.abs(got - want_lse) / np.maximum(1.0, np.abs(want_lse))) <= 2e-4
+
+
 def test_attention_is_deterministic(cf):
     lq, lk, cols = 300, 700, 128
     q, k, v = bf16_rand((lq, cols), 21).cuda(), bf16_rand((lk, cols), 22).cuda(), bf16_rand((lk, cols), 23).cuda()
