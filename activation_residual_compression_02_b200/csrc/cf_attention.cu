@@ -29,7 +29,12 @@
 //              blocks, P written to tensor memory in bf16; O rescaled in
 //              TMEM only when a row's running maximum grows by more than 2^8
 //              (otherwise the stale maximum is kept: the normalisation at the
-//              end divides by a sum taken against the same maximum);
+//              end divides by a sum taken against the same maximum).  The two
+//              warps of a sub-partition (one per tile) take turns at the
+//              exponentials, passing the turn halfway through a block, so one
+//              tile's loads and maximum overlap the other's use of the unit.
+//              On request each row's log-sum-exp goes to lse (the weight that
+//              merges partial results over several received blocks);
 //   warp 8(-9) allocates TMEM (S_t: 128 columns each, O_t: 64, P_t: 64) and
 //              issues tcgen05.mma.kind::f16 (bf16 operands, fp32
 //              accumulators): S_t = Q_t K^T from shared memory, then
@@ -48,7 +53,8 @@
 //              MN-major (the channels of a key are contiguous), so no operand
 //              is transposed.
 // Every mbarrier wait is bounded; on expiry the CTA raises an abort flag and
-// the status word's timeout bit, drains its MMAs, frees TMEM and returns.
+// the status word's timeout bit, drains its MMAs, frees TMEM and returns (a
+// test hook, AttnParams::starve, withholds every load to make that happen).
 #include <cuda_bf16.h>
 
 #include <mutex>
