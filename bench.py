@@ -323,6 +323,16 @@ def run_reference(args, w):
     return 0
 
 
+def payload_summary(ctx, w):
+    """What one compressed step sends per rank: the packed codes and scales of
+    every slot (cf_payload_bytes) against the raw bf16 activations, i.e. the
+    communication reduction the pages report (8-16x) for this workload's k and G."""
+    pay = sum(ctx.payload_bytes(s) for s in range(w.slots))
+    raw = w.elems * 2
+    return {"bytes_per_step": pay, "raw_bf16_bytes_per_step": raw, "reduction": raw / pay,
+            "bytes_per_elem": pay / w.elems}
+
+
 def workload_config(w):
     return {
         "workload": f"{w.name}: {w.slots} slots x {w.rows} tokens x {w.cols} channels bf16, k={w.bits}, "
@@ -659,6 +669,7 @@ def run_cf(args, w):
                           "alg_bytes_per_step": (bc + bd) * n_elem},
         "loopback": lb, "lean_state": lean, "recon": rc, "warmup_step": warm,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps,
+        "payload": payload_summary(ctx, w),
         "cogvideox": cog, "stress": stress, "lowrank": lowrank, "attention": attention,
         "clocks": clk.summary(),
     }
@@ -855,6 +866,9 @@ def lowrank_measure(args, w, world, rank, clk, steps, cpu_mats, through_slots=Fa
                      "ms_per_launch": e["ms_per_launch"]} for e in trace],
         "gpu_launches": steps * sum(e["launches_per_call"] for e in trace), "cpu_baseline": cpu,
         "lowrank_mode": lr_mode,
+        # what a step sends per matrix: U (m x r), R (r x r) and V (n x r) in fp32, against the bf16 activation
+        "payload": {"bytes_per_step": k * (m * r + r * r + n * r) * 4, "raw_bf16_bytes_per_step": k * m * n * 2,
+                    "reduction": (m * n * 2) / ((m * r + r * r + n * r) * 4)},
     }
     ctx.close()
     del A, Q0, U, R, V, E, ws
@@ -944,7 +958,7 @@ def quant_extra(args, w, world, rank, clk, steps):
                           "alg_bytes_per_launch": bd * n},
            "roofline_step": {"achieved": pair, "frac": pair / peak, "frac_of_8tbs": pair / 8000.0,
                              "alg_bytes_per_step": (bc + bd) * n},
-           "gpu_launches": 2 * steps}
+           "gpu_launches": 2 * steps, "payload": payload_summary(ctx, w)}
     ctx.close()
     del X, arrs, st
     torch.cuda.empty_cache()
