@@ -642,6 +642,16 @@ try {
         a.codes[i] = t.codes;
         a.scales[i] = t.scales;
     }
+    {
+        // out is written while other CTAs still read K and V (or the caches)
+        const size_t out_bytes = (size_t)lq * (size_t)cols * 2;
+        for (int i = 0; i < 2; ++i) {
+            const void *src = deq ? (const void *)a.cache_in[i] : a.kv[i];
+            const size_t src_bytes = deq ? state_bytes : (size_t)lk * (size_t)cols * 2;
+            if (ranges_overlap(out, out_bytes, src, src_bytes))
+                return fail(ctx, CF_E_ARG, "out must not overlap k or v");
+        }
+    }
     if (deq) {
         // the CTAs of the first query block write C_t while the others still read C_{t-1}
         for (int i = 0; i < 2; ++i)

@@ -284,7 +284,8 @@ typedef struct cf_kv {
  * (failure-detection test hook: CF_TEST_STARVE_ATTENTION=1 in the environment
  * when the context is created makes its first cf_attention call time out).
  * Errors before launch: CF_E_ARG (NULL
- * pointer, mixed forms, overlapping caches, wrong context), CF_E_SHAPE (lk <
+ * pointer, mixed forms, overlapping caches, out overlapping k or v, wrong
+ * context), CF_E_SHAPE (lk <
  * 1, cols not a multiple of 64 or of G), CF_E_ALIGN (q, out, k, v or lse
  * misaligned); device-side:
  * CF_E_TIMEOUT at the next cf_check.

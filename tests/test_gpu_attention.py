@@ -236,6 +236,13 @@ def test_attention_arguments_checked(cf):
         kv = cf.KV(cache_in=c_in, cache_out=c_in, codes=codes, scales=scales)
         ctx.attention(q, kv, kv, out)
     assert e.value.status == cf.CF_E_ARG
+    with pytest.raises(cf.CfError) as e:        # out written over the keys other CTAs still read
+        ctx.attention(q, cf.KV(bf16=k), cf.KV(bf16=k), k[:8 * cols].view(8, cols))
+    assert e.value.status == cf.CF_E_ARG
+    with pytest.raises(cf.CfError) as e:        # ... or over a cache being dequantised
+        kv = cf.KV(cache_in=c_in, codes=codes, scales=scales)
+        ctx.attention(q, kv, kv, c_in[:8 * cols // 2].view(torch.bfloat16).view(8, cols))
+    assert e.value.status == cf.CF_E_ARG
     q96 = torch.zeros(8, 96, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(cf.CfError) as e:        # heads are 64 channels
         ctx.attention(q96, cf.KV(bf16=k[:lk * 96]), cf.KV(bf16=k[:lk * 96]), torch.empty_like(q96))
